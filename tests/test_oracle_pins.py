@@ -1,0 +1,384 @@
+"""Pins of the CPU oracle against what the source pages and the mathematics fix (no GPU).
+
+Each test ties one oracle function to something other than itself: a worked example printed
+by the pages (tests/golden/worked_examples.json, cited there), a closed form, an invariant the
+pages prove, a library special case, or brute force on a tiny layer.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+from oracle import gptq_oracle as O
+
+
+# ---------------------------------------------------------------- P1: the quantizer
+def test_p1_quantizer_example(golden):
+    g = golden["P1_quantizer"]
+    c, q, u = O.quantize(np.array([g["w"]]), np.float32(g["delta"]), np.int64(g["zero"]), g["bits"])
+    assert abs(float(u[0]) - g["u"]) < 1e-6
+    assert int(c[0]) == g["code"]
+    assert abs(float(q[0]) - g["q"]) < 1e-12
+
+
+def test_quantizer_clip_and_half_even():
+    # clip at both ends, and round-half-to-even at exact ties (fp32-representable ties)
+    delta, z = np.float32(0.5), np.int64(2)
+    w = np.array([100.0, -100.0, 0.25, 0.75, -0.25])  # u = 200, -200, 0.5, 1.5, -0.5
+    c, q, _ = O.quantize(w, delta, z, 2)
+    assert list(c) == [3, 0, 2, 4 - 1, 2]  # 0.5->0 (+2), 1.5->2 (+2=4 clipped to 3), -0.5->-0 (+2)
+    assert list(q) == [0.5, -1.0, 0.0, 0.5, 0.0]
+
+
+# ---------------------------------------------------------------- P2: page-1 toy
+def test_p2_toy_two_weights(golden):
+    g = golden["P2_toy_two_weights"]
+    X = np.array(g["X"])
+    # the toy uses H = 2 X X^T (no 1/N): hessian() divides by N=2, so scale back
+    H = O.hessian(X) * X.shape[1]
+    assert np.allclose(H, [[2.08, 0.6], [0.6, 2.5]], atol=1e-12)
+    G = np.linalg.inv(H)
+    tol = 0.5 * 10 ** -g["printed_digits"]
+    assert abs(G[0, 0] - g["Hinv_11"]) <= tol and abs(G[1, 1] - g["Hinv_22"]) <= tol
+    w = np.array(g["w"])
+    grid = np.array(g["grid"])
+    q = grid[np.argmin(np.abs(grid[None, :] - w[:, None]), axis=1)]
+    crit = O.obs_criterion(w - q, np.diag(G))
+    assert abs(crit[0] - g["criterion_w1"]) <= 5e-5 and abs(crit[1] - g["criterion_w2"]) <= 5e-5
+    assert crit[0] < crit[1]  # OBS quantizes w1 first
+    delta = O.obs_update(G, 0, w[0] - q[0])
+    w_new = w + delta
+    assert abs(w_new[0] - q[0]) < 1e-12
+    assert abs(w_new[1] - g["w2_after_compensation"]) <= 5e-4
+    d_before = np.linalg.norm((w - np.array([q[0], w[1]])) @ X)
+    d_after = np.linalg.norm((w - w_new) @ X)
+    assert abs(d_before - g["output_distance_before"]) <= 5e-4
+    assert abs(d_after - g["output_distance_after"]) <= 5e-4
+
+
+# ---------------------------------------------------------------- P3: 2-D update, R form
+def test_p3_two_dim_update(golden):
+    g = golden["P3_two_dim_update"]
+    G = np.array(g["G"])
+    w = np.array(g["w"])
+    rho = w[0] - g["q0"]
+    assert abs(rho - g["rho0"]) < 1e-12
+    w_after = w + O.obs_update(G, 0, rho)
+    assert np.allclose(w_after, g["w_after"], atol=1e-12)
+    # R form (eq.(41)/(42)): the explicit recursion's recorded R rows
+    _, _, _, Rrows = O.gptq_explicit(w[None, :], G, np.array([[0.25]], np.float32),
+                                     np.array([[8]], np.int32), np.array([0, 0]), 4)
+    assert np.allclose(Rrows, g["R"], atol=1e-12)
+    assert np.allclose(Rrows.T @ Rrows, G, atol=1e-12)
+    assert abs(O.downdate(G, 0)[1, 1] - g["next_conditional_G"]) < 1e-12
+
+
+# ---------------------------------------------------------------- P4: downdate counterexample
+def test_p4_downdate(golden):
+    g = golden["P4_downdate_counterexample"]
+    H = np.array(g["H_F"])
+    G = np.linalg.inv(H)
+    assert np.allclose(G, g["G_F"], atol=1e-12)
+    assert abs(G[1, 1] - g["truncation_wrong"]) < 1e-12
+    Gd = O.downdate(G, g["p"])
+    assert abs(Gd[1, 1] - g["downdate_right"]) < 1e-12
+    assert np.allclose(Gd[0, :], 0) and np.allclose(Gd[:, 0], 0)
+    assert abs(Gd[1, 1] - 1.0 / H[1, 1]) < 1e-12  # the inverse of the remaining Hessian
+
+
+def test_downdate_is_inverse_of_submatrix():
+    rng = np.random.default_rng(0)
+    A = rng.standard_normal((7, 12))
+    H = A @ A.T + 0.1 * np.eye(7)
+    G = np.linalg.inv(H)
+    for p in range(7):
+        keep = [i for i in range(7) if i != p]
+        Gd = O.downdate(G, p)
+        assert np.allclose(Gd[np.ix_(keep, keep)], np.linalg.inv(H[np.ix_(keep, keep)]),
+                           rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P5: 3-D block constraint
+def test_p5_three_dim_block(golden):
+    g = golden["P5_three_dim_block"]
+    H = np.array(g["H_F"])
+    delta, dloss, G_T, T = O.block_constraint_solution(np.linalg.inv(H), g["B"], g["a_B"])
+    assert np.allclose(delta, g["delta_star"], atol=1e-12)
+    assert abs(dloss - g["dloss"]) < 1e-12
+    assert abs(G_T[0, 0] - g["G_T"]) < 1e-12
+    # the middle coordinate held at 0 costs more
+    d0 = np.array([-1.0, 0.0, -1.0])
+    assert abs(0.5 * d0 @ H @ d0 - g["cost_if_middle_fixed"]) < 1e-12
+
+
+# ---------------------------------------------------------------- P6: full 2x2 layer
+def test_p6_full_layer(golden):
+    g = golden["P6_full_layer_2x2"]
+    X = np.array(g["X"])
+    W = np.array(g["W"])
+    H = O.hessian(X)
+    assert np.allclose(H, g["H"], atol=1e-12)
+    grid = (np.full((2, 1), g["delta"], np.float32), np.full((2, 1), g["zero"], np.int32))
+    for method in ("explicit", "lazy"):
+        out = O.gptq_layer(W, H, g["bits"], -1, block=1 if method == "lazy" else 128,
+                           percdamp=0.0, eps=0.0, method=method, grid=grid)
+        assert np.allclose(out["G"], g["G"], atol=1e-12)
+        assert out["codes"].tolist() == g["K"]
+        assert np.allclose(out["W_hat"], g["W_hat"], atol=1e-7)
+        # col_loss sums the two rows' per-step losses (each row has the same |rho|)
+        tol = 0.5 * 10 ** -g["step_loss_printed_digits"]
+        assert np.allclose(out["col_loss"] / 2, g["row_step_losses"], atol=tol)
+        le = O.layer_error(W, out["W_hat"], H)
+        assert abs(le - g["layer_error"]) <= 0.5 * 10 ** -g["layer_error_printed_digits"]
+        assert abs(le - O.layer_error_tokens(W, out["W_hat"], X.T)) < 1e-12
+        assert abs(out["col_loss"].sum() - le) < 1e-12  # eq.(67)
+    # first column's compensation, as printed in eq.(59)
+    Wwork = W.copy()
+    rho = Wwork[:, 0] - np.array(g["W_hat"])[:, 0]
+    Wwork += O.obs_update(np.array(g["G"]), 0, rho)
+    assert np.allclose(Wwork, g["W_work_after_col0"], atol=1e-12)
+    # RTN baseline eq.(68)
+    c, q = O.quantize_rtn(W, grid[0], grid[1], 4, -1)
+    assert np.allclose(q, g["rtn_W"], atol=1e-7)
+    assert abs(O.layer_error(W, q, H) - g["rtn_layer_error"]) < 1e-9
+
+
+# ---------------------------------------------------------------- P9: library special cases
+def _spd(d, seed, cond_decay=1e-2):
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((d, 3 * d)) * np.logspace(0, np.log10(cond_decay), d)[:, None]
+    return O.hessian(A)
+
+
+def test_p9_hessian_and_inverse_library():
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((9, 40))
+    assert np.allclose(O.hessian(X), 2.0 / 40 * np.einsum("it,jt->ij", X, X), rtol=1e-13)
+    assert np.allclose(O.hessian_tokens(X.T), O.hessian(X), rtol=1e-13)
+    H = _spd(30, 4)
+    Hl, perm, dead, lam, _ = O.prepare(H, 0.01, False)
+    G, R = O.inverse_and_factor(Hl)
+    assert np.allclose(G, np.linalg.inv(Hl), rtol=1e-9, atol=1e-12)
+    assert np.allclose(R, np.triu(R)) and np.all(np.diag(R) > 0)
+    assert np.allclose(R.T @ R, G, rtol=1e-10, atol=1e-12)
+    assert np.allclose(R, np.linalg.cholesky(np.linalg.inv(Hl)).T, rtol=1e-8, atol=1e-10)
+
+
+def test_p7iv_tail_property_and_eq41_rows():
+    H = _spd(24, 5)
+    Hl, *_ = O.prepare(H, 0.01, False)
+    G, R = O.inverse_and_factor(Hl)
+    for j in [0, 5, 17, 23]:
+        tail = np.linalg.cholesky(np.linalg.inv(Hl[j:, j:])).T
+        assert np.allclose(R[j:, j:], tail, rtol=1e-9, atol=1e-11)  # eq.(40)
+    W = np.random.default_rng(6).standard_normal((3, 24)) * 0.02
+    sc, ze = O.fit_grid(W, 4, -1)
+    _, _, _, Rrows = O.gptq_explicit(W, G, sc, ze, np.zeros(24, int), 4)
+    assert np.allclose(Rrows, R, rtol=1e-9, atol=1e-11)  # eq.(41) rows from explicit downdates
+
+
+# ---------------------------------------------------------------- grid fit
+def test_grid_fit_closed_form():
+    W = np.array([[-0.3, 0.0, 0.45, 0.1], [0.2, 0.4, 0.6, 0.8], [0.0, 0.0, 0.0, 0.0],
+                  [-1.0, -0.5, -0.25, -0.75]], np.float32)
+    sc, ze = O.fit_grid(W, 4, -1)
+    f = np.float32
+    assert sc[0, 0] == (f(0.45) - f(-0.3)) / f(15) and ze[0, 0] == int(np.rint(f(0.3) / sc[0, 0]))
+    assert sc[1, 0] == f(0.8) / f(15) and ze[1, 0] == 0          # range extended down to 0
+    assert sc[2, 0] == 1.0 and ze[2, 0] == 0                      # degenerate range
+    assert sc[3, 0] == f(1.0) / f(15) and ze[3, 0] == 15          # range extended up to 0
+    # every original weight is representable within half a step (no clipping inside the range)
+    for r in range(4):
+        c, q, _ = O.quantize(W[r], sc[r, 0], ze[r, 0], 4)
+        assert np.all(np.abs(q - W[r]) <= sc[r, 0] / 2 + 1e-7)
+
+
+def test_grid_fit_groups_and_tail():
+    rng = np.random.default_rng(7)
+    W = rng.standard_normal((5, 300)).astype(np.float32)
+    sc, ze = O.fit_grid(W, 3, 128)
+    assert sc.shape == (5, 3)
+    for k, (a, b) in enumerate([(0, 128), (128, 256), (256, 300)]):
+        s2, z2 = O.fit_grid(W[:, a:b], 3, -1)
+        assert np.array_equal(sc[:, k], s2[:, 0]) and np.array_equal(ze[:, k], z2[:, 0])
+
+
+# ---------------------------------------------------------------- P7 invariants
+def _layer(m, d, n, seed, bits=4, group=-1, outliers=True):
+    rng = np.random.default_rng(seed)
+    F = rng.standard_normal((d, max(2, d // 3)))
+    X = F @ rng.standard_normal((F.shape[1], n)) + 0.1 * rng.standard_normal((d, n))
+    X *= np.abs(rng.standard_t(3, size=d))[:, None]
+    W = rng.standard_normal((m, d)) * 0.02
+    if outliers:
+        W[:, rng.choice(d, max(1, d // 20), replace=False)] *= 10
+    W = W.astype(np.float16).astype(np.float64)
+    return W, X
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+@pytest.mark.parametrize("group", [-1, 16])
+def test_p7i_lazy_equals_unblocked(act_order, group):
+    W, X = _layer(12, 48, 200, 11)
+    H = O.hessian(X)
+    ref = O.gptq_layer(W, H, 3, group, method="explicit", act_order=act_order)
+    for block in [1, 5, 16, 48, 100]:
+        out = O.gptq_layer(W, H, 3, group, block=block, method="lazy", act_order=act_order)
+        assert np.array_equal(out["codes"], ref["codes"])
+        assert np.allclose(out["W_hat"], ref["W_hat"], atol=1e-12)
+        assert np.allclose(out["col_loss"], ref["col_loss"], rtol=1e-8, atol=1e-14)
+
+
+def test_p7ii_diagonal_hessian_is_rtn():
+    W, _ = _layer(9, 20, 10, 12)
+    H = np.diag(np.random.default_rng(1).uniform(0.5, 2.0, 20))
+    sc, ze = O.fit_grid(W, 4, 8)
+    out = O.gptq_layer(W, H, 4, 8, method="explicit")
+    c, q = O.quantize_rtn(W, sc, ze, 4, 8)
+    assert np.array_equal(out["codes"], c) and np.allclose(out["W_hat"], q)
+
+
+def test_p7iii_loss_identity():
+    W, X = _layer(10, 30, 120, 13)
+    H = O.hessian(X)
+    out = O.gptq_layer(W, H, 3, -1, method="explicit", percdamp=0.02)
+    Hl_orig = np.empty_like(H)
+    p = out["perm"]
+    Hl_orig[np.ix_(p, p)] = out["H_lambda"]
+    dW = W.copy()
+    dW[:, out["dead"]] = 0
+    assert abs(out["col_loss"].sum() - O.layer_error(dW, out["W_hat"], Hl_orig)) < 1e-10
+    # undamped: the recorded losses are the exact layer error (1/N)||ΔW X||^2
+    out0 = O.gptq_layer(W, H, 3, -1, method="explicit", percdamp=0.0, eps=0.0)
+    assert abs(out0["col_loss"].sum() - O.layer_error_tokens(W, out0["W_hat"], X.T)) < 1e-10
+
+
+def test_p7v_act_order_identity_and_equivalence():
+    W, X = _layer(8, 24, 100, 14)
+    H = O.hessian(X)
+    # a Hessian whose diagonal is already descending gives π = identity: same as no act-order
+    order = np.argsort(-np.diag(H), kind="stable")
+    Hs, Ws = H[np.ix_(order, order)], W[:, order]
+    a = O.gptq_layer(Ws, Hs, 4, -1, act_order=True)
+    b = O.gptq_layer(Ws, Hs, 4, -1, act_order=False)
+    assert np.array_equal(a["perm"], np.arange(24))
+    assert np.array_equal(a["codes"], b["codes"])
+    # eq.(35): permuting W's columns and X's rows leaves W X unchanged
+    pi = np.random.default_rng(2).permutation(24)
+    assert np.allclose(W[:, pi] @ X[pi, :], W @ X)
+    # act-order on a permuted problem gives the permuted answer
+    c1 = O.gptq_layer(W, H, 4, -1, act_order=True)
+    c2 = O.gptq_layer(W[:, pi], H[np.ix_(pi, pi)], 4, -1, act_order=True)
+    assert np.array_equal(c1["codes"][:, pi], c2["codes"])
+
+
+def test_p7vi_rows_independent_and_vii_landing():
+    W, X = _layer(12, 20, 80, 15)
+    H = O.hessian(X)
+    full = O.gptq_layer(W, H, 4, -1)
+    rows = [1, 4, 9]
+    sub = O.gptq_layer(W[rows], H, 4, -1, grid=(full["scale"][rows], full["zero"][rows]))
+    assert np.array_equal(sub["codes"], full["codes"][rows])
+    # each column lands exactly on its grid value: Ŵ = Δ (c - z)
+    q = full["scale"][:, [0]] * (full["codes"] - full["zero"][:, [0]])
+    assert np.allclose(full["W_hat"], q, atol=1e-7)
+
+
+def test_dead_features():
+    W, X = _layer(6, 10, 40, 16)
+    X[[2, 7], :] = 0.0
+    H = O.hessian(X)
+    out = O.gptq_layer(W, H, 4, -1)
+    assert out["dead"].tolist() == [j in (2, 7) for j in range(10)]
+    sc, ze = O.fit_grid(W, 4, -1)  # grid fit on the original W (before zeroing)
+    assert np.array_equal(out["scale"], sc)
+    assert np.allclose(out["W_hat"][:, [2, 7]], 0.0) and np.all(out["codes"][:, [2, 7]] == ze)
+
+
+def test_retry_raises_damping():
+    H = np.array([[1.0, 2.0], [2.0, 1.0]])  # indefinite: eigenvalues 3, -1
+    out = O.prepare_with_retry(H, percdamp=0.01)
+    assert out["retries"] >= 2 and abs(out["percdamp"] - 0.01 * 10 ** out["retries"]) < 1e-12
+    with pytest.raises(np.linalg.LinAlgError):
+        O.prepare_with_retry(np.array([[1.0, 0.0], [0.0, -100.0]]), percdamp=0.01)
+
+
+# ---------------------------------------------------------------- block formula ≡ lazy update
+def test_eq32_block_formula_equals_lazy_tail():
+    """eq.(32)/(49): D Γ^{-1} G_BT equals E R_BT for a block of already-chosen grid values."""
+    H = _spd(14, 17)
+    Hl, *_ = O.prepare(H, 0.01, False)
+    G, R = O.inverse_and_factor(Hl)
+    rng = np.random.default_rng(8)
+    Win = rng.standard_normal((4, 14)) * 0.02
+    Bn = 5
+    Wcur = Win.copy()
+    E = np.zeros((4, Bn))
+    Q = np.zeros((4, Bn))
+    for j in range(Bn):
+        Q[:, j] = np.round(Wcur[:, j] / 0.01) * 0.01
+        E[:, j] = (Wcur[:, j] - Q[:, j]) / R[j, j]
+        Wcur[:, j:Bn] -= np.outer(E[:, j], R[j, j:Bn])
+    D = Win[:, :Bn] - Q
+    assert np.allclose(D, E @ R[:Bn, :Bn], atol=1e-13)          # eq.(47)
+    for r in range(4):
+        delta, dloss, _, T = O.block_constraint_solution(G, list(range(Bn)), -D[r])
+        assert np.allclose(Win[r] + delta - (Win[r] - E[r] @ R[:Bn, :]), 0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P8: brute force
+@pytest.mark.parametrize("bits,d,seed", [(2, 1, 0), (2, 4, 1), (3, 4, 2), (2, 6, 3), (3, 5, 4)])
+def test_p8_brute_force(bits, d, seed):
+    rng = np.random.default_rng(100 + seed)
+    n = 3 * d + 2
+    X = rng.standard_normal((d, n)) + 0.5 * rng.standard_normal((1, n))
+    W = (rng.standard_normal((2, d)) * 0.3).astype(np.float16).astype(np.float64)
+    H = O.hessian(X)
+    sc, ze = O.fit_grid(W, bits, -1)
+    out = O.gptq_layer(W, H, bits, -1, percdamp=0.0, eps=0.0, grid=(sc, ze))
+    levels = 2 ** bits
+    for r in range(2):
+        vals = (sc[r, 0] * (np.arange(levels) - ze[r, 0]).astype(np.float32)).astype(np.float64)
+        best = np.inf
+        for combo in itertools.product(range(levels), repeat=d):
+            dw = W[r] - vals[list(combo)]
+            best = min(best, 0.5 * dw @ H @ dw)
+        dw = W[r] - out["W_hat"][r]
+        gptq_obj = 0.5 * dw @ H @ dw
+        assert best <= gptq_obj + 1e-12
+        if d == 1:
+            assert abs(best - gptq_obj) < 1e-12
+        # the last column's choice is the conditional optimum given the earlier codes
+        cand = [0.5 * (W[r] - np.r_[out["W_hat"][r, :-1], v]) @ H @ (W[r] - np.r_[out["W_hat"][r, :-1], v])
+                for v in vals]
+        assert abs(min(cand) - gptq_obj) < 1e-12
+
+
+# ---------------------------------------------------------------- decision replay
+def test_decision_replay_accepts_self_and_flags_planted_mistake():
+    W, X = _layer(16, 40, 160, 18)
+    H = O.hessian(X)
+    out = O.gptq_layer(W, H, 4, 8, method="lazy", block=8)
+    codes_p = out["codes"][:, out["perm"]]
+    rep = O.decision_replay(out["Wp"], out["R"], out["scale"], out["zero"], out["gcol"], 4, codes_p)
+    assert rep["identical"] == rep["n"] and rep["violations"] == 0
+    bad = codes_p.copy()
+    bad[3, 10] = (bad[3, 10] + 2) % 16
+    rep = O.decision_replay(out["Wp"], out["R"], out["scale"], out["zero"], out["gcol"], 4, bad)
+    assert rep["violations"] >= 1
+
+
+# ---------------------------------------------------------------- packing
+def test_pack_layout_definition():
+    codes = np.array([[1, 2, 3, 4, 5, 6, 7, 8, 9]])
+    p = O.pack(codes, 4)
+    assert p.shape == (1, 2) and p[0, 0] == 0x87654321 and p[0, 1] == 0x9
+    codes3 = np.array([[7, 0, 5] + [0] * 7 + [6, 3]])   # 12 codes, 36 bits -> 2 words
+    p3 = O.pack(codes3, 3)
+    assert p3[0, 0] == (7 | (5 << 6) | (6 << 30)) & 0xFFFFFFFF
+    assert p3[0, 1] == ((6 >> 2) | (3 << 1))
+    rng = np.random.default_rng(9)
+    for bits in (2, 3, 4, 8):
+        c = rng.integers(0, 2 ** bits, size=(3, 37))
+        assert np.array_equal(O.unpack(O.pack(c, bits), 37, bits), c)
+        assert O.pack(c, bits).shape[1] == O.words_per_row(37, bits)
