@@ -1,0 +1,149 @@
+/*
+ * gptq.h — C ABI of the B200 (sm_100a) GPTQ layer-quantization library (libgptq_b200.so).
+ *
+ * The library computes GPTQ's per-layer hot path: the Hessian H = 2 X X^T / N of the
+ * calibration activations, its damped inverse in upper-Cholesky form R (R^T R = H_λ^{-1}),
+ * the column-by-column quantization of W to a fixed affine grid with lazy block error
+ * feedback, and the dense bit-packing of the integer codes.
+ *
+ * Sources, cited by page title and section / equation:
+ *   [T] "GPTQ 从零推导：4-bit 权重量化为什么能‘量化一列，补偿一列’" (hbblog.cn derivation tutorial)
+ *   [W] "GPTQ 完全拆解：二阶信息驱动的权重量化，如何把 175B 模型塞进一张 A100" (pinghaoyang.com.cn)
+ *
+ * Conventions shared by every entry point
+ *   - Every array argument is a DEVICE pointer owned by the caller, unless the parameter
+ *     says "host".  The library never frees caller memory.
+ *   - Matrices are dense and row-major with the row stride equal to their column count.
+ *   - Work is enqueued asynchronously on the context's CUDA stream.  Only
+ *     gptq_prepare_hinv and gptq_sync_status synchronize that stream.
+ *   - Argument errors return GPTQ_ERR_ARG before anything is enqueued.  Errors found on
+ *     the device (non-finite input, non-positive-definite matrix, a bounded wait that ran
+ *     out) are recorded in a device status word and returned by the next
+ *     gptq_sync_status (or by gptq_prepare_hinv, which synchronizes).
+ *   - Scratch memory comes from the workspace given to gptq_create; a call whose needs
+ *     exceed it returns GPTQ_ERR_NOMEM without enqueuing work.
+ *   - gptq_last_error(ctx) describes the most recent host-side failure.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct gptq_ctx gptq_ctx;
+
+/* Status codes. */
+enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_ARG = 1,        /* invalid argument (nothing enqueued) */
+  GPTQ_ERR_CUDA = 2,       /* a CUDA runtime call or launch failed */
+  GPTQ_ERR_NOT_PD = 3,     /* H_λ not positive definite after the damping retries */
+  GPTQ_ERR_NONFINITE = 4,  /* NaN/Inf in X, H or W */
+  GPTQ_ERR_TIMEOUT = 5,    /* a bounded on-device wait gave up */
+  GPTQ_ERR_NOMEM = 6       /* workspace too small */
+};
+
+/* Element types of X and W. */
+enum { GPTQ_BF16 = 0, GPTQ_F16 = 1, GPTQ_F32 = 2 };
+
+/* Workspace bytes that gptq_prepare_hinv and gptq_quantize_layer need for a layer with m
+ * output rows and d input columns (the larger of the two, plus the status block).  Pure
+ * host function. */
+size_t gptq_workspace_bytes(int64_t m, int64_t d, int act_order);
+
+/* Creates a context bound to the current CUDA device and to `cuda_stream` (a cudaStream_t;
+ * NULL = legacy default stream).  `workspace` is a caller-owned device buffer of
+ * `workspace_bytes` bytes (>= 256); if `workspace` is NULL the library allocates
+ * `workspace_bytes` itself and frees them in gptq_destroy.  The first 256 bytes hold the
+ * device status word.  Returns GPTQ_OK, GPTQ_ERR_ARG or GPTQ_ERR_CUDA. */
+int gptq_create(gptq_ctx** ctx, void* cuda_stream, void* workspace, size_t workspace_bytes);
+
+/* Releases the context (and the workspace if the library allocated it). */
+int gptq_destroy(gptq_ctx* ctx);
+
+/* Text of the most recent host-side error on this context ("" if none).  Owned by ctx. */
+const char* gptq_last_error(const gptq_ctx* ctx);
+
+/* Number of kernels this context has launched so far (a host-side counter; no sync). */
+uint64_t gptq_kernel_launches(const gptq_ctx* ctx);
+
+/* Synchronizes the context stream, returns and clears the device status word
+ * (GPTQ_OK, GPTQ_ERR_NONFINITE, GPTQ_ERR_NOT_PD or GPTQ_ERR_TIMEOUT), or GPTQ_ERR_CUDA. */
+int gptq_sync_status(gptq_ctx* ctx);
+
+/* Hessian statistic, [T] §2.1 eq.(5) and §2.4 eq.(9); accumulated in batches as [T] §9.4
+ * allows.  Computes S += Xc^T Xc for one token chunk:
+ *   Xc      [n_chunk, d] token-major activations (row t = token t's input vector), of type
+ *           `dtype` (GPTQ_BF16 / GPTQ_F16: tensor-core path, products exact in fp32;
+ *           GPTQ_F32: CUDA-core fp32 path).
+ *   S       [d, d] fp32.  Only the lower triangle (i >= j) is defined on return.
+ *   n_total host int64: tokens accumulated so far.  If *n_total == 0, S is overwritten
+ *           (not read); afterwards *n_total += n_chunk.
+ * Then H = 2 S / n_total.  Errors: ARG (d < 1, n_chunk < 1, bad dtype, NULL pointers). */
+int gptq_hessian_accumulate(gptq_ctx* ctx, const void* Xc, int dtype, int64_t n_chunk,
+                            int64_t d, float* S, int64_t* n_total);
+
+/* Preconditioning and inverse factor, [T] §10 (order: dead features, act-order permutation,
+ * damping), eq.(12), §8.3 eq.(34), §9.1 eq.(37)-(40).
+ *   S        [d, d] fp32, lower triangle read: the unnormalised statistic with
+ *            H = 2 S / n_total when n_total > 0, or H itself when n_total <= 0.
+ *            Overwritten with the permuted, normalised, undamped H' = Π H Π^T.
+ *   percdamp damping ratio: λ = max(percdamp * mean(diag H'), 2^-23).
+ *   act_order 0: π = identity; 1: π = stable argsort of diag(H) descending.
+ *   R        [d, d] fp32 out: upper-triangular factor with R^T R = H_λ^{-1} and a positive
+ *            diagonal, in processing order (strictly lower part set to 0).
+ *   perm     [d] int32 out: perm[j] = original column processed at position j.
+ *   dead     [d] uint8 out: 1 where diag(H) == 0 (original column order); such diagonal
+ *            entries are replaced by 1 before damping.
+ *   damp_used host float* (may be NULL): the λ finally used.
+ *   retries  host int* (may be NULL): how many times percdamp was multiplied by 10 after a
+ *            failed factorization ([T] §10 remark; at most 3).
+ * Synchronizes the stream.  Errors: ARG, NOMEM, NONFINITE (non-finite diag of S),
+ * NOT_PD (still not positive definite after 3 retries), CUDA. */
+int gptq_prepare_hinv(gptq_ctx* ctx, float* S, int64_t n_total, int64_t d, float percdamp,
+                      int act_order, float* R, int32_t* perm, uint8_t* dead,
+                      float* damp_used, int* retries);
+
+/* Column-by-column quantization with lazy block updates, [W] Algorithm 1, [T] §9.2-9.3
+ * eq.(42)-(46) and §10; quantizer [T] eq.(36); static groups [T] §8.3.
+ *   W        [m, d] weights of type w_dtype (GPTQ_F16 / GPTQ_BF16 / GPTQ_F32), ORIGINAL
+ *            column order; not modified.
+ *   R, perm, dead  as produced by gptq_prepare_hinv for this layer's H.
+ *   bits     1..8 (2, 3, 4 are the pages' cases); codes lie in 0 .. 2^bits - 1.
+ *   group    -1 (one grid per row) or > 0 (one grid per `group` original columns; the last
+ *            group may be shorter).  n_g = 1 or ceil(d / group).
+ *   block    lazy block size B >= 1.  Blocks of up to 128 columns are run as given; a larger
+ *            B is run as 128-column blocks, which gives the same result in exact arithmetic
+ *            ([T] eq.(47)-(49)).
+ *   grid_given 0: fit a min-max grid on the original W (range extended to contain 0,
+ *            Δ = (max - min) / (2^b - 1), z = clip(rint(-min / Δ)); all-zero range -> Δ = 1)
+ *            and write it to scales/zeros; 1: read scales/zeros as the fixed grid.
+ *   scales   [m, n_g] fp32, zeros [m, n_g] int32 (in or out, see grid_given).
+ *   codes    [m, d] uint8 out, W_hat [m, d] fp32 out (= Δ (c - z)), col_loss [d] fp32 out
+ *            (Σ_rows ρ² / (2 R_jj²), [T] eq.(43)); all in ORIGINAL column order.
+ * Asynchronous.  Errors: ARG, NOMEM; NONFINITE (W) via gptq_sync_status. */
+int gptq_quantize_layer(gptq_ctx* ctx, const void* W, int w_dtype, int64_t m, int64_t d,
+                        const float* R, const int32_t* perm, const uint8_t* dead, int bits,
+                        int group, int block, int grid_given, float* scales, int32_t* zeros,
+                        uint8_t* codes, float* W_hat, float* col_loss);
+
+/* Dense packing of the codes ([T] §3.1 output table, §9.4: about m d b / 8 bytes, stored as
+ * 32-bit words).  Layout: per row a little-endian bitstream in which code k occupies bits
+ * [b k, b k + b); word w of the row holds stream bits [32 w, 32 w + 32); every row starts on
+ * a new word.  codes [m, d] uint8 (values < 2^bits) -> packed [m, ceil(d bits / 32)] uint32.
+ * Asynchronous.  Errors: ARG. */
+int gptq_pack(gptq_ctx* ctx, const uint8_t* codes, int64_t m, int64_t d, int bits,
+              uint32_t* packed);
+
+/* Inverse of gptq_pack. */
+int gptq_unpack(gptq_ctx* ctx, const uint32_t* packed, int64_t m, int64_t d, int bits,
+                uint8_t* codes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTQ_B200_H */

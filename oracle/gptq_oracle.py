@@ -117,7 +117,8 @@ def quantize_rtn(W, scale, zero, bits: int, group: int):
 # --------------------------------------------------------------------------------------------
 # Preconditioning: dead features, act-order, damping, inverse and its Cholesky factor
 # --------------------------------------------------------------------------------------------
-def prepare(H, percdamp: float = 0.01, act_order: bool = False, eps: float = FP32_EPS):
+def prepare(H, percdamp: float = 0.01, act_order: bool = False, eps: float = FP32_EPS,
+            perm=None):
     """The preparation steps of [T] §10 in its order: dead features, then the processing
     permutation, then damping.
 
@@ -126,6 +127,10 @@ def prepare(H, percdamp: float = 0.01, act_order: bool = False, eps: float = FP3
       H' = Π H Π^T  ([T] §8.3 eq.(34));
     * damping: λ = max(percdamp * mean(diag H'), eps), H_λ = H' + λ I  ([T] eq.(12), §10).
 
+    `perm` (optional) imposes a processing order instead of computing it; callers use it to
+    replay another implementation's act-order permutation after checking that it is a valid
+    descending order of diag(H) (near-ties may be ordered either way).
+
     Returns (H_lambda, perm, dead, lam, H_perm_undamped).
     """
     H = np.array(H, dtype=np.float64, copy=True)
@@ -133,7 +138,9 @@ def prepare(H, percdamp: float = 0.01, act_order: bool = False, eps: float = FP3
     dead = np.diag(H) == 0.0
     idx = np.nonzero(dead)[0]
     H[idx, idx] = 1.0
-    if act_order:
+    if perm is not None:
+        perm = np.asarray(perm, dtype=np.int64)
+    elif act_order:
         perm = np.argsort(-np.diag(H), kind="stable")
     else:
         perm = np.arange(d)
@@ -156,15 +163,15 @@ def inverse_and_factor(H_lambda):
 
 
 def prepare_with_retry(H, percdamp: float = 0.01, act_order: bool = False,
-                       eps: float = FP32_EPS, max_retries: int = 3):
+                       eps: float = FP32_EPS, max_retries: int = 3, perm=None):
     """[T] §10 remark: on a failed Cholesky raise the damping and retry.  Reading: percdamp is
     multiplied by 10 per retry, at most `max_retries` times."""
     pd = percdamp
     for attempt in range(max_retries + 1):
-        Hl, perm, dead, lam, Hp = prepare(H, pd, act_order, eps)
+        Hl, order, dead, lam, Hp = prepare(H, pd, act_order, eps, perm)
         try:
             G, R = inverse_and_factor(Hl)
-            return dict(H_lambda=Hl, H_perm=Hp, perm=perm, dead=dead, lam=lam, G=G, R=R,
+            return dict(H_lambda=Hl, H_perm=Hp, perm=order, dead=dead, lam=lam, G=G, R=R,
                         retries=attempt, percdamp=pd)
         except np.linalg.LinAlgError:
             pd *= 10.0
@@ -342,7 +349,7 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
 # --------------------------------------------------------------------------------------------
 def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 0.01,
                act_order: bool = False, method: str = "explicit", grid=None,
-               eps: float = FP32_EPS):
+               eps: float = FP32_EPS, perm=None):
     """The layer-wise hot path of [T] §10, end to end on one layer.
 
     1. grid: fitted on the original W before anything else (static groups), unless given;
@@ -360,7 +367,7 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
         scale, zero = fit_grid(W, bits, group)
     else:
         scale, zero = (np.asarray(grid[0], np.float32), np.asarray(grid[1], np.int32))
-    prep = prepare_with_retry(H, percdamp, act_order, eps)
+    prep = prepare_with_retry(H, percdamp, act_order, eps, perm=perm)
     perm, dead = prep["perm"], prep["dead"]
     Wwork = W.copy()
     Wwork[:, dead] = 0.0
@@ -381,6 +388,19 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     return dict(codes=codes, W_hat=W_hat, scale=scale, zero=zero, col_loss=col_loss,
                 perm=perm, dead=dead, lam=prep["lam"], G=prep["G"], R=prep["R"],
                 H_lambda=prep["H_lambda"], retries=prep["retries"], Wp=Wp, gcol=gcol)
+
+
+def is_valid_act_order(perm, H, rtol: float = 1e-5) -> bool:
+    """True if `perm` lists the columns by descending diag(H) (dead entries counted as 1), up to
+    ties within `rtol` relative: the decision taken in another precision may order near-ties
+    differently ([T] §8.3: act-order is a heuristic over diag(H))."""
+    diag = np.array(np.diag(np.asarray(H, np.float64)), copy=True)
+    diag[diag == 0.0] = 1.0
+    perm = np.asarray(perm, np.int64)
+    if sorted(perm.tolist()) != list(range(len(diag))):
+        return False
+    v = diag[perm]
+    return bool(np.all(v[1:] <= v[:-1] * (1.0 + rtol) + 1e-30))
 
 
 def layer_error(W, W_hat, H):

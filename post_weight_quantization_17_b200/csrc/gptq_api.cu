@@ -1,0 +1,241 @@
+// C ABI of the library (declared and documented in include/gptq.h).
+#include <algorithm>
+#include <new>
+
+#include "kernels.h"
+
+struct gptq_ctx {
+  gptq::Ctx c;
+};
+
+using gptq::Carver;
+using gptq::Ctx;
+
+namespace {
+
+inline bool valid_dtype(int t) { return t == GPTQ_BF16 || t == GPTQ_F16 || t == GPTQ_F32; }
+
+size_t prep_bytes(int64_t d) {
+  size_t b = gptq::kStatusBytes + 256 * 4;
+  b += d * sizeof(float);
+  b += gptq::factor_tmp_floats((int)d) * sizeof(float);
+  return b;
+}
+
+size_t quant_bytes(int64_t m, int64_t d, bool general_perm) {
+  size_t b = gptq::kStatusBytes + 256 * 10;
+  b += 2 * d * sizeof(int32_t);                                  // gcol, inv
+  b += (size_t)m * gptq::kColMax * sizeof(float);                // E
+  b += (size_t)((m + gptq::kColRows - 1) / gptq::kColRows) * d * sizeof(float);  // loss parts
+  b += d * sizeof(float);                                        // loss in processing order
+  if (general_perm) b += (size_t)m * d * (sizeof(float) + 1);    // W_work, codes (permuted)
+  return b;
+}
+
+int read_status(Ctx* c, gptq::DeviceStatus* out) {
+  GPTQ_CUDA_CHECK(c, cudaMemcpyAsync(out, c->status, sizeof(*out), cudaMemcpyDeviceToHost,
+                                     c->stream));
+  GPTQ_CUDA_CHECK(c, cudaStreamSynchronize(c->stream));
+  return GPTQ_OK;
+}
+
+int clear_status(Ctx* c) {
+  GPTQ_CUDA_CHECK(c, cudaMemsetAsync(c->status, 0, sizeof(gptq::DeviceStatus), c->stream));
+  return GPTQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gptq_workspace_bytes(int64_t m, int64_t d, int act_order) {
+  if (m < 1 || d < 1) return gptq::kStatusBytes;
+  return std::max(prep_bytes(d), quant_bytes(m, d, act_order != 0));
+}
+
+int gptq_create(gptq_ctx** out, void* stream, void* workspace, size_t workspace_bytes) {
+  if (!out || workspace_bytes < gptq::kStatusBytes) return GPTQ_ERR_ARG;
+  *out = nullptr;
+  gptq_ctx* h = new (std::nothrow) gptq_ctx();
+  if (!h) return GPTQ_ERR_NOMEM;
+  Ctx* c = &h->c;
+  c->stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  if (e == cudaSuccess && !workspace) {
+    void* p = nullptr;
+    e = cudaMalloc(&p, workspace_bytes);
+    workspace = p;
+    c->owns_ws = (e == cudaSuccess);
+  }
+  if (e != cudaSuccess) {
+    delete h;
+    return GPTQ_ERR_CUDA;
+  }
+  c->ws = reinterpret_cast<char*>(workspace);
+  c->ws_bytes = workspace_bytes;
+  c->status = reinterpret_cast<gptq::DeviceStatus*>(c->ws);
+  if (clear_status(c) != GPTQ_OK || cudaStreamSynchronize(c->stream) != cudaSuccess) {
+    if (c->owns_ws) cudaFree(c->ws);
+    delete h;
+    return GPTQ_ERR_CUDA;
+  }
+  *out = h;
+  return GPTQ_OK;
+}
+
+int gptq_destroy(gptq_ctx* h) {
+  if (!h) return GPTQ_ERR_ARG;
+  if (h->c.owns_ws) cudaFree(h->c.ws);
+  delete h;
+  return GPTQ_OK;
+}
+
+const char* gptq_last_error(const gptq_ctx* h) { return h ? h->c.last_error.c_str() : ""; }
+
+uint64_t gptq_kernel_launches(const gptq_ctx* h) { return h ? h->c.launches : 0; }
+
+int gptq_sync_status(gptq_ctx* h) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  gptq::DeviceStatus st{};
+  int rc = read_status(c, &st);
+  if (rc) return rc;
+  if (st.code) {
+    c->last_error = "device status " + std::to_string(st.code) + " at " + std::to_string(st.where);
+    if ((rc = clear_status(c))) return rc;
+    return st.code;
+  }
+  return GPTQ_OK;
+}
+
+int gptq_hessian_accumulate(gptq_ctx* h, const void* Xc, int dtype, int64_t n_chunk, int64_t d,
+                            float* S, int64_t* n_total) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!Xc || !S || !n_total || !valid_dtype(dtype) || d < 1 || d > (1 << 20) || n_chunk < 1 ||
+      n_chunk > INT32_MAX || *n_total < 0)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "hessian_accumulate: bad argument (d=%lld n_chunk=%lld)",
+                 (long long)d, (long long)n_chunk);
+  int rc = gptq::syrk_accumulate(c, Xc, dtype, n_chunk, (int)d, S, *n_total == 0);
+  if (rc) return rc;
+  *n_total += n_chunk;
+  return GPTQ_OK;
+}
+
+int gptq_prepare_hinv(gptq_ctx* h, float* S, int64_t n_total, int64_t d, float percdamp,
+                      int act_order, float* R, int32_t* perm, uint8_t* dead, float* damp_used,
+                      int* retries) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!S || !R || !perm || !dead || d < 1 || d > 65535 || !(percdamp >= 0.f) || S == R)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "prepare_hinv: bad argument (d=%lld)", (long long)d);
+  Carver cv(c);
+  float* diagv = cv.take<float>(d);
+  float* tmp = cv.take<float>(gptq::factor_tmp_floats((int)d));
+  if (!cv.ok())
+    GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "prepare_hinv: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
+  const int di = (int)d;
+  const float scale = n_total > 0 ? (float)(2.0 / (double)n_total) : 1.f;
+  const size_t dd = (size_t)d * d;
+  int rc;
+  if ((rc = gptq::prep_diag(c, S, di, scale, diagv, dead))) return rc;
+  if ((rc = gptq::prep_mean(c, diagv, di))) return rc;
+  if ((rc = gptq::prep_perm(c, diagv, di, act_order, perm))) return rc;
+  if ((rc = gptq::prep_build(c, S, di, scale, diagv, perm, !act_order, R))) return rc;
+  if ((rc = gptq::prep_copy(c, R, S, dd))) return rc;
+  float pd = percdamp;
+  for (int attempt = 0; attempt <= 3; ++attempt) {
+    if (attempt > 0 && (rc = gptq::prep_copy(c, S, R, dd))) return rc;
+    if ((rc = gptq::prep_damp(c, R, di, pd))) return rc;
+    if ((rc = gptq::factor_inverse(c, R, di, tmp))) return rc;
+    gptq::DeviceStatus st{};
+    if ((rc = read_status(c, &st))) return rc;
+    if (st.code == 0) {
+      if (damp_used) *damp_used = st.lam;
+      if (retries) *retries = attempt;
+      return GPTQ_OK;
+    }
+    if ((rc = clear_status(c))) return rc;
+    if (st.code != GPTQ_ERR_NOT_PD) {
+      c->last_error = "prepare_hinv: device status " + std::to_string(st.code) + " at " +
+                      std::to_string(st.where);
+      return st.code;
+    }
+    pd *= 10.f;
+  }
+  if (retries) *retries = 3;
+  GPTQ_SET_ERR(c, GPTQ_ERR_NOT_PD, "prepare_hinv: H not positive definite after 3 retries");
+}
+
+int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int64_t d,
+                        const float* R, const int32_t* perm, const uint8_t* dead, int bits,
+                        int group, int block, int grid_given, float* scales, int32_t* zeros,
+                        uint8_t* codes, float* W_hat, float* col_loss) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!W || !R || !scales || !zeros || !codes || !W_hat || !col_loss || !valid_dtype(w_dtype) ||
+      m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || (long long)m * d > (1LL << 40) ||
+      bits < 1 || bits > 8 || !(group == -1 || group > 0) || block < 1)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "quantize_layer: bad argument (m=%lld d=%lld bits=%d group=%d block=%d)",
+                 (long long)m, (long long)d, bits, group, block);
+  const int mi = (int)m, di = (int)d;
+  const bool general = perm != nullptr;
+  const int g = (group == -1) ? di : group;
+  const int ng = (di + g - 1) / g;
+  const int parts = (mi + gptq::kColRows - 1) / gptq::kColRows;
+  Carver cv(c);
+  int32_t* gcol = cv.take<int32_t>(d);
+  int32_t* inv = cv.take<int32_t>(d);
+  float* E = cv.take<float>((size_t)m * gptq::kColMax);
+  float* loss_part = cv.take<float>((size_t)parts * d);
+  float* loss_p = cv.take<float>(d);
+  float* Wk = W_hat;
+  uint8_t* codes_p = codes;
+  if (general) {
+    Wk = cv.take<float>((size_t)m * d);
+    codes_p = cv.take<uint8_t>((size_t)m * d);
+  }
+  if (!cv.ok())
+    GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "quantize_layer: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
+  int rc;
+  if (!grid_given && (rc = gptq::grid_fit(c, W, w_dtype, mi, di, bits, group, scales, zeros)))
+    return rc;
+  if ((rc = gptq::make_gcol(c, perm, di, group, gcol, general ? inv : nullptr))) return rc;
+  if ((rc = gptq::init_work(c, W, w_dtype, mi, di, perm, dead, !general, Wk))) return rc;
+  const int bk = std::min(block, gptq::kColMax);
+  for (int i = 0; i < di; i += bk) {
+    const int nb = std::min(bk, di - i);
+    const bool uniform = (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
+    if ((rc = gptq::column_block(c, Wk, mi, di, i, nb, R, scales, zeros, ng, gcol, uniform, bits,
+                                 E, codes_p, loss_part)))
+      return rc;
+    if ((rc = gptq::trailing_update(c, Wk, mi, di, i, nb, E, R))) return rc;
+  }
+  if ((rc = gptq::loss_reduce(c, loss_part, parts, di, general ? loss_p : col_loss))) return rc;
+  if (general &&
+      (rc = gptq::unpermute(c, mi, di, inv, codes_p, Wk, loss_p, codes, W_hat, col_loss)))
+    return rc;
+  return GPTQ_OK;
+}
+
+int gptq_pack(gptq_ctx* h, const uint8_t* codes, int64_t m, int64_t d, int bits,
+              uint32_t* packed) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!codes || !packed || m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || bits < 1 || bits > 8)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "pack: bad argument");
+  return gptq::pack_codes(c, codes, (int)m, (int)d, bits, packed);
+}
+
+int gptq_unpack(gptq_ctx* h, const uint32_t* packed, int64_t m, int64_t d, int bits,
+                uint8_t* codes) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!codes || !packed || m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || bits < 1 || bits > 8)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "unpack: bad argument");
+  return gptq::unpack_codes(c, packed, (int)m, (int)d, bits, codes);
+}
+
+}  // extern "C"

@@ -1,0 +1,329 @@
+// a4-a7: grid fit, working copy, in-block column quantization, lazy trailing update,
+// per-column loss, un-permute.
+//
+// [W] Algorithm 1 and [T] §9.2-§9.3, §10: for each block [i, i+nb) of processing positions,
+// each column j is quantized (c = clip(rint(w/Δ)+z), q = Δ(c-z), [T] eq.(36)), its scaled
+// residual η = (w - q) / R_jj is kept in E, the block's remaining columns receive
+// w_k -= η R_jk immediately (eq.(42)), and after the block the rest of W receives
+// W[:, i+nb:] -= E R[i:i+nb, i+nb:] (eq.(46)).
+#include "kernels.h"
+#include "gemm_simt.cuh"
+
+#include <utility>
+
+namespace gptq {
+
+// ------------------------------------------------------------------------------------------
+// a4: static min-max grid per (row, group of original columns), [T] §1.1 and §8.3.
+// One warp per (row, group); the range is extended to contain 0; fp32 arithmetic.
+template <class T>
+__global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, int bits,
+                          float* __restrict__ scales, int32_t* __restrict__ zeros,
+                          DeviceStatus* st) {
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= (long long)m * ng) return;
+  const int r = (int)(warp / ng), k = (int)(warp % ng);
+  const int c0 = k * g, c1 = min(d, c0 + g);
+  float mn = 0.f, mx = 0.f;
+  bool bad = false;
+  const T* row = W + (long long)r * d;
+  for (int cc = c0 + lane; cc < c1; cc += 32) {
+    float v = to_f32<T>(row[cc]);
+    bad |= !isfinite(v);
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (lane == 0) {
+    if (bad) raise_error(st, GPTQ_ERR_NONFINITE, r);
+    const float maxq = (float)((1 << bits) - 1);
+    float delta = (mx == mn) ? 1.f : __fdiv_rn(__fsub_rn(mx, mn), maxq);
+    float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, delta)), 0.f), maxq);
+    scales[(long long)r * ng + k] = delta;
+    zeros[(long long)r * ng + k] = (int32_t)z;
+  }
+}
+
+int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int group,
+             float* scales, int32_t* zeros) {
+  const int g = (group == -1) ? d : group;
+  const int ng = (d + g - 1) / g;
+  const long long warps = (long long)m * ng;
+  const int blocks = (int)((warps * 32 + 255) / 256);
+  if (w_dtype == GPTQ_F16)
+    k_gridfit<__half><<<blocks, 256, 0, c->stream>>>((const __half*)W, m, d, g, ng, bits, scales, zeros, c->status);
+  else if (w_dtype == GPTQ_BF16)
+    k_gridfit<__nv_bfloat16><<<blocks, 256, 0, c->stream>>>((const __nv_bfloat16*)W, m, d, g, ng, bits, scales, zeros, c->status);
+  else
+    k_gridfit<float><<<blocks, 256, 0, c->stream>>>((const float*)W, m, d, g, ng, bits, scales, zeros, c->status);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
+
+// grid index of each processing position (static groups: floor(π_j / g)) and the inverse
+// permutation.
+__global__ void k_gcol(const int32_t* __restrict__ perm, int d, int group,
+                       int32_t* __restrict__ gcol, int32_t* __restrict__ inv) {
+  int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  int p = perm ? perm[j] : j;
+  gcol[j] = (group == -1) ? 0 : p / group;
+  if (inv) inv[p] = j;
+}
+
+int make_gcol(Ctx* c, const int32_t* perm, int d, int group, int32_t* gcol, int32_t* inv) {
+  k_gcol<<<(d + 255) / 256, 256, 0, c->stream>>>(perm, d, group, gcol, inv);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
+
+// working copy in processing order: Wk[r][j] = dead[π_j] ? 0 : W[r][π_j]  ([T] §10)
+template <class T>
+__global__ void k_init_work(const T* __restrict__ W, long long m, int d,
+                            const int32_t* __restrict__ perm, const uint8_t* __restrict__ dead,
+                            float* __restrict__ Wk) {
+  const long long total = m * d;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    long long r = e / d;
+    int j = (int)(e - r * d);
+    int src = perm ? perm[j] : j;
+    float v = to_f32<T>(W[r * d + src]);
+    if (dead && dead[src]) v = 0.f;
+    Wk[e] = v;
+  }
+}
+
+int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* perm,
+              const uint8_t* dead, bool, float* Wk) {
+  const long long total = (long long)m * d;
+  int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
+  if (w_dtype == GPTQ_F16)
+    k_init_work<__half><<<blocks, 256, 0, c->stream>>>((const __half*)W, m, d, perm, dead, Wk);
+  else if (w_dtype == GPTQ_BF16)
+    k_init_work<__nv_bfloat16><<<blocks, 256, 0, c->stream>>>((const __nv_bfloat16*)W, m, d, perm, dead, Wk);
+  else
+    k_init_work<float><<<blocks, 256, 0, c->stream>>>((const float*)W, m, d, perm, dead, Wk);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// a5: one block of up to 128 columns.  One warp per CTA, one row per lane: the lane keeps its
+// row's block in 128 registers, so the sequential chain of a column step (divide, round,
+// clip, residual, η, update of the next column) stays inside the lane.  R's diagonal block
+// is read from shared memory as warp-wide broadcasts.  Global traffic is staged through
+// shared memory so that every global access is a coalesced row segment.
+// Shared memory: R block (64 KB), W/E staging (32 x 129 floats), q staging, code staging.
+constexpr int kColSmem = 128 * 128 * 4 + 2 * 32 * 129 * 4 + 32 * 132;
+
+struct ColStepArgs {
+  const float (*Rs)[128];
+  float (*St)[129];
+  uint8_t (*Cs)[132];
+  const int* gs;
+  const float* rinv;
+  const float* scales;
+  const int32_t* zeros;
+  long long srow;  // row * ng
+  int lane, nb;
+  bool active;
+  float maxq, D0, Z0;
+};
+
+// One column step; block column OFF + J, with J compile-time so that w[] stays in registers.
+// Only the columns of the same half (J+1 .. 63) are updated immediately.
+template <int J, int OFF, bool UNIFORM>
+__device__ __forceinline__ void col_step(float (&w)[64], const ColStepArgs& a) {
+  constexpr int C = OFF + J;
+  if (C < a.nb) {
+    float Dj = a.D0, Zj = a.Z0;
+    if (!UNIFORM && a.active) {
+      const int gj = a.gs[C];
+      Dj = a.scales[a.srow + gj];
+      Zj = (float)a.zeros[a.srow + gj];
+    }
+    const float u = __fdiv_rn(w[J], Dj);
+    const float cq = fminf(fmaxf(rintf(u) + Zj, 0.f), a.maxq);
+    const float q = __fmul_rn(Dj, cq - Zj);
+    const float eta = __fmul_rn(__fsub_rn(w[J], q), a.rinv[C]);
+    a.Cs[a.lane][C] = (uint8_t)cq;
+    a.St[a.lane][C] = eta;
+    w[J] = q;
+#pragma unroll
+    for (int k = J + 1; k < 64; ++k) w[k] = fmaf(-eta, a.Rs[C][OFF + k], w[k]);
+  }
+}
+
+template <int OFF, bool UNIFORM, int... Js>
+__device__ __forceinline__ void col_steps(float (&w)[64], const ColStepArgs& a,
+                                          std::integer_sequence<int, Js...>) {
+  (col_step<Js, OFF, UNIFORM>(w, a), ...);
+}
+
+template <bool UNIFORM>
+__global__ void __launch_bounds__(32) k_colblock(
+    float* __restrict__ Wk, int m, int d, int i, int nb, const float* __restrict__ R,
+    const float* __restrict__ scales, const int32_t* __restrict__ zeros, int ng,
+    const int32_t* __restrict__ gcol, int bits, float* __restrict__ E,
+    uint8_t* __restrict__ codes, float* __restrict__ loss_part) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float(*Rs)[128] = reinterpret_cast<float(*)[128]>(smem);
+  float(*St)[129] = reinterpret_cast<float(*)[129]>(smem + 128 * 128 * 4);
+  float(*Qs)[129] = reinterpret_cast<float(*)[129]>(smem + 128 * 128 * 4 + 32 * 129 * 4);
+  uint8_t(*Cs)[132] =
+      reinterpret_cast<uint8_t(*)[132]>(smem + 128 * 128 * 4 + 2 * 32 * 129 * 4);
+  __shared__ int gs[128];
+  __shared__ float rinv[128];
+
+  const int lane = threadIdx.x;
+  const int row0 = blockIdx.x * 32;
+  const int row = row0 + lane;
+  const bool active = row < m;
+
+  for (int e = lane; e < 128 * 128; e += 32) {
+    const int a = e >> 7, b = e & 127;
+    Rs[a][b] = (a < nb && b < nb && b >= a) ? R[(long long)(i + a) * d + i + b] : 0.f;
+  }
+  for (int a = lane; a < 128; a += 32) gs[a] = (a < nb) ? gcol[i + a] : 0;
+  for (int r = 0; r < 32; ++r) {
+    const int gr = row0 + r;
+    for (int t = lane; t < 128; t += 32)
+      St[r][t] = (gr < m && t < nb) ? Wk[(long long)gr * d + i + t] : 0.f;
+  }
+  __syncwarp();
+  for (int a = lane; a < 128; a += 32) rinv[a] = (a < nb) ? 1.f / Rs[a][a] : 0.f;
+
+  ColStepArgs args;
+  args.Rs = Rs; args.St = St; args.Cs = Cs; args.gs = gs; args.rinv = rinv;
+  args.scales = scales; args.zeros = zeros;
+  args.srow = (long long)row * ng;
+  args.lane = lane; args.nb = nb; args.active = active;
+  args.maxq = (float)((1 << bits) - 1);
+  args.D0 = 1.f; args.Z0 = 0.f;
+  if (UNIFORM && active) {
+    args.D0 = scales[args.srow + gs[0]];
+    args.Z0 = (float)zeros[args.srow + gs[0]];
+  }
+  float w[64];
+  // first half: columns 0..63
+#pragma unroll
+  for (int t = 0; t < 64; ++t) w[t] = St[lane][t];
+  __syncwarp();
+  col_steps<0, UNIFORM>(w, args, std::make_integer_sequence<int, 64>{});
+#pragma unroll
+  for (int t = 0; t < 64; ++t) Qs[lane][t] = w[t];
+  if (nb > 64) {
+    // second half: receive the first half's residuals (E[:, 0:64] R[0:64, 64:128]) first
+#pragma unroll
+    for (int t = 0; t < 64; ++t) w[t] = St[lane][64 + t];
+    for (int j = 0; j < 64; ++j) {
+      const float e = St[lane][j];
+#pragma unroll
+      for (int t = 0; t < 64; ++t) w[t] = fmaf(-e, Rs[j][64 + t], w[t]);
+    }
+    col_steps<64, UNIFORM>(w, args, std::make_integer_sequence<int, 64>{});
+#pragma unroll
+    for (int t = 0; t < 64; ++t) Qs[lane][64 + t] = w[t];
+  }
+  __syncwarp();
+  // E (scaled residuals) and the per-column loss partial Σ_rows η² over this CTA's rows
+  for (int r = 0; r < 32; ++r) {
+    const int gr = row0 + r;
+    if (gr >= m) break;
+    for (int t = lane; t < nb; t += 32) E[(long long)gr * kColMax + t] = St[r][t];
+  }
+  for (int t = lane; t < nb; t += 32) {
+    float s = 0.f;
+    for (int r = 0; r < 32 && row0 + r < m; ++r) s = fmaf(St[r][t], St[r][t], s);
+    loss_part[(long long)blockIdx.x * d + i + t] = s;
+  }
+  for (int r = 0; r < 32; ++r) {
+    const int gr = row0 + r;
+    if (gr >= m) break;
+    for (int t = lane; t < nb; t += 32) {
+      Wk[(long long)gr * d + i + t] = Qs[r][t];
+      codes[(long long)gr * d + i + t] = Cs[r][t];
+    }
+  }
+}
+
+int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
+                 const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
+                 bool uniform_grid, int bits, float* E, uint8_t* codes, float* loss_part) {
+  GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<true>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
+  GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
+  const int blocks = (m + 31) / 32;
+  if (uniform_grid)
+    k_colblock<true><<<blocks, 32, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
+                                                          gcol, bits, E, codes, loss_part);
+  else
+    k_colblock<false><<<blocks, 32, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
+                                                           gcol, bits, E, codes, loss_part);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
+
+// a6: W[:, i+nb:] -= E R[i:i+nb, i+nb:]  ([T] eq.(46)), fp32 on CUDA cores.
+int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* E,
+                    const float* R) {
+  const int n = d - i - nb;
+  if (n <= 0) return GPTQ_OK;
+  int rc;
+  GemmArgs g{m, n, nb, E, kColMax, 1, R + (long long)i * d + i + nb, d, 1,
+             Wk + i + nb, d, -1.f, 1.f, 0};
+  if ((rc = gemm_simt(c, g))) return rc;
+  return GPTQ_OK;
+}
+
+// col_loss[j] = ½ Σ_parts Σ_rows η²  (= Σ_rows ρ² / (2 R_jj²), [T] eq.(43))
+__global__ void k_loss_reduce(const float* __restrict__ part, int parts, int d,
+                              float* __restrict__ out) {
+  int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  double s = 0.0;
+  for (int p = 0; p < parts; ++p) s += (double)part[(long long)p * d + j];
+  out[j] = (float)(0.5 * s);
+}
+
+int loss_reduce(Ctx* c, const float* loss_part, int parts, int d, float* loss_p) {
+  k_loss_reduce<<<(d + 255) / 256, 256, 0, c->stream>>>(loss_part, parts, d, loss_p);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
+
+// a7: back to original column order ([T] §10: undo the column permutation).
+__global__ void k_unpermute(long long m, int d, const int32_t* __restrict__ inv,
+                            const uint8_t* __restrict__ codes_p, const float* __restrict__ Wk,
+                            const float* __restrict__ loss_p, uint8_t* __restrict__ codes,
+                            float* __restrict__ W_hat, float* __restrict__ col_loss) {
+  const long long total = m * d;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    long long r = e / d;
+    int k = (int)(e - r * d);
+    long long src = r * d + inv[k];
+    codes[e] = codes_p[src];
+    W_hat[e] = Wk[src];
+    if (r == 0) col_loss[k] = loss_p[inv[k]];
+  }
+}
+
+int unpermute(Ctx* c, int m, int d, const int32_t* inv, const uint8_t* codes_p, const float* Wk,
+              const float* loss_p, uint8_t* codes, float* W_hat, float* col_loss) {
+  const long long total = (long long)m * d;
+  int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
+  k_unpermute<<<blocks, 256, 0, c->stream>>>(m, d, inv, codes_p, Wk, loss_p, codes, W_hat,
+                                             col_loss);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

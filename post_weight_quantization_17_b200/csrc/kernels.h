@@ -1,0 +1,47 @@
+// Host-side launchers of the library's kernels (internal; the C ABI is in include/gptq.h).
+#pragma once
+#include "common.cuh"
+
+namespace gptq {
+
+// ---- a1 Hessian statistic
+int syrk_accumulate(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool overwrite);
+
+// ---- a2 preconditioning
+int prep_diag(Ctx* c, const float* S, int d, float scale, float* diagv, uint8_t* dead);
+int prep_mean(Ctx* c, const float* diagv, int d);
+int prep_perm(Ctx* c, const float* diagv, int d, int act_order, int32_t* perm);
+int prep_build(Ctx* c, const float* S, int d, float scale, const float* diagv, const int32_t* perm,
+               bool identity, float* Hp);
+int prep_copy(Ctx* c, const float* src, float* dst, size_t count);
+int prep_damp(Ctx* c, float* Hl, int d, float percdamp);
+
+// ---- a3 factorization: M (ld) holds H_λ (symmetric); on return its upper triangle is R with
+// R^T R = H_λ^{-1} and its strict lower triangle is zero.  tmp: factor_tmp_floats(d) floats.
+size_t factor_tmp_floats(int d);
+int factor_inverse(Ctx* c, float* M, int d, float* tmp);
+
+// ---- a4-a7 quantization
+int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int group,
+             float* scales, int32_t* zeros);
+int make_gcol(Ctx* c, const int32_t* perm, int d, int group, int32_t* gcol, int32_t* inv);
+int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* perm,
+              const uint8_t* dead, bool identity, float* Wk);
+int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
+                 const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
+                 bool uniform_grid, int bits, float* E, uint8_t* codes, float* loss_part);
+int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* E,
+                    const float* R);
+int loss_reduce(Ctx* c, const float* loss_part, int parts, int d, float* loss_p);
+int unpermute(Ctx* c, int m, int d, const int32_t* inv, const uint8_t* codes_p,
+              const float* Wk, const float* loss_p, uint8_t* codes, float* W_hat,
+              float* col_loss);
+
+// ---- a8 packing
+int pack_codes(Ctx* c, const uint8_t* codes, int m, int d, int bits, uint32_t* packed);
+int unpack_codes(Ctx* c, const uint32_t* packed, int m, int d, int bits, uint8_t* codes);
+
+constexpr int kColRows = 32;      // rows per column-block CTA (one warp, one row per lane)
+constexpr int kColMax = 128;      // columns per kernel block
+
+}  // namespace gptq

@@ -1,0 +1,97 @@
+"""GPU parity: the C-ABI path against the fp64 oracle on the same seeded inputs, at sizes the
+oracle finishes in seconds that still span several tiles and ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+from tests import _parity as P  # noqa: E402
+from workloads.synth import CONFIGS, LayerSpec  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    import post_weight_quantization_17_b200 as G
+    c = G.Context(m_max=512, d_max=1024, act_order=True)
+    yield c
+    c.close()
+
+
+SMALL = [
+    ("config1_tiny", CONFIGS[1][0], 0),
+    ("qproj_shape", CONFIGS[2][0].scaled(160, 384, 3000, chunk=1024), 1),
+    ("downproj_actorder_3bit", CONFIGS[3][0].scaled(96, 300, 2000, chunk=700), 2),
+    ("block7b_down_shape", CONFIGS[4][6].scaled(72, 256, 1500), 3),
+    ("fc2_shape_2bit", CONFIGS[5][1].scaled(130, 256, 2048, chunk=512), 4),
+    ("fc2_shape_4bit", CONFIGS[5][0].scaled(40, 200, 900, chunk=300), 9),
+    ("ragged_all", LayerSpec("ragged", 77, 333, 1001, bits=4, group=128, block=128,
+                             act_order=False, x_kind="lowrank_t3", x_rank=40, chunk=333), 5),
+    ("ragged_actorder_rowgrid", LayerSpec("ragged2", 33, 197, 517, bits=3, group=-1, block=64,
+                                          act_order=True, x_kind="swiglu", x_rank=30,
+                                          chunk=200), 6),
+    ("degenerate_1x1", LayerSpec("one", 1, 1, 1, bits=4, group=-1, block=128, act_order=False,
+                                 x_kind="lowrank_t3", x_rank=1, chunk=1), 7),
+    ("tiny_3x5", LayerSpec("tiny35", 3, 5, 4, bits=2, group=2, block=2, act_order=True,
+                           x_kind="relu_lowrank", x_rank=2, chunk=3), 8),
+]
+
+
+@pytest.mark.parametrize("name,spec,seed", SMALL, ids=[c[0] for c in SMALL])
+def test_layer_parity(ctx, name, spec, seed):
+    W, chunks = P.make_inputs(spec, seed)
+    gpu = P.gpu_run(ctx, spec, W, chunks)
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    Wn = P.to_np64(W)
+    H, herr = P.check_hessian(gpu, Xt)
+    res = P.check_layer(gpu, Wn, H, spec)
+    print(name, f"H={herr:.2e}", {k: (f"{v:.2e}" if isinstance(v, float) else v) for k, v in res.items()})
+
+
+def test_factor_stage_isolated(ctx):
+    """Same fp32 H handed to both sides: R and H^-1 from the factorization alone."""
+    from oracle import gptq_oracle as O
+    spec = CONFIGS[2][0].scaled(64, 700, 4000, chunk=4000)
+    W, chunks = P.make_inputs(spec, 11)
+    H32 = O.hessian_tokens(torch.cat(chunks).cpu().double().numpy()).astype(np.float32)
+    gpu = P.gpu_run(ctx, spec, W, chunks, H32=H32)
+    o = O.prepare_with_retry(H32.astype(np.float64), spec.percdamp, False)
+    Rg = gpu["R"].astype(np.float64)
+    assert P.rel_fro(Rg, o["R"]) <= P.TOL_HINV
+    assert P.rel_fro(Rg.T @ Rg, o["G"]) <= P.TOL_HINV
+    assert abs(gpu["lam"] - o["lam"]) <= 1e-6 * o["lam"]
+
+
+@pytest.mark.parametrize("block", [1, 7, 32, 128, 200])
+def test_block_size_invariance(ctx, block):
+    """Lazy blocks of any size give the unblocked result ([T] eq.(47)-(49))."""
+    spec = CONFIGS[2][0].scaled(64, 260, 1200, chunk=600)
+    W, chunks = P.make_inputs(spec, 21)
+    gpu = P.gpu_run(ctx, spec, W, chunks, block=block)
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    H, _ = P.check_hessian(gpu, Xt)
+    P.check_layer(gpu, P.to_np64(W), H, spec, block=block)
+
+
+def test_dead_features(ctx):
+    spec = CONFIGS[3][0].scaled(48, 200, 800, chunk=400)
+    W, chunks = P.make_inputs(spec, 31, zero_features=(0, 17, 130, 199))
+    gpu = P.gpu_run(ctx, spec, W, chunks)
+    assert gpu["dead"].nonzero()[0].tolist() == [0, 17, 130, 199]
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    H, _ = P.check_hessian(gpu, Xt)
+    P.check_layer(gpu, P.to_np64(W), H, spec)
+    assert np.all(gpu["W_hat"][:, [0, 17, 130, 199]] == 0)
+
+
+def test_unpack_roundtrip(ctx):
+    import post_weight_quantization_17_b200 as G
+    g = torch.Generator(device="cuda").manual_seed(5)
+    for bits, d in [(2, 37), (3, 333), (4, 256), (8, 65)]:
+        codes = torch.randint(0, 2 ** bits, (9, d), generator=g, device="cuda", dtype=torch.int32).to(torch.uint8)
+        packed = torch.empty(9, G.words_per_row(d, bits), dtype=torch.int32, device="cuda")
+        G.gptq_pack(ctx, codes, bits, packed)
+        back = torch.empty_like(codes)
+        G.gptq_unpack(ctx, packed, d, bits, back)
+        torch.cuda.synchronize()
+        assert torch.equal(back, codes)
