@@ -39,8 +39,10 @@ int read_status(Ctx* c, gptq::DeviceStatus* out) {
   return GPTQ_OK;
 }
 
+// Clears the error code and its location only; the cached reductions (mean diagonal, λ)
+// survive so that a damping retry can reuse them.
 int clear_status(Ctx* c) {
-  GPTQ_CUDA_CHECK(c, cudaMemsetAsync(c->status, 0, sizeof(gptq::DeviceStatus), c->stream));
+  GPTQ_CUDA_CHECK(c, cudaMemsetAsync(c->status, 0, 2 * sizeof(int), c->stream));
   return GPTQ_OK;
 }
 
@@ -76,7 +78,8 @@ int gptq_create(gptq_ctx** out, void* stream, void* workspace, size_t workspace_
   c->ws = reinterpret_cast<char*>(workspace);
   c->ws_bytes = workspace_bytes;
   c->status = reinterpret_cast<gptq::DeviceStatus*>(c->ws);
-  if (clear_status(c) != GPTQ_OK || cudaStreamSynchronize(c->stream) != cudaSuccess) {
+  if (cudaMemsetAsync(c->ws, 0, gptq::kStatusBytes, c->stream) != cudaSuccess ||
+      cudaStreamSynchronize(c->stream) != cudaSuccess) {
     if (c->owns_ws) cudaFree(c->ws);
     delete h;
     return GPTQ_ERR_CUDA;

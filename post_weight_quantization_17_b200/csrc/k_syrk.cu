@@ -1,12 +1,265 @@
 // a1: Hessian statistic S += Xc^T Xc over one token chunk ([T] eq.(9); accumulated in batches,
-// [T] §9.4).  This translation unit holds the CUDA-core path (fp32 inputs, and any input when
-// the tensor-core path does not apply); only tiles touching the lower triangle are computed.
+// [T] §9.4).  Only the lower triangle of S is produced.
+//
+// Tensor-core path (bf16 / f16 X, d % 8 == 0): a persistent kernel over 128 x 256 output
+// tiles that touch the lower triangle.  X is token-major, so for a tile (I, J) both MMA
+// operands are MN-major slices of the same chunk: A[i, t] = X[t, 128 I + i] and
+// B[j, t] = X[t, 256 J + j].  Products of two 16-bit values are exact in fp32; sums are fp32
+// in TMEM.
+//   warp 0      TMA producer: 64-token slabs of A (2 boxes) and B (4 boxes), 4-stage ring
+//   warp 1      MMA issuer: tcgen05.mma kind::f16, M=128 N=256 K=16, fp32 accumulator in TMEM
+//   warps 2..5  epilogue: TMEM -> registers -> S (+=), double-buffered accumulators so the
+//               epilogue of one tile overlaps the main loop of the next
+// Every wait is bounded; a wait that runs out records GPTQ_ERR_TIMEOUT and the CTA unwinds
+// (drains its own TMA copies, frees TMEM) instead of hanging.
+//
+// CUDA-core path: fp32 X, or shapes the tensor path does not take.
 #include "kernels.h"
 #include "gemm_simt.cuh"
+#include "tc_util.cuh"
 
 namespace gptq {
 
-int syrk_tc(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool overwrite);
+constexpr int SY_BM = 128, SY_BN = 256, SY_BK = 64, SY_STAGES = 4;
+constexpr int SY_BOX_BYTES = SY_BK * 64 * 2;             // one 64 x 64 box of 16-bit values
+constexpr int SY_A_BYTES = (SY_BM / 64) * SY_BOX_BYTES;  // 16 KB
+constexpr int SY_B_BYTES = (SY_BN / 64) * SY_BOX_BYTES;  // 32 KB
+constexpr int SY_STAGE_BYTES = SY_A_BYTES + SY_B_BYTES;
+constexpr int SY_SMEM = SY_STAGES * SY_STAGE_BYTES + 1024 + 256;
+constexpr int SY_THREADS = 192;
+
+__device__ __forceinline__ void syrk_tile_coords(int t, int& I, int& J) {
+  int i = 0;
+  for (;;) {
+    const int cnt = i / 2 + 1;  // tiles of row-block i touching j <= i: J = 0 .. floor(i/2)
+    if (t < cnt) {
+      I = i;
+      J = t;
+      return;
+    }
+    t -= cnt;
+    ++i;
+  }
+}
+
+__global__ void __launch_bounds__(SY_THREADS, 1)
+    k_syrk_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ S, int d,
+              int n_tokens, int accumulate, int num_tiles, uint32_t idesc, DeviceStatus* st,
+              long long budget) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SY_STAGES * SY_STAGE_BYTES);
+  uint64_t* empty = full + SY_STAGES;
+  uint64_t* tfull = empty + SY_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SY_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tfull[a], 1);
+      tc::mbar_init(&tempty[a], 128);
+    }
+    *abort_flag = 0;
+    tc::mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) tc::prefetch_tmap(&tmap);
+  if (warp == 1) tc::tmem_alloc(tmem_slot, 512);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int kblocks = (n_tokens + SY_BK - 1) / SY_BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued[SY_STAGES] = {};
+      uint32_t issued_phase[SY_STAGES] = {};
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        int I, J;
+        syrk_tile_coords(t, I, J);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1, budget)) {
+            raise_error(st, GPTQ_ERR_TIMEOUT, 1);
+            *abort_flag = 1;
+            break;
+          }
+          uint8_t* sA = smem + stage * SY_STAGE_BYTES;
+          uint8_t* sB = sA + SY_A_BYTES;
+          tc::mbar_expect_tx(&full[stage], SY_STAGE_BYTES);
+          const int y = kb * SY_BK;
+          tc::tma_load_2d(sA, &tmap, &full[stage], I * SY_BM, y);
+          tc::tma_load_2d(sA + SY_BOX_BYTES, &tmap, &full[stage], I * SY_BM + 64, y);
+#pragma unroll
+          for (int b = 0; b < SY_BN / 64; ++b)
+            tc::tma_load_2d(sB + b * SY_BOX_BYTES, &tmap, &full[stage], J * SY_BN + 64 * b, y);
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == SY_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // drain: every copy this thread issued has landed before the CTA may exit
+      for (int s = 0; s < SY_STAGES; ++s)
+        if (issued[s] && !tc::mbar_wait(&full[s], issued_phase[s], budget))
+          raise_error(st, GPTQ_ERR_TIMEOUT, 2);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+        if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, budget)) {
+          raise_error(st, GPTQ_ERR_TIMEOUT, 3);
+          *abort_flag = 1;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem + acc * SY_BN;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!tc::mbar_wait(&full[stage], phase, budget)) {
+            raise_error(st, GPTQ_ERR_TIMEOUT, 4);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t a0 = tc::smem_u32(smem + stage * SY_STAGE_BYTES);
+          const uint32_t b0 = a0 + SY_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < SY_BK / 16; ++kk) {
+            const uint64_t ad = tc::sdesc_sw128(a0 + kk * 2048, SY_BOX_BYTES, 1024);
+            const uint64_t bd = tc::sdesc_sw128(b0 + kk * 2048, SY_BOX_BYTES, 1024);
+            tc::mma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc::mma_commit(&empty[stage]);
+          if (++stage == SY_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc::mma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31, i.e. tile rows of that quarter
+    const int q = warp & 3;
+    const int r = 32 * q + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+      int I, J;
+      syrk_tile_coords(t, I, J);
+      if (!tc::mbar_wait(&tfull[acc], acc_phase, budget)) {
+        raise_error(st, GPTQ_ERR_TIMEOUT, 5);
+        *abort_flag = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      const int gi = I * SY_BM + r;
+      float* srow = S + (long long)gi * d;
+#pragma unroll 1
+      for (int cc = 0; cc < SY_BN / 32; ++cc) {
+        uint32_t v[32];
+        tc::tmem_ld32(tmem + acc * SY_BN + ((uint32_t)(32 * q) << 16) + cc * 32, v);
+        const int gj0 = J * SY_BN + cc * 32;
+        if (gi >= d || gj0 > gi) continue;
+        if (gj0 + 31 <= gi && gj0 + 32 <= d) {
+          float4* p = reinterpret_cast<float4*>(srow + gj0);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float4 x = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                   __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+            if (accumulate) {
+              const float4 o = p[u];
+              x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
+            }
+            p[u] = x;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int gj = gj0 + u;
+            if (gj <= gi && gj < d) {
+              const float x = __uint_as_float(v[u]);
+              srow[gj] = accumulate ? srow[gj] + x : x;
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int syrk_tc(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool overwrite) {
+  auto encode = get_encode();
+  if (!encode) GPTQ_SET_ERR(c, GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  CUtensorMap map;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)n};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, SY_BK};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&map, dtype == GPTQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                      2, const_cast<void*>(X), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) GPTQ_SET_ERR(c, GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  const int nI = (d + SY_BM - 1) / SY_BM;
+  int num_tiles = 0;
+  for (int i = 0; i < nI; ++i) num_tiles += i / 2 + 1;
+  const int grid = std::min(num_tiles, c->num_sms);
+  GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_syrk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          SY_SMEM));
+  const uint32_t idesc = tc::idesc_f32acc(dtype == GPTQ_BF16 ? 1u : 0u, true, true, SY_BM, SY_BN);
+  k_syrk_tc<<<grid, SY_THREADS, SY_SMEM, c->stream>>>(map, S, d, (int)n, overwrite ? 0 : 1,
+                                                      num_tiles, idesc, c->status,
+                                                      c->timeout_cycles);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
 
 int syrk_simt(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool overwrite) {
   GemmArgs g{d, d, (int)n, X, 1, d, X, d, 1, S, d, 1.f, overwrite ? 0.f : 1.f, kCLower};
@@ -15,9 +268,17 @@ int syrk_simt(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bo
   return gemm_simt<float, float>(c, g);
 }
 
+// The tensor path needs 16-byte aligned rows for TMA (d % 8 == 0, aligned base) and takes
+// shapes at least one box wide; smaller or fp32 inputs use the CUDA-core kernel.
+static bool syrk_tc_applies(const void* X, int dtype, long long n, int d) {
+  return (dtype == GPTQ_BF16 || dtype == GPTQ_F16) && d % 8 == 0 && d >= 128 && n >= SY_BK &&
+         (reinterpret_cast<uintptr_t>(X) & 15) == 0;
+}
+
 int syrk_accumulate(Ctx* c, const void* X, int dtype, long long n, int d, float* S,
                     bool overwrite) {
-  return syrk_simt(c, X, dtype, n, d, S, overwrite);
+  if (!syrk_tc_applies(X, dtype, n, d)) return syrk_simt(c, X, dtype, n, d, S, overwrite);
+  return syrk_tc(c, X, dtype, n, d, S, overwrite);
 }
 
 }  // namespace gptq

@@ -13,7 +13,7 @@ from workloads.synth import CONFIGS, LayerSpec  # noqa: E402
 @pytest.fixture(scope="module")
 def ctx():
     import post_weight_quantization_17_b200 as G
-    c = G.Context(m_max=512, d_max=1024, act_order=True)
+    c = G.Context(m_max=512, d_max=1024, act_order=True)  # Hessian-only calls need no workspace
     yield c
     c.close()
 
@@ -95,3 +95,24 @@ def test_unpack_roundtrip(ctx):
         G.gptq_unpack(ctx, packed, d, bits, back)
         torch.cuda.synchronize()
         assert torch.equal(back, codes)
+
+
+@pytest.mark.parametrize("d,n_tok,chunk", [(4096, 8192, 4096), (1000, 3001, 1024), (264, 130, 65)])
+def test_hessian_tensor_path(ctx, d, n_tok, chunk):
+    """The tensor-core Hessian over several waves of tiles, ragged d and token tails, and
+    accumulation across chunks, against the fp64 oracle."""
+    import post_weight_quantization_17_b200 as G
+    from oracle import gptq_oracle as O
+    spec = CONFIGS[2][0].scaled(64, d, n_tok, chunk=chunk)
+    _, chunks = P.make_inputs(spec, 41)
+    S = torch.empty(d, d, dtype=torch.float32, device="cuda")
+    n = 0
+    for c in chunks:
+        n = G.gptq_hessian_accumulate(ctx, c, S, n)
+    G.gptq_sync_status(ctx)
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    H = O.hessian_tokens(Xt)
+    Hg = np.tril(S.cpu().double().numpy()) * (2.0 / n)
+    err = P.rel_fro(Hg, np.tril(H))
+    print(f"d={d} N={n_tok} H rel err {err:.3e}")
+    assert err <= P.TOL_H
