@@ -306,7 +306,11 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
     a violation.  Several outputs are correct near a boundary, so the decisions that are
     unique are compared and the rest are checked for validity.
 
-    Returns dict(n, identical, in_band, violations, max_excess, replay_Q).
+    Along the replayed decisions it also records Ŵ (replay_Q) and the per-column loss
+    Σ_r ρ² / (2 R_jj²) ([T] eq.(43)), which are the oracle's values for those decisions.
+
+    Returns dict(n, identical, in_band, violations, max_excess, replay_Q, replay_loss,
+    rows_with_flips).
     """
     W = np.array(Wp, dtype=np.float64, copy=True)
     R = np.asarray(R, np.float64)
@@ -316,6 +320,8 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
     identical = in_band = violations = 0
     max_excess = 0.0
     Qr = np.zeros((m, d), np.float64)
+    loss = np.zeros(d, np.float64)
+    flipped = np.zeros(m, bool)
     for j in range(d):
         delta = np.asarray(scale[:, gcol[j]], np.float32)
         z = np.asarray(zero[:, gcol[j]], np.int64)
@@ -324,6 +330,7 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
         same = c_o == c_g
         identical += int(np.sum(same))
         diff = ~same
+        flipped |= diff
         if np.any(diff):
             lo = np.minimum(c_o[diff], c_g[diff])
             adjacent = np.abs(c_o[diff] - c_g[diff]) == 1
@@ -338,10 +345,11 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
         q = (delta * (cg - z).astype(np.float32)).astype(np.float32).astype(np.float64)
         rho = W[:, j] - q
         eta = rho / R[j, j]
+        loss[j] = float(np.sum(rho ** 2)) / (2.0 * R[j, j] ** 2)
         W[:, j:] -= np.outer(eta, R[j, j:])
         Qr[:, j] = q
     return dict(n=m * d, identical=identical, in_band=in_band, violations=violations,
-                max_excess=max_excess, replay_Q=Qr)
+                max_excess=max_excess, replay_Q=Qr, replay_loss=loss, rows_with_flips=flipped)
 
 
 # --------------------------------------------------------------------------------------------

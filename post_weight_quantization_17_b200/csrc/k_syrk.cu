@@ -4,12 +4,15 @@
 // Tensor-core path (bf16 / f16 X, d % 8 == 0): a persistent kernel over 128 x 256 output
 // tiles that touch the lower triangle.  X is token-major, so for a tile (I, J) both MMA
 // operands are MN-major slices of the same chunk: A[i, t] = X[t, 128 I + i] and
-// B[j, t] = X[t, 256 J + j].  Products of two 16-bit values are exact in fp32; sums are fp32
-// in TMEM.
+// B[j, t] = X[t, 256 J + j].  Products of two 16-bit values are exact in fp32.
 //   warp 0      TMA producer: 64-token slabs of A (2 boxes) and B (4 boxes), 4-stage ring
-//   warp 1      MMA issuer: tcgen05.mma kind::f16, M=128 N=256 K=16, fp32 accumulator in TMEM
-//   warps 2..5  epilogue: TMEM -> registers -> S (+=), double-buffered accumulators so the
-//               epilogue of one tile overlaps the main loop of the next
+//   warp 1      MMA issuer: tcgen05.mma kind::f16, M=128 N=256 K=16, fp32 partial sums in TMEM
+//   warps 2..9  epilogue: every SY_KP tokens the TMEM partial is added (fp32, round to
+//               nearest) into a 128 x 256 accumulator held in the epilogue warps' registers
+//               (each thread: one row, 128 columns); at the end of the tile it goes to S.
+// The tensor core's own fp32 accumulation loses precision roughly in proportion to the number
+// of MMA steps it sums, so partial sums are kept short (256 tokens) and the long sum over all
+// tokens is done with IEEE adds.  Two TMEM partial buffers let the MMA run ahead of the adds.
 // Every wait is bounded; a wait that runs out records GPTQ_ERR_TIMEOUT and the CTA unwinds
 // (drains its own TMA copies, frees TMEM) instead of hanging.
 //
@@ -21,12 +24,15 @@
 namespace gptq {
 
 constexpr int SY_BM = 128, SY_BN = 256, SY_BK = 64, SY_STAGES = 4;
+constexpr int SY_KP = 256;                               // tokens per TMEM partial sum
+constexpr int SY_KB_PER_PART = SY_KP / SY_BK;
 constexpr int SY_BOX_BYTES = SY_BK * 64 * 2;             // one 64 x 64 box of 16-bit values
 constexpr int SY_A_BYTES = (SY_BM / 64) * SY_BOX_BYTES;  // 16 KB
 constexpr int SY_B_BYTES = (SY_BN / 64) * SY_BOX_BYTES;  // 32 KB
 constexpr int SY_STAGE_BYTES = SY_A_BYTES + SY_B_BYTES;
 constexpr int SY_SMEM = SY_STAGES * SY_STAGE_BYTES + 1024 + 256;
-constexpr int SY_THREADS = 192;
+constexpr int SY_EPI_WARPS = 8;
+constexpr int SY_THREADS = 64 + 32 * SY_EPI_WARPS;
 
 __device__ __forceinline__ void syrk_tile_coords(int t, int& I, int& J) {
   int i = 0;
@@ -64,7 +70,7 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       tc::mbar_init(&tfull[a], 1);
-      tc::mbar_init(&tempty[a], 128);
+      tc::mbar_init(&tempty[a], 32 * SY_EPI_WARPS);
     }
     *abort_flag = 0;
     tc::mbar_fence_init();
@@ -76,6 +82,7 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const int kblocks = (n_tokens + SY_BK - 1) / SY_BK;
+  const int nparts = (kblocks + SY_KB_PER_PART - 1) / SY_KB_PER_PART;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -118,96 +125,119 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
     if (lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, budget)) {
-          raise_error(st, GPTQ_ERR_TIMEOUT, 3);
-          *abort_flag = 1;
-          break;
-        }
-        tc::fence_after_sync();
-        const uint32_t d_tmem = tmem + acc * SY_BN;
-        bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!tc::mbar_wait(&full[stage], phase, budget)) {
-            raise_error(st, GPTQ_ERR_TIMEOUT, 4);
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok && !*abort_flag; t += gridDim.x) {
+        for (int p = 0; p < nparts && ok; ++p) {
+          if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, budget)) {
+            raise_error(st, GPTQ_ERR_TIMEOUT, 3);
             *abort_flag = 1;
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          const uint32_t a0 = tc::smem_u32(smem + stage * SY_STAGE_BYTES);
-          const uint32_t b0 = a0 + SY_A_BYTES;
+          const uint32_t d_tmem = tmem + acc * SY_BN;
+          const int kb1 = min(kblocks, (p + 1) * SY_KB_PER_PART);
+          for (int kb = p * SY_KB_PER_PART; kb < kb1; ++kb) {
+            if (!tc::mbar_wait(&full[stage], phase, budget)) {
+              raise_error(st, GPTQ_ERR_TIMEOUT, 4);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+            const uint32_t a0 = tc::smem_u32(smem + stage * SY_STAGE_BYTES);
+            const uint32_t b0 = a0 + SY_A_BYTES;
+            const bool first = (kb == p * SY_KB_PER_PART);
 #pragma unroll
-          for (int kk = 0; kk < SY_BK / 16; ++kk) {
-            const uint64_t ad = tc::sdesc_sw128(a0 + kk * 2048, SY_BOX_BYTES, 1024);
-            const uint64_t bd = tc::sdesc_sw128(b0 + kk * 2048, SY_BOX_BYTES, 1024);
-            tc::mma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < SY_BK / 16; ++kk) {
+              const uint64_t ad = tc::sdesc_sw128(a0 + kk * 2048, SY_BOX_BYTES, 1024);
+              const uint64_t bd = tc::sdesc_sw128(b0 + kk * 2048, SY_BOX_BYTES, 1024);
+              tc::mma_f16(d_tmem, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+            }
+            tc::mma_commit(&empty[stage]);
+            if (++stage == SY_STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
-          tc::mma_commit(&empty[stage]);
-          if (++stage == SY_STAGES) {
-            stage = 0;
-            phase ^= 1;
+          if (!ok) break;
+          tc::mma_commit(&tfull[acc]);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1;
           }
         }
-        if (!ok) break;
-        tc::mma_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (tile rows of that quarter) and
+    // the 128-column half h of the tile
+    const int q = warp & 3;
+    const int h = (warp - 2) / 4;
+    const int r = 32 * q + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok && !*abort_flag; t += gridDim.x) {
+      int I, J;
+      syrk_tile_coords(t, I, J);
+      float m[128];
+#pragma unroll
+      for (int u = 0; u < 128; ++u) m[u] = 0.f;
+      for (int p = 0; p < nparts; ++p) {
+        if (!tc::mbar_wait(&tfull[acc], acc_phase, budget)) {
+          raise_error(st, GPTQ_ERR_TIMEOUT, 5);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t base = tmem + acc * SY_BN + ((uint32_t)(32 * q) << 16) + h * 128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tc::tmem_ld32(base + cc * 32, v);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) m[cc * 32 + u] += __uint_as_float(v[u]);
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&tempty[acc]);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
-    }
-  } else {
-    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31, i.e. tile rows of that quarter
-    const int q = warp & 3;
-    const int r = 32 * q + lane;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-      int I, J;
-      syrk_tile_coords(t, I, J);
-      if (!tc::mbar_wait(&tfull[acc], acc_phase, budget)) {
-        raise_error(st, GPTQ_ERR_TIMEOUT, 5);
-        *abort_flag = 1;
-        break;
-      }
-      tc::fence_after_sync();
+      if (!ok) break;
       const int gi = I * SY_BM + r;
-      float* srow = S + (long long)gi * d;
-#pragma unroll 1
-      for (int cc = 0; cc < SY_BN / 32; ++cc) {
-        uint32_t v[32];
-        tc::tmem_ld32(tmem + acc * SY_BN + ((uint32_t)(32 * q) << 16) + cc * 32, v);
-        const int gj0 = J * SY_BN + cc * 32;
-        if (gi >= d || gj0 > gi) continue;
-        if (gj0 + 31 <= gi && gj0 + 32 <= d) {
-          float4* p = reinterpret_cast<float4*>(srow + gj0);
+      if (gi < d) {
+        float* srow = S + (long long)gi * d;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            float4 x = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                                   __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
-            if (accumulate) {
-              const float4 o = p[u];
-              x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
+        for (int cc = 0; cc < 4; ++cc) {
+          const int gj0 = J * SY_BN + h * 128 + cc * 32;
+          if (gj0 > gi) continue;
+          if (gj0 + 31 <= gi && gj0 + 32 <= d) {
+            float4* p4 = reinterpret_cast<float4*>(srow + gj0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4 x = make_float4(m[cc * 32 + 4 * u], m[cc * 32 + 4 * u + 1],
+                                     m[cc * 32 + 4 * u + 2], m[cc * 32 + 4 * u + 3]);
+              if (accumulate) {
+                const float4 o = p4[u];
+                x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
+              }
+              p4[u] = x;
             }
-            p[u] = x;
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int gj = gj0 + u;
-            if (gj <= gi && gj < d) {
-              const float x = __uint_as_float(v[u]);
-              srow[gj] = accumulate ? srow[gj] + x : x;
+            for (int u = 0; u < 32; ++u) {
+              const int gj = gj0 + u;
+              if (gj <= gi && gj < d) {
+                const float x = m[cc * 32 + u];
+                srow[gj] = accumulate ? srow[gj] + x : x;
+              }
             }
           }
         }
-      }
-      tc::fence_before_sync();
-      tc::mbar_arrive(&tempty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1;
       }
     }
   }

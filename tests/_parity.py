@@ -4,6 +4,11 @@ oracle on the same bytes, and compare with the tolerances of the hot-path contra
   H and H^-1 (and R) within 1e-4 relative Frobenius; codes identical for >= 99.9% of weights with
   every mismatch within 1e-3·Δ of a rounding boundary (decision replay); Ŵ within 1e-3
   relative; layer error within 1% of the oracle's; grid (Δ, z) and packed words bit-exact.
+
+Ŵ and the per-column loss are compared with the oracle's values for the same decisions (the
+replay): one legitimate boundary flip moves the rest of its row by whole grid steps, so a
+free-running comparison measures how many rows flipped, not the arithmetic.  Rows whose
+decisions all agree are also compared with the free-running oracle.
 """
 from __future__ import annotations
 
@@ -116,15 +121,24 @@ def check_layer(gpu, Wn, H, spec, block=None, method="explicit"):
     res["violations"] = rep["violations"]
     assert rep["violations"] == 0, f"{rep['violations']} code decisions outside the band"
     assert res["identical"] >= TOL_CODES_IDENTICAL, res
-    # Ŵ, layer error, per-column loss
-    res["W_hat"] = rel_fro(gpu["W_hat"], o["W_hat"])
+    # Ŵ against the replay (same decisions) and, on rows without flips, the free-running oracle
+    inv = np.argsort(o["perm"])
+    Q_replay = rep["replay_Q"][:, inv]
+    res["W_hat"] = rel_fro(gpu["W_hat"], Q_replay)
     assert res["W_hat"] <= TOL_WHAT, res
+    clean = ~rep["rows_with_flips"]
+    res["rows_with_flips"] = int(np.sum(~clean))
+    if np.any(clean):
+        res["W_hat_clean_rows"] = rel_fro(gpu["W_hat"][clean], o["W_hat"][clean])
+        assert res["W_hat_clean_rows"] <= TOL_WHAT, res
+    # layer error of the free-running outputs
     e_g = O.layer_error(Wn, gpu["W_hat"], H)
     e_o = O.layer_error(Wn, o["W_hat"], H)
     res["layer_err"] = abs(e_g - e_o) / e_o if e_o > 0 else abs(e_g)
     assert res["layer_err"] <= TOL_LAYER_ERR, res
-    res["col_loss"] = rel_fro(gpu["col_loss"], o["col_loss"])
-    assert res["col_loss"] <= 1e-2, res
+    # per-column loss ([T] eq.(43)) against the replay's
+    res["col_loss"] = rel_fro(gpu["col_loss"], rep["replay_loss"][inv])
+    assert res["col_loss"] <= 1e-3, res
     # Ŵ is exactly Δ (c - z) in fp32
     gcol_orig = o["gcol"][np.argsort(o["perm"])]
     sc = gpu["scales"][:, gcol_orig]

@@ -362,10 +362,14 @@ def test_decision_replay_accepts_self_and_flags_planted_mistake():
     codes_p = out["codes"][:, out["perm"]]
     rep = O.decision_replay(out["Wp"], out["R"], out["scale"], out["zero"], out["gcol"], 4, codes_p)
     assert rep["identical"] == rep["n"] and rep["violations"] == 0
+    assert np.allclose(rep["replay_loss"][np.argsort(out["perm"])], out["col_loss"], rtol=1e-10)
+    assert np.allclose(rep["replay_Q"][:, np.argsort(out["perm"])], out["W_hat"], atol=1e-12)
+    assert not rep["rows_with_flips"].any()
     bad = codes_p.copy()
     bad[3, 10] = (bad[3, 10] + 2) % 16
     rep = O.decision_replay(out["Wp"], out["R"], out["scale"], out["zero"], out["gcol"], 4, bad)
     assert rep["violations"] >= 1
+    assert rep["rows_with_flips"][3] and rep["rows_with_flips"].sum() == 1
 
 
 # ---------------------------------------------------------------- packing
