@@ -2,8 +2,8 @@
 // per product (factorization recursion, fp32 Hessian, first trailing update):
 //   C[i, j] = alpha * sum_k opA(i, k) opB(k, j) + beta * C[i, j]
 //   opA(i, k) = A[i * sai + k * sak], opB(k, j) = B[k * sbk + j * sbj]
-// Tiles of 128 x 128 x 8, 256 threads, 8 x 8 outputs per thread, register prefetch of the
-// next k-slab.  Structure flags skip work that is known to be zero:
+// Tiles of 128 x 128 (8 x 8 outputs per thread) or 64 x 64 (4 x 4), k-slabs of 8, 256 threads,
+// register prefetch of the next k-slab.  Structure flags skip work that is known to be zero:
 //   kAUpper: opA(i,k) = 0 for k < i      kALower: opA(i,k) = 0 for k > i
 //   kBUpper: opB(k,j) = 0 for k > j      kBLower: opB(k,j) = 0 for k < j
 //   kCUpper: only tiles touching i <= j are computed   kCLower: only tiles touching i >= j
@@ -25,63 +25,78 @@ struct GemmArgs {
   int flags;
 };
 
-constexpr int GBM = 128, GBN = 128, GBK = 8, GTHREADS = 256;
+constexpr int GBK = 8, GTHREADS = 256;
 
-template <class TA, class TB>
+// BM x BN tile, 16 x 16 threads, each computing (BM/16) x (BN/16) outputs split into groups of
+// 4 rows / 4 columns spaced BM/2 (BN/2) apart, so that the shared-memory reads are float4s.
+template <class TA, class TB, int BM, int BN>
 __global__ void __launch_bounds__(GTHREADS) k_gemm_simt(GemmArgs g) {
-  __shared__ __align__(16) float As[2][GBK][GBM + 4];
-  __shared__ __align__(16) float Bs[2][GBK][GBN + 4];
+  constexpr int TM = BM / 16, TN = BN / 16;          // 8 or 4
+  constexpr int LA = BM * GBK / GTHREADS, LB = BN * GBK / GTHREADS;
+  __shared__ __align__(16) float As[2][GBK][BM + 4];
+  __shared__ __align__(16) float Bs[2][GBK][BN + 4];
   const int tid = threadIdx.x;
-  const int i0 = blockIdx.y * GBM, j0 = blockIdx.x * GBN;
-  if ((g.flags & kCUpper) && i0 > j0 + GBN - 1) return;
-  if ((g.flags & kCLower) && j0 > i0 + GBM - 1) return;
+  const int i0 = blockIdx.y * BM, j0 = blockIdx.x * BN;
+  if ((g.flags & kCUpper) && i0 > j0 + BN - 1) return;
+  if ((g.flags & kCLower) && j0 > i0 + BM - 1) return;
   int kbeg = 0, kend = g.K;
   if (g.flags & kAUpper) kbeg = max(kbeg, i0);
   if (g.flags & kBLower) kbeg = max(kbeg, j0);
-  if (g.flags & kALower) kend = min(kend, i0 + GBM);
-  if (g.flags & kBUpper) kend = min(kend, j0 + GBN);
+  if (g.flags & kALower) kend = min(kend, i0 + BM);
+  if (g.flags & kBUpper) kend = min(kend, j0 + BN);
   kbeg = kbeg / GBK * GBK;
 
   const TA* A = reinterpret_cast<const TA*>(g.A);
   const TB* B = reinterpret_cast<const TB*>(g.B);
-  // loader mapping: 1024 elements per operand slab, 4 per thread; consecutive threads walk the
-  // unit-stride dimension so that global reads coalesce.
+  // loader mapping: consecutive threads walk the unit-stride dimension so reads coalesce
   const bool a_kcontig = (g.sak == 1);
   const bool b_ncontig = (g.sbj == 1);
-  float ra[4], rb[4];
+  float ra[LA], rb[LB];
+  auto a_idx = [&](int e, int& ii, int& kk) {
+    if (a_kcontig) { ii = e / GBK; kk = e % GBK; } else { kk = e / BM; ii = e % BM; }
+  };
+  auto b_idx = [&](int e, int& jj, int& kb) {
+    if (b_ncontig) { kb = e / BN; jj = e % BN; } else { jj = e / GBK; kb = e % GBK; }
+  };
   auto load_slab = [&](int k0) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      int e = tid + r * GTHREADS;
+    for (int r = 0; r < LA; ++r) {
       int ii, kk;
-      if (a_kcontig) { ii = e >> 3; kk = e & 7; } else { kk = e >> 7; ii = e & 127; }
-      int gi = i0 + ii, gk = k0 + kk;
-      ra[r] = (gi < g.M && gk < kend && gk >= kbeg) ? to_f32<TA>(A[(long long)gi * g.sai + (long long)gk * g.sak]) : 0.f;
+      a_idx(tid + r * GTHREADS, ii, kk);
+      const int gi = i0 + ii, gk = k0 + kk;
+      ra[r] = (gi < g.M && gk < kend && gk >= kbeg)
+                  ? to_f32<TA>(A[(long long)gi * g.sai + (long long)gk * g.sak]) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < LB; ++r) {
       int jj, kb;
-      if (b_ncontig) { kb = e >> 7; jj = e & 127; } else { jj = e >> 3; kb = e & 7; }
-      int gj = j0 + jj, gkb = k0 + kb;
-      rb[r] = (gj < g.N && gkb < kend && gkb >= kbeg) ? to_f32<TB>(B[(long long)gkb * g.sbk + (long long)gj * g.sbj]) : 0.f;
+      b_idx(tid + r * GTHREADS, jj, kb);
+      const int gj = j0 + jj, gkb = k0 + kb;
+      rb[r] = (gj < g.N && gkb < kend && gkb >= kbeg)
+                  ? to_f32<TB>(B[(long long)gkb * g.sbk + (long long)gj * g.sbj]) : 0.f;
     }
   };
   auto store_slab = [&](int buf) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      int e = tid + r * GTHREADS;
+    for (int r = 0; r < LA; ++r) {
       int ii, kk;
-      if (a_kcontig) { ii = e >> 3; kk = e & 7; } else { kk = e >> 7; ii = e & 127; }
+      a_idx(tid + r * GTHREADS, ii, kk);
       As[buf][kk][ii] = ra[r];
+    }
+#pragma unroll
+    for (int r = 0; r < LB; ++r) {
       int jj, kb;
-      if (b_ncontig) { kb = e >> 7; jj = e & 127; } else { jj = e >> 3; kb = e & 7; }
+      b_idx(tid + r * GTHREADS, jj, kb);
       Bs[buf][kb][jj] = rb[r];
     }
   };
 
   const int tx = tid & 15, ty = tid >> 4;
-  float acc[8][8];
+  float acc[TM][TN];
 #pragma unroll
-  for (int a = 0; a < 8; ++a)
+  for (int a = 0; a < TM; ++a)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+    for (int b = 0; b < TN; ++b) acc[a][b] = 0.f;
 
   if (kbeg < kend) {
     load_slab(kbeg);
@@ -93,16 +108,21 @@ __global__ void __launch_bounds__(GTHREADS) k_gemm_simt(GemmArgs g) {
       if (more) load_slab(k0 + GBK);
 #pragma unroll
       for (int kk = 0; kk < GBK; ++kk) {
-        float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-        float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
-        float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-        float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
-        float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        float av[TM], bv[TN];
 #pragma unroll
-        for (int a = 0; a < 8; ++a)
+        for (int h = 0; h < TM / 4; ++h) {
+          const float4 x = *reinterpret_cast<const float4*>(&As[buf][kk][h * (BM / 2) + ty * 4]);
+          av[4 * h] = x.x; av[4 * h + 1] = x.y; av[4 * h + 2] = x.z; av[4 * h + 3] = x.w;
+        }
 #pragma unroll
-          for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
+        for (int h = 0; h < TN / 4; ++h) {
+          const float4 x = *reinterpret_cast<const float4*>(&Bs[buf][kk][h * (BN / 2) + tx * 4]);
+          bv[4 * h] = x.x; bv[4 * h + 1] = x.y; bv[4 * h + 2] = x.z; bv[4 * h + 3] = x.w;
+        }
+#pragma unroll
+        for (int a = 0; a < TM; ++a)
+#pragma unroll
+          for (int b = 0; b < TN; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
       }
       if (more) {
         store_slab(buf ^ 1);
@@ -112,25 +132,32 @@ __global__ void __launch_bounds__(GTHREADS) k_gemm_simt(GemmArgs g) {
     }
   }
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    int gi = i0 + (a < 4 ? ty * 4 + a : 64 + ty * 4 + a - 4);
+  for (int a = 0; a < TM; ++a) {
+    const int gi = i0 + (a / 4) * (BM / 2) + ty * 4 + (a % 4);
     if (gi >= g.M) continue;
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      int gj = j0 + (b < 4 ? tx * 4 + b : 64 + tx * 4 + b - 4);
+    for (int b = 0; b < TN; ++b) {
+      const int gj = j0 + (b / 4) * (BN / 2) + tx * 4 + (b % 4);
       if (gj >= g.N) continue;
       float* c = g.C + (long long)gi * g.ldc + gj;
-      float v = g.alpha * acc[a][b];
+      const float v = g.alpha * acc[a][b];
       *c = (g.beta == 0.f) ? v : fmaf(g.beta, *c, v);
     }
   }
 }
 
+// Picks 128 x 128 tiles when they fill the GPU, else 64 x 64 tiles.
 template <class TA = float, class TB = float>
 inline int gemm_simt(Ctx* c, const GemmArgs& g) {
   if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
-  dim3 grid((g.N + GBN - 1) / GBN, (g.M + GBM - 1) / GBM);
-  k_gemm_simt<TA, TB><<<grid, GTHREADS, 0, c->stream>>>(g);
+  const long long big = (long long)((g.N + 127) / 128) * ((g.M + 127) / 128);
+  if (big >= 2LL * c->num_sms) {
+    dim3 grid((g.N + 127) / 128, (g.M + 127) / 128);
+    k_gemm_simt<TA, TB, 128, 128><<<grid, GTHREADS, 0, c->stream>>>(g);
+  } else {
+    dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
+    k_gemm_simt<TA, TB, 64, 64><<<grid, GTHREADS, 0, c->stream>>>(g);
+  }
   GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
 }

@@ -12,7 +12,7 @@
 //   U12 = B R22^T            (from B = U12 U22^T)
 //   A - U12 U12^T = U11 U11^T -> (U11, R11) by recursion
 //   R12 = -R11 U12 R22
-// All off-diagonal work is GEMM (fp32, CUDA cores); blocks of <= 64 are factored and
+// All off-diagonal work is GEMM (fp32, CUDA cores); blocks of <= 128 are factored and
 // inverted inside one CTA.  A non-positive or non-finite pivot raises GPTQ_ERR_NOT_PD /
 // GPTQ_ERR_NONFINITE in the device status word (the host retries with more damping).
 #include "kernels.h"
@@ -20,68 +20,96 @@
 
 namespace gptq {
 
-constexpr int FB = 64;
+constexpr int FB = 128;
+constexpr int FB_THREADS = 1024;                       // 32 x 32 threads, 4 x 4 elements each
+constexpr int FB_SMEM = FB * (FB + 1) * 4;
+
+__device__ __forceinline__ float pick4(const float (&v)[4], int k) {
+  return k == 0 ? v[0] : k == 1 ? v[1] : k == 2 ? v[2] : v[3];
+}
 
 // Factor + invert the diagonal block M[s:s+n, s:s+n] (upper triangle read), n <= FB.
 // Writes R = U^{-1} into the upper triangle and zeros below it.
-__global__ void __launch_bounds__(256) k_factor_base(float* __restrict__ M, long long ld, int s,
-                                                      int n, DeviceStatus* st) {
-  __shared__ float A[FB][FB + 1];
-  __shared__ float U[FB][FB + 1];
+__global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ M, long long ld,
+                                                             int s, int n, DeviceStatus* st) {
+  extern __shared__ float fsm[];
+  float(*U)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(fsm);
+  __shared__ float ucol[FB];
+  __shared__ float s_piv;
   __shared__ int bad;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
   if (tid == 0) bad = 0;
-  for (int e = tid; e < FB * FB; e += blockDim.x) {
-    int i = e / FB, k = e % FB;
-    float v = 0.f;
-    if (i < n && k < n) {
-      int a = min(i, k), b = max(i, k);
-      v = M[(long long)(s + a) * ld + s + b];
+  float a[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = 4 * ty + r, k = 4 * tx + c;
+      float v = 0.f;
+      if (i < n && k < n) v = M[(long long)(s + min(i, k)) * ld + s + max(i, k)];
+      a[r][c] = v;
     }
-    A[i][k] = v;
-    U[i][k] = 0.f;
-  }
-  __syncthreads();
-  // reverse Cholesky: H = U U^T, eliminating from the last index
+  // reverse Cholesky H = U U^T, eliminating from the last index; U's column j goes to U[:, j]
   for (int j = n - 1; j >= 0; --j) {
-    float piv = A[j][j];
-    bool good = (piv > 0.f) && isfinite(piv);
+    const int jb = j >> 2, jr = j & 3;
+    if (ty == jb && tx == jb) {
+      float d0[4] = {a[0][0], a[1][1], a[2][2], a[3][3]};
+      s_piv = pick4(d0, jr);
+    }
+    __syncthreads();
+    float piv = s_piv;
+    const bool good = (piv > 0.f) && isfinite(piv);
     if (!good) {
       if (tid == 0 && bad == 0) bad = isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE;
       piv = 1.f;
     }
     const float dj = sqrtf(piv);
-    for (int i = tid; i < j; i += blockDim.x) U[i][j] = A[i][j] / dj;
+    if (tx == jb) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = 4 * ty + r;
+        if (i < j) {
+          const float v = pick4(a[r], jr) / dj;
+          ucol[i] = v;
+          U[i][j] = v;
+        }
+      }
+    }
     if (tid == 0) U[j][j] = dj;
     __syncthreads();
-    const int jj = j * j;
-    for (int e = tid; e < jj; e += blockDim.x) {
-      int i = e / j, k = e - i * j;
-      A[i][k] = fmaf(-U[i][j], U[k][j], A[i][k]);
+    if (4 * ty < j && 4 * tx < j) {
+      float ur[4], uc[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        ur[r] = ucol[4 * ty + r];
+        uc[r] = ucol[4 * tx + r];
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (4 * ty + r < j && 4 * tx + c < j) a[r][c] = fmaf(-ur[r], uc[c], a[r][c]);
     }
-    __syncthreads();
   }
-  // R = U^{-1} (upper), row by row from the bottom; A is reused to hold R.
-  // 4 threads per column c share one dot product.
-  const int c = tid >> 2, part = tid & 3;
+  __syncthreads();
+  // R = U^{-1} (upper), in place in U, row by row from the bottom:
+  // R[i][c] = -(sum_{l=i+1..c} U[i][l] R[l][c]) / U[i][i].  8 threads per column c.
+  const int c = tid >> 3, part = tid & 7;
   for (int i = n - 1; i >= 0; --i) {
     const float uii = U[i][i];
     float acc = 0.f;
-    if (c > i && c < n) {
-      for (int l = i + 1 + part; l <= c; l += 4) acc = fmaf(U[i][l], A[l][c], acc);
-    }
+    if (c > i && c < n)
+      for (int l = i + 1 + part; l <= c; l += 8) acc = fmaf(U[i][l], U[l][c], acc);
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    __syncthreads();  // all reads of row i+1.. done before row i is written
-    if (part == 0 && c < n) {
-      if (c == i) A[i][c] = 1.f / uii;
-      else if (c > i) A[i][c] = -acc / uii;
-    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    __syncthreads();
+    if (part == 0 && c < n && c >= i) U[i][c] = (c == i) ? 1.f / uii : -acc / uii;
     __syncthreads();
   }
-  for (int e = tid; e < n * n; e += blockDim.x) {
-    int i = e / n, k = e % n;
-    M[(long long)(s + i) * ld + s + k] = (k >= i) ? A[i][k] : 0.f;
+  for (int e = tid; e < n * n; e += FB_THREADS) {
+    const int i = e / n, k = e - i * n;
+    M[(long long)(s + i) * ld + s + k] = (k >= i) ? U[i][k] : 0.f;
   }
   if (tid == 0 && bad) raise_error(st, bad, s);
 }
@@ -114,7 +142,7 @@ size_t factor_tmp_floats(int d) {
 static int rec(Ctx* c, float* M, long long ld, int s, int e, float* tmp) {
   const int n = e - s;
   if (n <= FB) {
-    k_factor_base<<<1, 256, 0, c->stream>>>(M, ld, s, n, c->status);
+    k_factor_base<<<1, FB_THREADS, FB_SMEM, c->stream>>>(M, ld, s, n, c->status);
     GPTQ_LAUNCH_CHECK(c);
     return GPTQ_OK;
   }
@@ -144,6 +172,10 @@ static int rec(Ctx* c, float* M, long long ld, int s, int e, float* tmp) {
   return copy2d(c, nullptr, 0, M + (long long)mid * ld + s, ld, n2, n1);
 }
 
-int factor_inverse(Ctx* c, float* M, int d, float* tmp) { return rec(c, M, d, 0, d, tmp); }
+int factor_inverse(Ctx* c, float* M, int d, float* tmp) {
+  GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_factor_base,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, FB_SMEM));
+  return rec(c, M, d, 0, d, tmp);
+}
 
 }  // namespace gptq

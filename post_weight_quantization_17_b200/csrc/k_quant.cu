@@ -114,13 +114,25 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 }
 
 // ------------------------------------------------------------------------------------------
-// a5: one block of up to 128 columns.  One warp per CTA, one row per lane: the lane keeps its
-// row's block in 128 registers, so the sequential chain of a column step (divide, round,
-// clip, residual, η, update of the next column) stays inside the lane.  R's diagonal block
-// is read from shared memory as warp-wide broadcasts.  Global traffic is staged through
-// shared memory so that every global access is a coalesced row segment.
-// Shared memory: R block (64 KB), W/E staging (32 x 129 floats), q staging, code staging.
-constexpr int kColSmem = 128 * 128 * 4 + 2 * 32 * 129 * 4 + 32 * 132;
+// a5: one block of up to 128 columns.  A CTA has 4 warps; each warp owns 32 rows, one row per
+// lane, and keeps its row's block in registers, so the sequential chain of a column step
+// (divide, round, clip, residual, η, update of the next column) stays inside the lane.  R's
+// diagonal block is read from shared memory as warp-wide broadcasts.  R's block and the W
+// block are staged with asynchronous copies (cp.async, all in flight at once); outputs leave
+// through shared memory as coalesced row segments.
+constexpr int kColWarps = 4;
+constexpr int kColWarpSmem = 32 * 129 * 4 + 32 * 65 * 4 + 32 * 132;
+constexpr int kColSmem = 128 * 128 * 4 + kColWarps * kColWarpSmem;
+
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(gsrc),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 
 struct ColStepArgs {
   const float (*Rs)[128];
@@ -167,37 +179,45 @@ __device__ __forceinline__ void col_steps(float (&w)[64], const ColStepArgs& a,
 }
 
 template <bool UNIFORM>
-__global__ void __launch_bounds__(32) k_colblock(
+__global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     float* __restrict__ Wk, int m, int d, int i, int nb, const float* __restrict__ R,
     const float* __restrict__ scales, const int32_t* __restrict__ zeros, int ng,
     const int32_t* __restrict__ gcol, int bits, float* __restrict__ E,
     uint8_t* __restrict__ codes, float* __restrict__ loss_part) {
   extern __shared__ __align__(16) unsigned char smem[];
   float(*Rs)[128] = reinterpret_cast<float(*)[128]>(smem);
-  float(*St)[129] = reinterpret_cast<float(*)[129]>(smem + 128 * 128 * 4);
-  float(*Qs)[129] = reinterpret_cast<float(*)[129]>(smem + 128 * 128 * 4 + 32 * 129 * 4);
-  uint8_t(*Cs)[132] =
-      reinterpret_cast<uint8_t(*)[132]>(smem + 128 * 128 * 4 + 2 * 32 * 129 * 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char* wbase = smem + 128 * 128 * 4 + warp * kColWarpSmem;
+  float(*St)[129] = reinterpret_cast<float(*)[129]>(wbase);
+  float(*Qs)[65] = reinterpret_cast<float(*)[65]>(wbase + 32 * 129 * 4);
+  uint8_t(*Cs)[132] = reinterpret_cast<uint8_t(*)[132]>(wbase + 32 * 129 * 4 + 32 * 65 * 4);
   __shared__ int gs[128];
   __shared__ float rinv[128];
 
-  const int lane = threadIdx.x;
-  const int row0 = blockIdx.x * 32;
+  const int row0 = (blockIdx.x * kColWarps + warp) * 32;  // first row of this warp
   const int row = row0 + lane;
   const bool active = row < m;
+  const bool warp_active = row0 < m;
 
-  for (int e = lane; e < 128 * 128; e += 32) {
+  // asynchronous staging: R's diagonal block (upper triangle) and this warp's W rows
+  for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x) {
     const int a = e >> 7, b = e & 127;
-    Rs[a][b] = (a < nb && b < nb && b >= a) ? R[(long long)(i + a) * d + i + b] : 0.f;
+    const bool v = a < nb && b < nb && b >= a;
+    cp_async4(&Rs[a][b], v ? R + (long long)(i + a) * d + i + b : R, v);
   }
-  for (int a = lane; a < 128; a += 32) gs[a] = (a < nb) ? gcol[i + a] : 0;
   for (int r = 0; r < 32; ++r) {
     const int gr = row0 + r;
-    for (int t = lane; t < 128; t += 32)
-      St[r][t] = (gr < m && t < nb) ? Wk[(long long)gr * d + i + t] : 0.f;
+    for (int t = lane; t < 128; t += 32) {
+      const bool v = gr < m && t < nb;
+      cp_async4(&St[r][t], v ? Wk + (long long)gr * d + i + t : Wk, v);
+    }
   }
-  __syncwarp();
-  for (int a = lane; a < 128; a += 32) rinv[a] = (a < nb) ? 1.f / Rs[a][a] : 0.f;
+  for (int a = threadIdx.x; a < 128; a += blockDim.x) gs[a] = (a < nb) ? gcol[i + a] : 0;
+  cp_async_wait_all();
+  __syncthreads();
+  for (int a = threadIdx.x; a < 128; a += blockDim.x) rinv[a] = (a < nb) ? 1.f / Rs[a][a] : 0.f;
+  __syncthreads();
+  if (!warp_active) return;
 
   ColStepArgs args;
   args.Rs = Rs; args.St = St; args.Cs = Cs; args.gs = gs; args.rinv = rinv;
@@ -228,11 +248,9 @@ __global__ void __launch_bounds__(32) k_colblock(
       for (int t = 0; t < 64; ++t) w[t] = fmaf(-e, Rs[j][64 + t], w[t]);
     }
     col_steps<64, UNIFORM>(w, args, std::make_integer_sequence<int, 64>{});
-#pragma unroll
-    for (int t = 0; t < 64; ++t) Qs[lane][64 + t] = w[t];
   }
   __syncwarp();
-  // E (scaled residuals) and the per-column loss partial Σ_rows η² over this CTA's rows
+  // E (scaled residuals) and the per-column loss partial Σ_rows η² over this warp's rows
   for (int r = 0; r < 32; ++r) {
     const int gr = row0 + r;
     if (gr >= m) break;
@@ -241,13 +259,20 @@ __global__ void __launch_bounds__(32) k_colblock(
   for (int t = lane; t < nb; t += 32) {
     float s = 0.f;
     for (int r = 0; r < 32 && row0 + r < m; ++r) s = fmaf(St[r][t], St[r][t], s);
-    loss_part[(long long)blockIdx.x * d + i + t] = s;
+    loss_part[(long long)(row0 / 32) * d + i + t] = s;
   }
+  __syncwarp();
+  // q of the second half goes to St (E is out), then the block leaves as row segments
+  if (nb > 64) {
+#pragma unroll
+    for (int t = 0; t < 64; ++t) St[lane][64 + t] = w[t];
+  }
+  __syncwarp();
   for (int r = 0; r < 32; ++r) {
     const int gr = row0 + r;
     if (gr >= m) break;
     for (int t = lane; t < nb; t += 32) {
-      Wk[(long long)gr * d + i + t] = Qs[r][t];
+      Wk[(long long)gr * d + i + t] = (t < 64) ? Qs[r][t] : St[r][t];
       codes[(long long)gr * d + i + t] = Cs[r][t];
     }
   }
@@ -260,12 +285,12 @@ int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<false>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
-  const int blocks = (m + 31) / 32;
+  const int blocks = (m + 32 * kColWarps - 1) / (32 * kColWarps);
   if (uniform_grid)
-    k_colblock<true><<<blocks, 32, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
+    k_colblock<true><<<blocks, 32 * kColWarps, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
                                                           gcol, bits, E, codes, loss_part);
   else
-    k_colblock<false><<<blocks, 32, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
+    k_colblock<false><<<blocks, 32 * kColWarps, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
                                                            gcol, bits, E, codes, loss_part);
   GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
