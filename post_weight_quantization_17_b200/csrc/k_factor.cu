@@ -21,15 +21,20 @@
 namespace gptq {
 
 constexpr int FB = 128;
-constexpr int FB_THREADS = 1024;                       // 32 x 32 threads, 4 x 4 elements each
+constexpr int FB_THREADS = 256;                        // 16 x 16 threads, 8 x 8 elements each
 constexpr int FB_SMEM = FB * (FB + 1) * 4;
 
-__device__ __forceinline__ float pick4(const float (&v)[4], int k) {
-  return k == 0 ? v[0] : k == 1 ? v[1] : k == 2 ? v[2] : v[3];
+template <int N>
+__device__ __forceinline__ float pick(const float (&v)[N], int k) {
+  float r = v[0];
+#pragma unroll
+  for (int t = 1; t < N; ++t) r = (k == t) ? v[t] : r;
+  return r;
 }
 
 // Factor + invert the diagonal block M[s:s+n, s:s+n] (upper triangle read), n <= FB.
-// Writes R = U^{-1} into the upper triangle and zeros below it.
+// Writes R = U^{-1} into the upper triangle and zeros below it.  Thread (ty, tx) holds rows
+// 8 ty .. 8 ty + 7 and columns 8 tx .. 8 tx + 7 of the symmetric block in registers.
 __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ M, long long ld,
                                                              int s, int n, DeviceStatus* st) {
   extern __shared__ float fsm[];
@@ -37,24 +42,26 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
   __shared__ float ucol[FB];
   __shared__ float s_piv;
   __shared__ int bad;
-  const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   if (tid == 0) bad = 0;
-  float a[4][4];
+  float a[8][8];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = 4 * ty + r, k = 4 * tx + c;
+    for (int c = 0; c < 8; ++c) {
+      const int i = 8 * ty + r, k = 8 * tx + c;
       float v = 0.f;
       if (i < n && k < n) v = M[(long long)(s + min(i, k)) * ld + s + max(i, k)];
       a[r][c] = v;
     }
   // reverse Cholesky H = U U^T, eliminating from the last index; U's column j goes to U[:, j]
   for (int j = n - 1; j >= 0; --j) {
-    const int jb = j >> 2, jr = j & 3;
+    const int jb = j >> 3, jr = j & 7;
     if (ty == jb && tx == jb) {
-      float d0[4] = {a[0][0], a[1][1], a[2][2], a[3][3]};
-      s_piv = pick4(d0, jr);
+      float dg[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) dg[t] = a[t][t];
+      s_piv = pick(dg, jr);
     }
     __syncthreads();
     float piv = s_piv;
@@ -66,10 +73,10 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
     const float dj = sqrtf(piv);
     if (tx == jb) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = 4 * ty + r;
+      for (int r = 0; r < 8; ++r) {
+        const int i = 8 * ty + r;
         if (i < j) {
-          const float v = pick4(a[r], jr) / dj;
+          const float v = pick(a[r], jr) / dj;
           ucol[i] = v;
           U[i][j] = v;
         }
@@ -77,32 +84,37 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
     }
     if (tid == 0) U[j][j] = dj;
     __syncthreads();
-    if (4 * ty < j && 4 * tx < j) {
-      float ur[4], uc[4];
+    if (8 * ty < j && 8 * tx < j) {
+      float ur[8], uc[8];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        ur[r] = ucol[4 * ty + r];
-        uc[r] = ucol[4 * tx + r];
+      for (int r = 0; r < 8; ++r) {
+        ur[r] = ucol[8 * ty + r];
+        uc[r] = ucol[8 * tx + r];
       }
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (4 * ty + r < j && 4 * tx + c < j) a[r][c] = fmaf(-ur[r], uc[c], a[r][c]);
+        for (int c = 0; c < 8; ++c)
+          if (8 * ty + r < j && 8 * tx + c < j) a[r][c] = fmaf(-ur[r], uc[c], a[r][c]);
     }
   }
   __syncthreads();
   // R = U^{-1} (upper), in place in U, row by row from the bottom:
-  // R[i][c] = -(sum_{l=i+1..c} U[i][l] R[l][c]) / U[i][i].  8 threads per column c.
-  const int c = tid >> 3, part = tid & 7;
+  // R[i][c] = -(sum_{l=i+1..c} U[i][l] R[l][c]) / U[i][i].  2 threads per column c.
+  const int c = tid >> 1, part = tid & 1;
   for (int i = n - 1; i >= 0; --i) {
     const float uii = U[i][i];
-    float acc = 0.f;
-    if (c > i && c < n)
-      for (int l = i + 1 + part; l <= c; l += 8) acc = fmaf(U[i][l], U[l][c], acc);
+    float acc0 = 0.f, acc1 = 0.f;
+    if (c > i && c < n) {
+      int l = i + 1 + part;
+      for (; l + 2 <= c; l += 4) {
+        acc0 = fmaf(U[i][l], U[l][c], acc0);
+        acc1 = fmaf(U[i][l + 2], U[l + 2][c], acc1);
+      }
+      if (l <= c) acc0 = fmaf(U[i][l], U[l][c], acc0);
+    }
+    float acc = acc0 + acc1;
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
     __syncthreads();
     if (part == 0 && c < n && c >= i) U[i][c] = (c == i) ? 1.f / uii : -acc / uii;
     __syncthreads();

@@ -115,13 +115,17 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 
 // ------------------------------------------------------------------------------------------
 // a5: one block of up to 128 columns.  A CTA has 4 warps; each warp owns 32 rows, one row per
-// lane, and keeps its row's block in registers, so the sequential chain of a column step
-// (divide, round, clip, residual, η, update of the next column) stays inside the lane.  R's
-// diagonal block is read from shared memory as warp-wide broadcasts.  R's block and the W
+// lane.  The block is walked in four 32-column sub-blocks whose values stay in registers, so
+// the sequential chain of a column step (divide, round, clip, residual, η, update of the next
+// column) stays inside the lane; a sub-block first receives the residuals of the sub-blocks
+// before it (E R, the lazy update of [T] eq.(46) at a finer grain, exact by eq.(47)-(49)).
+// Only one 32-step body is unrolled, which keeps the kernel inside the instruction cache.
+// R's diagonal block is read from shared memory as warp-wide broadcasts; R's block and the W
 // block are staged with asynchronous copies (cp.async, all in flight at once); outputs leave
 // through shared memory as coalesced row segments.
 constexpr int kColWarps = 4;
-constexpr int kColWarpSmem = 32 * 129 * 4 + 32 * 65 * 4 + 32 * 132;
+constexpr int kColSub = 32;
+constexpr int kColWarpSmem = 32 * 129 * 4 + 32 * 132;
 constexpr int kColSmem = 128 * 128 * 4 + kColWarps * kColWarpSmem;
 
 __device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool valid) {
@@ -148,11 +152,11 @@ struct ColStepArgs {
   float maxq, D0, Z0;
 };
 
-// One column step; block column OFF + J, with J compile-time so that w[] stays in registers.
-// Only the columns of the same half (J+1 .. 63) are updated immediately.
-template <int J, int OFF, bool UNIFORM>
-__device__ __forceinline__ void col_step(float (&w)[64], const ColStepArgs& a) {
-  constexpr int C = OFF + J;
+// One column step at block column off + J (J compile-time so that w[] stays in registers);
+// the sub-block's later columns (J+1 .. 31) are updated immediately.
+template <int J, bool UNIFORM>
+__device__ __forceinline__ void col_step(float (&w)[kColSub], const ColStepArgs& a, int off) {
+  const int C = off + J;
   if (C < a.nb) {
     float Dj = a.D0, Zj = a.Z0;
     if (!UNIFORM && a.active) {
@@ -167,15 +171,16 @@ __device__ __forceinline__ void col_step(float (&w)[64], const ColStepArgs& a) {
     a.Cs[a.lane][C] = (uint8_t)cq;
     a.St[a.lane][C] = eta;
     w[J] = q;
+    const float* rrow = &a.Rs[C][off];
 #pragma unroll
-    for (int k = J + 1; k < 64; ++k) w[k] = fmaf(-eta, a.Rs[C][OFF + k], w[k]);
+    for (int k = J + 1; k < kColSub; ++k) w[k] = fmaf(-eta, rrow[k], w[k]);
   }
 }
 
-template <int OFF, bool UNIFORM, int... Js>
-__device__ __forceinline__ void col_steps(float (&w)[64], const ColStepArgs& a,
+template <bool UNIFORM, int... Js>
+__device__ __forceinline__ void col_steps(float (&w)[kColSub], const ColStepArgs& a, int off,
                                           std::integer_sequence<int, Js...>) {
-  (col_step<Js, OFF, UNIFORM>(w, a), ...);
+  (col_step<Js, UNIFORM>(w, a, off), ...);
 }
 
 template <bool UNIFORM>
@@ -188,9 +193,9 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
   float(*Rs)[128] = reinterpret_cast<float(*)[128]>(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* wbase = smem + 128 * 128 * 4 + warp * kColWarpSmem;
+  // St: the W block on entry, then column by column η (scaled residual) replaces w
   float(*St)[129] = reinterpret_cast<float(*)[129]>(wbase);
-  float(*Qs)[65] = reinterpret_cast<float(*)[65]>(wbase + 32 * 129 * 4);
-  uint8_t(*Cs)[132] = reinterpret_cast<uint8_t(*)[132]>(wbase + 32 * 129 * 4 + 32 * 65 * 4);
+  uint8_t(*Cs)[132] = reinterpret_cast<uint8_t(*)[132]>(wbase + 32 * 129 * 4);
   __shared__ int gs[128];
   __shared__ float rinv[128];
 
@@ -230,24 +235,25 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     args.D0 = scales[args.srow + gs[0]];
     args.Z0 = (float)zeros[args.srow + gs[0]];
   }
-  float w[64];
-  // first half: columns 0..63
+  float qkeep[128 / kColSub][kColSub];  // q of finished sub-blocks (registers: static index)
 #pragma unroll
-  for (int t = 0; t < 64; ++t) w[t] = St[lane][t];
-  __syncwarp();
-  col_steps<0, UNIFORM>(w, args, std::make_integer_sequence<int, 64>{});
+  for (int sb = 0; sb < 128 / kColSub; ++sb) {
+    const int off = sb * kColSub;
+    if (off < nb) {
+      float w[kColSub];
 #pragma unroll
-  for (int t = 0; t < 64; ++t) Qs[lane][t] = w[t];
-  if (nb > 64) {
-    // second half: receive the first half's residuals (E[:, 0:64] R[0:64, 64:128]) first
+      for (int t = 0; t < kColSub; ++t) w[t] = St[lane][off + t];
+      // residuals of the earlier sub-blocks: w -= η[0:off] R[0:off, off:off+32]
+      for (int j = 0; j < off; ++j) {
+        const float e = St[lane][j];
+        const float* rrow = &Rs[j][off];
 #pragma unroll
-    for (int t = 0; t < 64; ++t) w[t] = St[lane][64 + t];
-    for (int j = 0; j < 64; ++j) {
-      const float e = St[lane][j];
+        for (int t = 0; t < kColSub; ++t) w[t] = fmaf(-e, rrow[t], w[t]);
+      }
+      col_steps<UNIFORM>(w, args, off, std::make_integer_sequence<int, kColSub>{});
 #pragma unroll
-      for (int t = 0; t < 64; ++t) w[t] = fmaf(-e, Rs[j][64 + t], w[t]);
+      for (int t = 0; t < kColSub; ++t) qkeep[sb][t] = w[t];
     }
-    col_steps<64, UNIFORM>(w, args, std::make_integer_sequence<int, 64>{});
   }
   __syncwarp();
   // E (scaled residuals) and the per-column loss partial Σ_rows η² over this warp's rows
@@ -262,17 +268,17 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     loss_part[(long long)(row0 / 32) * d + i + t] = s;
   }
   __syncwarp();
-  // q of the second half goes to St (E is out), then the block leaves as row segments
-  if (nb > 64) {
+  // q replaces η in St, then the block leaves as row segments
 #pragma unroll
-    for (int t = 0; t < 64; ++t) St[lane][64 + t] = w[t];
-  }
+  for (int sb = 0; sb < 128 / kColSub; ++sb)
+#pragma unroll
+    for (int t = 0; t < kColSub; ++t) St[lane][sb * kColSub + t] = qkeep[sb][t];
   __syncwarp();
   for (int r = 0; r < 32; ++r) {
     const int gr = row0 + r;
     if (gr >= m) break;
     for (int t = lane; t < nb; t += 32) {
-      Wk[(long long)gr * d + i + t] = (t < 64) ? Qs[r][t] : St[r][t];
+      Wk[(long long)gr * d + i + t] = St[r][t];
       codes[(long long)gr * d + i + t] = Cs[r][t];
     }
   }
