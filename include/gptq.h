@@ -131,6 +131,32 @@ int gptq_quantize_layer(gptq_ctx* ctx, const void* W, int w_dtype, int64_t m, in
                         int group, int block, int grid_given, float* scales, int32_t* zeros,
                         uint8_t* codes, float* W_hat, float* col_loss);
 
+/* Size of the fixed device scratch used by gptq_quantize_layer_noalloc. */
+#define GPTQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* gptq_quantize_layer for callers that cannot allocate device memory — for example code that
+ * runs inside another allocator's hooks, or a process whose device memory is fully committed
+ * before it loads this library.  It takes no context and no workspace: its scratch is one
+ * file-scope device array of GPTQ_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU loading the
+ * library holds until the process exits.  It calls no cudaMalloc, cudaFree or allocating
+ * library routine.  The pages have no counterpart; the arithmetic is that of
+ * gptq_quantize_layer.
+ *   cuda_stream  the cudaStream_t to enqueue on (NULL = legacy default stream), current device.
+ *   other arguments exactly as for gptq_quantize_layer.
+ * The scratch must hold about 4 m (128 + d / 32) + 12 d bytes, plus 5 m d bytes when perm is
+ * not NULL; a layer that needs more returns GPTQ_ERR_ARG (the only work enqueued then clears
+ * the scratch's status word).  The
+ * first call on a device looks up the array's device address (cudaGetSymbolAddress) and should
+ * come before any stream capture.  The call synchronizes `cuda_stream` and returns the device
+ * status (GPTQ_OK or GPTQ_ERR_NONFINITE) like gptq_sync_status.  Every call shares the one
+ * array and it keeps the last call's contents: calls whose work overlaps on the GPU (other
+ * streams or host threads) race and must be serialized by the caller. */
+int gptq_quantize_layer_noalloc(void* cuda_stream, const void* W, int w_dtype, int64_t m,
+                                int64_t d, const float* R, const int32_t* perm,
+                                const uint8_t* dead, int bits, int group, int block,
+                                int grid_given, float* scales, int32_t* zeros, uint8_t* codes,
+                                float* W_hat, float* col_loss);
+
 /* Dense packing of the codes ([T] §3.1 output table, §9.4: about m d b / 8 bytes, stored as
  * 32-bit words).  Layout: per row a little-endian bitstream in which code k occupies bits
  * [b k, b k + b); word w of the row holds stream bits [32 w, 32 w + 32); every row starts on

@@ -52,6 +52,8 @@ _SIGS = {
                                  ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_i32)]),
     "gptq_quantize_layer": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i32, _i32, _i32,
                                    _i32, _vp, _vp, _vp, _vp, _vp]),
+    "gptq_quantize_layer_noalloc": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _vp, _vp, _i32, _i32,
+                                           _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "gptq_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
     "gptq_unpack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
 }
@@ -169,6 +171,20 @@ def gptq_quantize_layer(ctx: Context, W, R, perm, dead, bits: int, group: int, b
                                   1 if grid_given else 0, _ptr(scales), _ptr(zeros), _ptr(codes),
                                   _ptr(W_hat), _ptr(col_loss))
     ctx.check(rc, "gptq_quantize_layer")
+
+
+def gptq_quantize_layer_noalloc(W, R, perm, dead, bits: int, group: int, block: int,
+                                grid_given: bool, scales, zeros, codes, W_hat, col_loss,
+                                stream=None) -> int:
+    """gptq_quantize_layer without a context or workspace (fixed device scratch inside the
+    library); synchronizes the stream and returns the status code (0 = OK)."""
+    m, d = W.shape
+    _dev(W, name="W")
+    s = stream if stream is not None else torch.cuda.current_stream(W.device)
+    return int(_lib.gptq_quantize_layer_noalloc(
+        ctypes.c_void_p(s.cuda_stream), _ptr(W), _DTYPE_CODE[W.dtype], m, d, _ptr(R), _ptr(perm),
+        _ptr(dead), bits, group, block, 1 if grid_given else 0, _ptr(scales), _ptr(zeros),
+        _ptr(codes), _ptr(W_hat), _ptr(col_loss)))
 
 
 def gptq_pack(ctx: Context, codes, bits: int, packed):
