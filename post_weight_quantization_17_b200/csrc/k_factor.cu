@@ -20,108 +20,130 @@
 
 namespace gptq {
 
-constexpr int FB = 128;
-constexpr int FB_THREADS = 256;                        // 16 x 16 threads, 8 x 8 elements each
-constexpr int FB_SMEM = FB * (FB + 1) * 4;
-
-template <int N>
-__device__ __forceinline__ float pick(const float (&v)[N], int k) {
-  float r = v[0];
-#pragma unroll
-  for (int t = 1; t < N; ++t) r = (k == t) ? v[t] : r;
-  return r;
-}
+constexpr int FB = 128;                 // diagonal block factored inside one CTA
+constexpr int FP = 32;                  // panel width (one warp factors a panel's diagonal)
+constexpr int FB_THREADS = 256;
+// shared memory: A (the block, then U and R), the current panel, the diagonal inverses, T
+constexpr int FB_SMEM = (FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
+                         FP * (FB + 1)) * 4;
 
 // Factor + invert the diagonal block M[s:s+n, s:s+n] (upper triangle read), n <= FB.
-// Writes R = U^{-1} into the upper triangle and zeros below it.  Thread (ty, tx) holds rows
-// 8 ty .. 8 ty + 7 and columns 8 tx .. 8 tx + 7 of the symmetric block in registers.
+// Writes R = U^{-1} into the upper triangle and zeros below it.
+//
+// Blocked reverse Cholesky over four 32-column panels, last panel first:
+//   (a) one warp factors the panel's 32 x 32 diagonal block D = U_PP U_PP^T in registers
+//       (lane l holds row l; pivots and columns travel by shuffles) and inverts U_PP;
+//   (b) the rows above get their U panel U[0:p0, P] = A[0:p0, P] U_PP^{-T};
+//   (c) the rows above are updated, A[0:p0, 0:p0] -= U[0:p0, P] U[0:p0, P]^T.
+// Then R block row by block row, from the bottom: R[P, >P] = -R_PP (U[P, >P] R[>P, >P]).
+// Indices >= n are padded with the identity, which factors to itself without coupling.
 __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ M, long long ld,
                                                              int s, int n, DeviceStatus* st) {
   extern __shared__ float fsm[];
-  float(*U)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(fsm);
-  __shared__ float ucol[FB];
-  __shared__ float s_piv;
+  float(*A)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(fsm);
+  float(*Pn)[FP + 1] = reinterpret_cast<float(*)[FP + 1]>(fsm + FB * (FB + 1));
+  float(*Rd)[FP][FP + 1] =
+      reinterpret_cast<float(*)[FP][FP + 1]>(fsm + FB * (FB + 1) + (FB - FP) * (FP + 1));
+  float(*T)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(
+      fsm + FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1));
   __shared__ int bad;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tx = tid & 15, ty = tid >> 4;
   if (tid == 0) bad = 0;
-  float a[8][8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const int i = 8 * ty + r, k = 8 * tx + c;
-      float v = 0.f;
-      if (i < n && k < n) v = M[(long long)(s + min(i, k)) * ld + s + max(i, k)];
-      a[r][c] = v;
-    }
-  // reverse Cholesky H = U U^T, eliminating from the last index; U's column j goes to U[:, j]
-  for (int j = n - 1; j >= 0; --j) {
-    const int jb = j >> 3, jr = j & 7;
-    if (ty == jb && tx == jb) {
-      float dg[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) dg[t] = a[t][t];
-      s_piv = pick(dg, jr);
-    }
-    __syncthreads();
-    float piv = s_piv;
-    const bool good = (piv > 0.f) && isfinite(piv);
-    if (!good) {
-      if (tid == 0 && bad == 0) bad = isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE;
-      piv = 1.f;
-    }
-    const float dj = sqrtf(piv);
-    if (tx == jb) {
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int i = 8 * ty + r;
-        if (i < j) {
-          const float v = pick(a[r], jr) / dj;
-          ucol[i] = v;
-          U[i][j] = v;
-        }
-      }
-    }
-    if (tid == 0) U[j][j] = dj;
-    __syncthreads();
-    if (8 * ty < j && 8 * tx < j) {
-      float ur[8], uc[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        ur[r] = ucol[8 * ty + r];
-        uc[r] = ucol[8 * tx + r];
-      }
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          if (8 * ty + r < j && 8 * tx + c < j) a[r][c] = fmaf(-ur[r], uc[c], a[r][c]);
-    }
+  for (int e = tid; e < FB * FB; e += FB_THREADS) {
+    const int i = e >> 7, k = e & 127;
+    float v = (i == k) ? 1.f : 0.f;
+    if (i < n && k < n) v = M[(long long)(s + min(i, k)) * ld + s + max(i, k)];
+    A[i][k] = v;
   }
   __syncthreads();
-  // R = U^{-1} (upper), in place in U, row by row from the bottom:
-  // R[i][c] = -(sum_{l=i+1..c} U[i][l] R[l][c]) / U[i][i].  2 threads per column c.
-  const int c = tid >> 1, part = tid & 1;
-  for (int i = n - 1; i >= 0; --i) {
-    const float uii = U[i][i];
-    float acc0 = 0.f, acc1 = 0.f;
-    if (c > i && c < n) {
-      int l = i + 1 + part;
-      for (; l + 2 <= c; l += 4) {
-        acc0 = fmaf(U[i][l], U[l][c], acc0);
-        acc1 = fmaf(U[i][l + 2], U[l + 2][c], acc1);
+
+  for (int P = FB / FP - 1; P >= 0; --P) {
+    const int p0 = P * FP;
+    if (warp == 0) {
+      float dr[FP], u[FP], r[FP];
+#pragma unroll
+      for (int k = 0; k < FP; ++k) dr[k] = A[p0 + lane][p0 + k];
+      // (a) D = U_PP U_PP^T, eliminating from the last index; lane l keeps row l of U_PP
+#pragma unroll
+      for (int jj = FP - 1; jj >= 0; --jj) {
+        float piv = __shfl_sync(0xffffffffu, dr[jj], jj);
+        const bool good = (piv > 0.f) && isfinite(piv);
+        if (!good) {
+          if (lane == 0 && bad == 0) bad = isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE;
+          piv = 1.f;
+        }
+        const float dj = sqrtf(piv);
+        const float uj = (lane < jj) ? dr[jj] / dj : (lane == jj ? dj : 0.f);
+        u[jj] = uj;
+#pragma unroll
+        for (int k = 0; k < jj; ++k) dr[k] = fmaf(-uj, __shfl_sync(0xffffffffu, uj, k), dr[k]);
       }
-      if (l <= c) acc0 = fmaf(U[i][l], U[l][c], acc0);
+      // U_PP^{-1}: lane c computes column c, rows from the bottom
+#pragma unroll
+      for (int i = FP - 1; i >= 0; --i) {
+        const float uii = __shfl_sync(0xffffffffu, u[i], i);
+        float acc = 0.f;
+#pragma unroll
+        for (int l = i + 1; l < FP; ++l) acc = fmaf(__shfl_sync(0xffffffffu, u[l], i), r[l], acc);
+        r[i] = (lane == i) ? 1.f / uii : (lane > i ? -acc / uii : 0.f);
+      }
+#pragma unroll
+      for (int i = 0; i < FP; ++i) Rd[P][i][lane] = r[i];
     }
-    float acc = acc0 + acc1;
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     __syncthreads();
-    if (part == 0 && c < n && c >= i) U[i][c] = (c == i) ? 1.f / uii : -acc / uii;
+    if (p0 > 0) {
+      // (b) U panel of the rows above: Pn[i][c] = sum_{k >= c} A[i][p0 + k] Rd[c][k]
+      for (int e = tid; e < p0 * FP; e += FB_THREADS) {
+        const int i = e >> 5, c = e & 31;
+        float acc = 0.f;
+        for (int k = c; k < FP; ++k) acc = fmaf(A[i][p0 + k], Rd[P][c][k], acc);
+        Pn[i][c] = acc;
+      }
+      __syncthreads();
+      for (int e = tid; e < p0 * FP; e += FB_THREADS) {
+        const int i = e >> 5, c = e & 31;
+        A[i][p0 + c] = Pn[i][c];
+      }
+      // (c) A[0:p0, 0:p0] -= Pn Pn^T
+      for (int i = ty; i < p0; i += 16)
+        for (int k = tx; k < p0; k += 16) {
+          float acc = A[i][k];
+#pragma unroll 8
+          for (int c = 0; c < FP; ++c) acc = fmaf(-Pn[i][c], Pn[k][c], acc);
+          A[i][k] = acc;
+        }
+      __syncthreads();
+    }
+  }
+  // R: diagonal blocks from the panel inverses, then block rows from the bottom
+  for (int e = tid; e < FB * FP; e += FB_THREADS) {
+    const int P = e / (FP * FP), i = (e / FP) % FP, k = e % FP;
+    A[P * FP + i][P * FP + k] = (k >= i) ? Rd[P][i][k] : 0.f;
+  }
+  __syncthreads();
+  for (int P = FB / FP - 2; P >= 0; --P) {
+    const int p0 = P * FP, c0 = p0 + FP, nc = FB - c0;
+    // T[r][c'] = sum_{l = c0..c'} U[p0 + r][l] R[l][c']
+    for (int e = tid; e < FP * nc; e += FB_THREADS) {
+      const int rr = e & 31, cc = c0 + (e >> 5);
+      float acc = 0.f;
+      for (int l = c0; l <= cc; ++l) acc = fmaf(A[p0 + rr][l], A[l][cc], acc);
+      T[rr][cc] = acc;
+    }
+    __syncthreads();
+    // R[p0 + r][c'] = -sum_{k >= r} Rd[P][r][k] T[k][c']
+    for (int e = tid; e < FP * nc; e += FB_THREADS) {
+      const int rr = e & 31, cc = c0 + (e >> 5);
+      float acc = 0.f;
+      for (int k = rr; k < FP; ++k) acc = fmaf(Rd[P][rr][k], T[k][cc], acc);
+      A[p0 + rr][cc] = -acc;
+    }
     __syncthreads();
   }
   for (int e = tid; e < n * n; e += FB_THREADS) {
     const int i = e / n, k = e - i * n;
-    M[(long long)(s + i) * ld + s + k] = (k >= i) ? U[i][k] : 0.f;
+    M[(long long)(s + i) * ld + s + k] = (k >= i) ? A[i][k] : 0.f;
   }
   if (tid == 0 && bad) raise_error(st, bad, s);
 }

@@ -125,7 +125,7 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 // through shared memory as coalesced row segments.
 constexpr int kColWarps = 4;
 constexpr int kColSub = 32;
-constexpr int kColWarpSmem = 32 * 129 * 4 + 32 * 132;
+constexpr int kColWarpSmem = 2 * 32 * 129 * 4 + 32 * 132;
 constexpr int kColSmem = 128 * 128 * 4 + kColWarps * kColWarpSmem;
 
 __device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool valid) {
@@ -195,7 +195,8 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
   unsigned char* wbase = smem + 128 * 128 * 4 + warp * kColWarpSmem;
   // St: the W block on entry, then column by column η (scaled residual) replaces w
   float(*St)[129] = reinterpret_cast<float(*)[129]>(wbase);
-  uint8_t(*Cs)[132] = reinterpret_cast<uint8_t(*)[132]>(wbase + 32 * 129 * 4);
+  float(*Qs)[129] = reinterpret_cast<float(*)[129]>(wbase + 32 * 129 * 4);  // q per column
+  uint8_t(*Cs)[132] = reinterpret_cast<uint8_t(*)[132]>(wbase + 2 * 32 * 129 * 4);
   __shared__ int gs[128];
   __shared__ float rinv[128];
 
@@ -235,8 +236,7 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     args.D0 = scales[args.srow + gs[0]];
     args.Z0 = (float)zeros[args.srow + gs[0]];
   }
-  float qkeep[128 / kColSub][kColSub];  // q of finished sub-blocks (registers: static index)
-#pragma unroll
+#pragma unroll 1
   for (int sb = 0; sb < 128 / kColSub; ++sb) {
     const int off = sb * kColSub;
     if (off < nb) {
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
       }
       col_steps<UNIFORM>(w, args, off, std::make_integer_sequence<int, kColSub>{});
 #pragma unroll
-      for (int t = 0; t < kColSub; ++t) qkeep[sb][t] = w[t];
+      for (int t = 0; t < kColSub; ++t) Qs[lane][off + t] = w[t];
     }
   }
   __syncwarp();
@@ -268,17 +268,11 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     loss_part[(long long)(row0 / 32) * d + i + t] = s;
   }
   __syncwarp();
-  // q replaces η in St, then the block leaves as row segments
-#pragma unroll
-  for (int sb = 0; sb < 128 / kColSub; ++sb)
-#pragma unroll
-    for (int t = 0; t < kColSub; ++t) St[lane][sb * kColSub + t] = qkeep[sb][t];
-  __syncwarp();
   for (int r = 0; r < 32; ++r) {
     const int gr = row0 + r;
     if (gr >= m) break;
     for (int t = lane; t < nb; t += 32) {
-      Wk[(long long)gr * d + i + t] = St[r][t];
+      Wk[(long long)gr * d + i + t] = Qs[r][t];
       codes[(long long)gr * d + i + t] = Cs[r][t];
     }
   }
