@@ -50,12 +50,18 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tx = tid & 15, ty = tid >> 4;
   if (tid == 0) bad = 0;
+  // asynchronous load of the block (all copies in flight), identity padding beyond n
   for (int e = tid; e < FB * FB; e += FB_THREADS) {
     const int i = e >> 7, k = e & 127;
-    float v = (i == k) ? 1.f : 0.f;
-    if (i < n && k < n) v = M[(long long)(s + min(i, k)) * ld + s + max(i, k)];
-    A[i][k] = v;
+    if (i < n && k < n) {
+      const float* src = M + (long long)(s + min(i, k)) * ld + s + max(i, k);
+      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&A[i][k]));
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+    } else {
+      A[i][k] = (i == k) ? 1.f : 0.f;
+    }
   }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
   for (int P = FB / FP - 1; P >= 0; --P) {
