@@ -162,4 +162,8 @@ inline int gemm_simt(Ctx* c, const GemmArgs& g) {
   return GPTQ_OK;
 }
 
+// fp32-accurate GEMM: tcgen05 3xTF32 where TMA can take the operands, else CUDA cores
+// (k_gemm_tc.cu).
+int gemm_f32(Ctx* c, const GemmArgs& g);
+
 }  // namespace gptq

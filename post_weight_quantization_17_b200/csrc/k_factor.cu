@@ -12,7 +12,7 @@
 //   U12 = B R22^T            (from B = U12 U22^T)
 //   A - U12 U12^T = U11 U11^T -> (U11, R11) by recursion
 //   R12 = -R11 U12 R22
-// All off-diagonal work is GEMM (fp32, CUDA cores); blocks of <= 128 are factored and
+// All off-diagonal work is fp32-accurate GEMM (tcgen05 3xTF32); blocks of <= 128 are factored and
 // inverted inside one CTA.  A non-positive or non-finite pivot raises GPTQ_ERR_NOT_PD /
 // GPTQ_ERR_NONFINITE in the device status word (the host retries with more damping).
 #include "kernels.h"
@@ -196,18 +196,18 @@ static int rec(Ctx* c, float* M, long long ld, int s, int e, float* tmp) {
   float* Ablk = M + (long long)s * ld + s;
   // U12 = B R22^T  (opB(k,j) = R22[j][k], zero for k < j)
   GemmArgs g{n1, n2, n2, Bblk, ld, 1, R22, 1, ld, tmp, n2, 1.f, 0.f, kBLower};
-  if ((rc = gemm_simt(c, g))) return rc;
+  if ((rc = gemm_f32(c, g))) return rc;
   if ((rc = copy2d(c, tmp, n2, Bblk, ld, n1, n2))) return rc;
   // A' = A - U12 U12^T  (upper tiles only)
   GemmArgs g2{n1, n1, n2, tmp, n2, 1, tmp, 1, n2, Ablk, ld, -1.f, 1.f, kCUpper};
-  if ((rc = gemm_simt(c, g2))) return rc;
+  if ((rc = gemm_f32(c, g2))) return rc;
   if ((rc = rec(c, M, ld, s, mid, tmp))) return rc;
   // T2 = U12 R22  (R22(k,j) = 0 for k > j)
   GemmArgs g3{n1, n2, n2, Bblk, ld, 1, R22, ld, 1, tmp, n2, 1.f, 0.f, kBUpper};
-  if ((rc = gemm_simt(c, g3))) return rc;
+  if ((rc = gemm_f32(c, g3))) return rc;
   // R12 = -R11 T2  (R11(i,k) = 0 for k < i)
   GemmArgs g4{n1, n2, n1, Ablk, ld, 1, tmp, n2, 1, Bblk, ld, -1.f, 0.f, kAUpper};
-  if ((rc = gemm_simt(c, g4))) return rc;
+  if ((rc = gemm_f32(c, g4))) return rc;
   // strict lower block of this level
   return copy2d(c, nullptr, 0, M + (long long)mid * ld + s, ld, n2, n1);
 }

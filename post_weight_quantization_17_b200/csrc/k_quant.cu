@@ -304,7 +304,7 @@ int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int nb, const float*
   int rc;
   GemmArgs g{m, n, nb, E, kColMax, 1, R + (long long)i * d + i + nb, d, 1,
              Wk + i + nb, d, -1.f, 1.f, 0};
-  if ((rc = gemm_simt(c, g))) return rc;
+  if ((rc = gemm_f32(c, g))) return rc;
   return GPTQ_OK;
 }
 
