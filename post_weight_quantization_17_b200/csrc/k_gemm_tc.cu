@@ -10,7 +10,8 @@
 // core's accumulation over many MMAs loses low bits, so partial sums of KP = 128 k-elements are
 // taken from TMEM and added in fp32 into a register accumulator by the epilogue warps.
 //   warp 0       TMA producer: A box 128 x 32, B box 128 x 32 (K-major) or 4 x (32 x 32)
-//                (N-major), 128-byte swizzle, 3-stage ring
+//                (N-major), 128-byte swizzle (32-byte atoms for the N-major tf32 operand, the
+//                only smem layout the tensor core takes for it), 3-stage ring
 //   warps 2..5   split: tf32 hi in place, lo into its own buffer (same swizzled layout),
 //                then fence.proxy.async so the tensor core sees the writes
 //   warp 1       MMA issuer, M = N = 128, K = 8 per instruction, two TMEM accumulators
@@ -178,8 +179,9 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
               const uint64_t dal = tc::sdesc_sw128(alo + kk * 32, 16, 1024);
               uint64_t dbh, dbl;
               if (p.b_nmajor) {
-                dbh = tc::sdesc_sw128(bhi + kk * 1024, GT_TILE_BYTES / 4, 1024);
-                dbl = tc::sdesc_sw128(blo + kk * 1024, GT_TILE_BYTES / 4, 1024);
+                // MN-major tf32: 32-element atoms along N every 4 KB, 4-row K atoms of 512 B
+                dbh = tc::sdesc_sw128_32b(bhi + kk * 1024, GT_TILE_BYTES / 4, 512);
+                dbl = tc::sdesc_sw128_32b(blo + kk * 1024, GT_TILE_BYTES / 4, 512);
               } else {
                 dbh = tc::sdesc_sw128(bhi + kk * 32, 16, 1024);
                 dbl = tc::sdesc_sw128(blo + kk * 32, 16, 1024);
@@ -326,7 +328,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 static bool make_map_f32(CUtensorMap* map, const void* base, long long inner, long long outer,
-                         long long ld, int box_inner, int box_outer) {
+                         long long ld, int box_inner, int box_outer, CUtensorMapSwizzle swz) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
@@ -334,8 +336,7 @@ static bool make_map_f32(CUtensorMap* map, const void* base, long long inner, lo
   cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
   cuuint32_t es[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
 
@@ -354,10 +355,12 @@ bool gemm_tc_applies(const GemmArgs& g) {
 int gemm_tc(Ctx* c, const GemmArgs& g) {
   CUtensorMap ma, mb;
   const bool b_nmajor = (g.sbj == 1) && (g.sbk != 1);
-  if (!make_map_f32(&ma, g.A, g.K, g.M, g.sai, GT_BK, GT_BM))
+  if (!make_map_f32(&ma, g.A, g.K, g.M, g.sai, GT_BK, GT_BM, CU_TENSOR_MAP_SWIZZLE_128B))
     GPTQ_SET_ERR(c, GPTQ_ERR_CUDA, "tensor map for A failed");
-  const bool okb = b_nmajor ? make_map_f32(&mb, g.B, g.N, g.K, g.sbk, 32, GT_BK)
-                            : make_map_f32(&mb, g.B, g.K, g.N, g.sbj, GT_BK, GT_BN);
+  const bool okb =
+      b_nmajor ? make_map_f32(&mb, g.B, g.N, g.K, g.sbk, 32, GT_BK,
+                              CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)
+               : make_map_f32(&mb, g.B, g.K, g.N, g.sbj, GT_BK, GT_BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!okb) GPTQ_SET_ERR(c, GPTQ_ERR_CUDA, "tensor map for B failed");
   GemmTcParams p;
   p.M = g.M; p.N = g.N; p.K = g.K;

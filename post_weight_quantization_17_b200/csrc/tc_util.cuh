@@ -70,14 +70,23 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 // canonical layout, LBO is the distance between 64-element (128-byte) MN atoms and SBO the
 // distance between 8-row K groups; for a K-major one, SBO is the distance between 8-row MN
 // groups and LBO is unused.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Layout 1 (128-byte swizzle with 32-byte atoms, 4-row K atoms of 512 bytes) is the one
+// MN-major 32-bit (tf32) operands use; TMA writes it with SWIZZLE_128B_ATOM_32B.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                          uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFF);
   d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)(layout & 7) << 61;
   return d;
+}
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return sdesc(saddr, lbo, sbo, 2);
+}
+__device__ __forceinline__ uint64_t sdesc_sw128_32b(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return sdesc(saddr, lbo, sbo, 1);
 }
 // Instruction descriptor of kind::f16 / kind::tf32 with an fp32 accumulator.
 // fmt: 0 = f16, 1 = bf16, 2 = tf32.  a_mn / b_mn: operand is MN-major.
