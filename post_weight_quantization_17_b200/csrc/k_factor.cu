@@ -99,51 +99,126 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
     }
     __syncthreads();
     if (p0 > 0) {
-      // (b) U panel of the rows above: Pn[i][c] = sum_{k >= c} A[i][p0 + k] Rd[c][k]
-      for (int e = tid; e < p0 * FP; e += FB_THREADS) {
-        const int i = e >> 5, c = e & 31;
-        float acc = 0.f;
-        for (int k = c; k < FP; ++k) acc = fmaf(A[i][p0 + k], Rd[P][c][k], acc);
-        Pn[i][c] = acc;
+      // (b) U panel of the rows above: Pn[i][c] = sum_k A[i][p0 + k] Rd[c][k] (Rd upper, its
+      //     lower part stored as zeros).  Thread (ty, tx): rows ty + 16 a, columns tx, tx + 16.
+      const int na = p0 / 16;
+      {
+        float acc[6][2];
+#pragma unroll
+        for (int a = 0; a < 6; ++a) acc[a][0] = acc[a][1] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < FP; ++k) {
+          const float r0 = Rd[P][tx][k], r1 = Rd[P][tx + 16][k];
+#pragma unroll
+          for (int a = 0; a < 6; ++a)
+            if (a < na) {
+              const float x = A[ty + 16 * a][p0 + k];
+              acc[a][0] = fmaf(x, r0, acc[a][0]);
+              acc[a][1] = fmaf(x, r1, acc[a][1]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 6; ++a)
+          if (a < na) {
+            Pn[ty + 16 * a][tx] = acc[a][0];
+            Pn[ty + 16 * a][tx + 16] = acc[a][1];
+          }
       }
       __syncthreads();
       for (int e = tid; e < p0 * FP; e += FB_THREADS) {
         const int i = e >> 5, c = e & 31;
         A[i][p0 + c] = Pn[i][c];
       }
-      // (c) A[0:p0, 0:p0] -= Pn Pn^T
-      for (int i = ty; i < p0; i += 16)
-        for (int k = tx; k < p0; k += 16) {
-          float acc = A[i][k];
-#pragma unroll 8
-          for (int c = 0; c < FP; ++c) acc = fmaf(-Pn[i][c], Pn[k][c], acc);
-          A[i][k] = acc;
+      // (c) A[0:p0, 0:p0] -= Pn Pn^T; thread (ty, tx) owns rows ty + 16 a, columns tx + 16 b
+      {
+        float acc[6][6];
+#pragma unroll
+        for (int a = 0; a < 6; ++a)
+#pragma unroll
+          for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < FP; ++c) {
+          float xa[6], xb[6];
+#pragma unroll
+          for (int a = 0; a < 6; ++a) {
+            xa[a] = (a < na) ? Pn[ty + 16 * a][c] : 0.f;
+            xb[a] = (a < na) ? Pn[tx + 16 * a][c] : 0.f;
+          }
+#pragma unroll
+          for (int a = 0; a < 6; ++a)
+#pragma unroll
+            for (int b = 0; b < 6; ++b) acc[a][b] = fmaf(xa[a], xb[b], acc[a][b]);
         }
+#pragma unroll
+        for (int a = 0; a < 6; ++a)
+#pragma unroll
+          for (int b = 0; b < 6; ++b)
+            if (a < na && b < na) A[ty + 16 * a][tx + 16 * b] -= acc[a][b];
+      }
       __syncthreads();
     }
   }
-  // R: diagonal blocks from the panel inverses, then block rows from the bottom
-  for (int e = tid; e < FB * FP; e += FB_THREADS) {
-    const int P = e / (FP * FP), i = (e / FP) % FP, k = e % FP;
-    A[P * FP + i][P * FP + k] = (k >= i) ? Rd[P][i][k] : 0.f;
+  // R: diagonal blocks from the panel inverses; the strict lower part is zeroed so that the
+  // block products below can run over whole, uniform ranges
+  for (int e = tid; e < FB * FB; e += FB_THREADS) {
+    const int i = e >> 7, k = e & 127;
+    const int P = i / FP;
+    if (k < i) A[i][k] = 0.f;
+    else if (k < (P + 1) * FP) A[i][k] = Rd[P][i - P * FP][k - P * FP];
   }
   __syncthreads();
+  // block rows from the bottom: R[P, >P] = -R_PP (U[P, >P] R[>P, >P]).  Thread (ty, tx) owns
+  // rows ty, ty + 16 of the block row and columns c0 + tx + 16 b.
   for (int P = FB / FP - 2; P >= 0; --P) {
-    const int p0 = P * FP, c0 = p0 + FP, nc = FB - c0;
-    // T[r][c'] = sum_{l = c0..c'} U[p0 + r][l] R[l][c']
-    for (int e = tid; e < FP * nc; e += FB_THREADS) {
-      const int rr = e & 31, cc = c0 + (e >> 5);
-      float acc = 0.f;
-      for (int l = c0; l <= cc; ++l) acc = fmaf(A[p0 + rr][l], A[l][cc], acc);
-      T[rr][cc] = acc;
+    const int p0 = P * FP, c0 = p0 + FP, nb = (FB - c0) / 16;
+    {
+      float acc[2][6];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+      for (int l = c0; l < FB; ++l) {
+        const float u0 = A[p0 + ty][l], u1 = A[p0 + ty + 16][l];
+#pragma unroll
+        for (int b = 0; b < 6; ++b)
+          if (b < nb) {
+            const float rr = A[l][c0 + tx + 16 * b];
+            acc[0][b] = fmaf(u0, rr, acc[0][b]);
+            acc[1][b] = fmaf(u1, rr, acc[1][b]);
+          }
+      }
+#pragma unroll
+      for (int b = 0; b < 6; ++b)
+        if (b < nb) {
+          T[ty][c0 + tx + 16 * b] = acc[0][b];
+          T[ty + 16][c0 + tx + 16 * b] = acc[1][b];
+        }
     }
     __syncthreads();
-    // R[p0 + r][c'] = -sum_{k >= r} Rd[P][r][k] T[k][c']
-    for (int e = tid; e < FP * nc; e += FB_THREADS) {
-      const int rr = e & 31, cc = c0 + (e >> 5);
-      float acc = 0.f;
-      for (int k = rr; k < FP; ++k) acc = fmaf(Rd[P][rr][k], T[k][cc], acc);
-      A[p0 + rr][cc] = -acc;
+    {
+      float acc[2][6];
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < FP; ++k) {
+        const float r0 = Rd[P][ty][k], r1 = Rd[P][ty + 16][k];
+#pragma unroll
+        for (int b = 0; b < 6; ++b)
+          if (b < nb) {
+            const float tt = T[k][c0 + tx + 16 * b];
+            acc[0][b] = fmaf(r0, tt, acc[0][b]);
+            acc[1][b] = fmaf(r1, tt, acc[1][b]);
+          }
+      }
+#pragma unroll
+      for (int b = 0; b < 6; ++b)
+        if (b < nb) {
+          A[p0 + ty][c0 + tx + 16 * b] = -acc[0][b];
+          A[p0 + ty + 16][c0 + tx + 16 * b] = -acc[1][b];
+        }
     }
     __syncthreads();
   }

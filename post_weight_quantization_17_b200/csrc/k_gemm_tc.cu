@@ -294,12 +294,28 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       if (gi < p.M) {
         float* crow = p.C + (long long)gi * p.ldc;
         const int jb = j0 + h * 64;
+        const bool vec = (jb + 64 <= p.N) && ((reinterpret_cast<uintptr_t>(crow + jb) & 15) == 0);
+        if (vec) {
+          float4* c4 = reinterpret_cast<float4*>(crow + jb);
 #pragma unroll
-        for (int u = 0; u < 64; ++u) {
-          const int gj = jb + u;
-          if (gj < p.N) {
-            const float v = p.alpha * m[u];
-            crow[gj] = (p.beta == 0.f) ? v : fmaf(p.beta, crow[gj], v);
+          for (int u = 0; u < 16; ++u) {
+            float4 v = make_float4(p.alpha * m[4 * u], p.alpha * m[4 * u + 1],
+                                   p.alpha * m[4 * u + 2], p.alpha * m[4 * u + 3]);
+            if (p.beta != 0.f) {
+              const float4 o = c4[u];
+              v.x = fmaf(p.beta, o.x, v.x); v.y = fmaf(p.beta, o.y, v.y);
+              v.z = fmaf(p.beta, o.z, v.z); v.w = fmaf(p.beta, o.w, v.w);
+            }
+            c4[u] = v;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 64; ++u) {
+            const int gj = jb + u;
+            if (gj < p.N) {
+              const float v = p.alpha * m[u];
+              crow[gj] = (p.beta == 0.f) ? v : fmaf(p.beta, crow[gj], v);
+            }
           }
         }
       }
