@@ -24,8 +24,9 @@ constexpr int FB = 128;                 // diagonal block factored inside one CT
 constexpr int FP = 32;                  // panel width (one warp factors a panel's diagonal)
 constexpr int FB_THREADS = 256;
 // shared memory: A (the block, then U and R), the current panel, the diagonal inverses, T
+constexpr int FB_UP = 36;               // padded row of the warp-level panel buffers (16-B rows)
 constexpr int FB_SMEM = (FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
-                         FP * (FB + 1)) * 4;
+                         FP * (FB + 1) + 2 * FP * FB_UP) * 4;
 
 // Factor + invert the diagonal block M[s:s+n, s:s+n] (upper triangle read), n <= FB.
 // Writes R = U^{-1} into the upper triangle and zeros below it.
@@ -46,6 +47,10 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
       reinterpret_cast<float(*)[FP][FP + 1]>(fsm + FB * (FB + 1) + (FB - FP) * (FP + 1));
   float(*T)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(
       fsm + FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1));
+  float* fsm_panel = fsm + FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
+                     FP * (FB + 1);
+  float(*Uc)[FB_UP] = reinterpret_cast<float(*)[FB_UP]>(fsm_panel);  // Uc[j][l] = U_PP[l][j]
+  float(*Ur)[FB_UP] = reinterpret_cast<float(*)[FB_UP]>(fsm_panel + FP * FB_UP);  // rows
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tx = tid & 15, ty = tid >> 4;
@@ -70,7 +75,8 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
       float dr[FP], u[FP], r[FP];
 #pragma unroll
       for (int k = 0; k < FP; ++k) dr[k] = A[p0 + lane][p0 + k];
-      // (a) D = U_PP U_PP^T, eliminating from the last index; lane l keeps row l of U_PP
+      // (a) D = U_PP U_PP^T, eliminating from the last index.  Lane l keeps row l of D.  Column
+      // jj of U_PP is written to Uc[jj][:] and read back by every lane as float4 broadcasts.
 #pragma unroll
       for (int jj = FP - 1; jj >= 0; --jj) {
         float piv = __shfl_sync(0xffffffffu, dr[jj], jj);
@@ -79,20 +85,43 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
           if (lane == 0 && bad == 0) bad = isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE;
           piv = 1.f;
         }
-        const float dj = sqrtf(piv);
-        const float uj = (lane < jj) ? dr[jj] / dj : (lane == jj ? dj : 0.f);
+        const float rs = rsqrtf(piv);
+        const float uj = (lane < jj) ? dr[jj] * rs : (lane == jj ? piv * rs : 0.f);
         u[jj] = uj;
+        Uc[jj][lane] = uj;
+        __syncwarp();
 #pragma unroll
-        for (int k = 0; k < jj; ++k) dr[k] = fmaf(-uj, __shfl_sync(0xffffffffu, uj, k), dr[k]);
+        for (int k4 = 0; k4 < (jj + 3) / 4; ++k4) {
+          const float4 c4 = *reinterpret_cast<const float4*>(&Uc[jj][4 * k4]);
+          const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            if (4 * k4 + t < jj) dr[4 * k4 + t] = fmaf(-uj, cv[t], dr[4 * k4 + t]);
+        }
       }
-      // U_PP^{-1}: lane c computes column c, rows from the bottom
+      // rows of U_PP to Ur (lane l writes row l)
+#pragma unroll
+      for (int k = 0; k < FP; ++k) Ur[lane][k] = u[k];
+      __syncwarp();
+      // U_PP^{-1}: lane c computes column c, rows from the bottom.  Rows not yet computed are
+      // zero, so each dot product runs over the whole row (float4 broadcasts of U_PP's row i,
+      // four partial sums).
+#pragma unroll
+      for (int k = 0; k < FP; ++k) r[k] = 0.f;
 #pragma unroll
       for (int i = FP - 1; i >= 0; --i) {
-        const float uii = __shfl_sync(0xffffffffu, u[i], i);
-        float acc = 0.f;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int l = i + 1; l < FP; ++l) acc = fmaf(__shfl_sync(0xffffffffu, u[l], i), r[l], acc);
-        r[i] = (lane == i) ? 1.f / uii : (lane > i ? -acc / uii : 0.f);
+        for (int k4 = (i + 1) / 4; k4 < FP / 4; ++k4) {
+          const float4 u4 = *reinterpret_cast<const float4*>(&Ur[i][4 * k4]);
+          const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            if (4 * k4 + t > i) part[t] = fmaf(uv[t], r[4 * k4 + t], part[t]);
+        }
+        const float inv = 1.f / Ur[i][i];
+        const float acc = (part[0] + part[1]) + (part[2] + part[3]);
+        r[i] = (lane == i) ? inv : (lane > i ? -acc * inv : 0.f);
       }
 #pragma unroll
       for (int i = 0; i < FP; ++i) Rd[P][i][lane] = r[i];
