@@ -43,15 +43,20 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scale", type=float, default=1.0,
                     help="shrink the layer (tests only); the bench line is for 1.0")
+    ap.add_argument("--n-tokens", type=int, default=0,
+                    help="calibration tokens (profiling captures only; the bench line uses all)")
     return ap.parse_args()
 
 
-def workload(scale: float):
+def workload(scale: float, n_tokens: int = 0):
+    import dataclasses
     from workloads.synth import CONFIGS
     spec = CONFIGS[2][0]
     if scale != 1.0:
         spec = spec.scaled(max(32, int(spec.m * scale)), max(128, int(spec.d * scale)),
                            max(512, int(spec.n_tokens * scale)))
+    if n_tokens:
+        spec = dataclasses.replace(spec, n_tokens=n_tokens)
     return spec
 
 
@@ -222,7 +227,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    spec = workload(args.scale)
+    spec = workload(args.scale, args.n_tokens)
     n_tok, rows = min(2048, spec.n_tokens), min(16, spec.m)
     for _ in range(args.warmup):
         oracle_sample(spec, 1, n_tok, rows)
@@ -255,7 +260,7 @@ def run_ours(args):
     from workloads.synth import XSource, make_weight
 
     world, rank, local = dist_setup(args)
-    spec = workload(args.scale)
+    spec = workload(args.scale, args.n_tokens)
     seed = 1 + rank
     dev = torch.device("cuda", torch.cuda.current_device())
     W = make_weight(spec, seed, dev)
