@@ -35,7 +35,7 @@ UNIT = "weights/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--chunk", type=int, default=262144, help="tokens per accumulate call")
@@ -88,7 +88,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -301,6 +301,8 @@ def run_ours(args):
                               bufs.codes, bufs.W_hat, bufs.col_loss)
         G.gptq_pack(ctx, bufs.codes, spec.bits, bufs.packed)
 
+    clocks = ClockSampler(local)
+    clocks.start()  # sampling covers the warm-up and the timed steps (nvidia-smi needs ~0.2 s)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
@@ -308,8 +310,6 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
-        clocks = ClockSampler(local)
-        clocks.start()
         launches0 = G.gptq_kernel_launches(ctx)
         step_ev = []
         for _ in range(args.steps):
@@ -381,7 +381,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_tok, rows = min(8192, spec.n_tokens), min(64, spec.m)
+        n_tok, rows = min(32768, spec.n_tokens), min(256, spec.m)
         sample_s, full_s, desc = oracle_sample(spec, seed, n_tok, rows)
         cpu = {"value": spec.m * spec.d / full_s, "unit": UNIT, "cores": cores_used(),
                "kind": "oracle", "sample": desc, "sample_seconds": sample_s}
