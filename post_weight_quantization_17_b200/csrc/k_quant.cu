@@ -114,19 +114,20 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 }
 
 // ------------------------------------------------------------------------------------------
-// a5: one block of up to 128 columns.  A CTA has 4 warps; each warp owns 32 rows, one row per
-// lane.  The block is walked in four 32-column sub-blocks whose values stay in registers, so
-// the sequential chain of a column step (divide, round, clip, residual, η, update of the next
-// column) stays inside the lane; a sub-block first receives the residuals of the sub-blocks
-// before it (E R, the lazy update of [T] eq.(46) at a finer grain, exact by eq.(47)-(49)).
-// Only one 32-step body is unrolled, which keeps the kernel inside the instruction cache.
-// R's diagonal block is read from shared memory as warp-wide broadcasts; R's block and the W
-// block are staged with asynchronous copies (cp.async, all in flight at once); outputs leave
-// through shared memory as coalesced row segments.
+// a5: one block of up to 128 columns for 32 rows per CTA (4 warps, 8 rows per warp, 4 lanes
+// per row).  The block is walked in four 32-column sub-blocks; in a sub-block lane q of a row
+// owns the columns q, q+4, ..., q+28 in registers.  A column step fetches the column's value
+// from its owner lane (width-4 shuffle), the 4 lanes run the sequential chain (divide, round,
+// clip, residual, η) side by side, and each lane updates only its own later columns
+// ([T] eq.(42)).  A sub-block first receives the residuals of the sub-blocks before it
+// (E R, the lazy update of [T] eq.(46) at a finer grain, exact by eq.(47)-(49)).  R's block
+// and the W block are staged with asynchronous copies; outputs leave through shared memory
+// as coalesced row segments.
 constexpr int kColWarps = 4;
 constexpr int kColSub = 32;
-constexpr int kColWarpSmem = 2 * 32 * 129 * 4 + 32 * 132;
-constexpr int kColSmem = 128 * 128 * 4 + kColWarps * kColWarpSmem;
+constexpr int kColCtaRows = 32;
+constexpr int kColLd = 132;  // padded row of the staging buffers (conflict-free for 8 rows)
+constexpr int kColSmem = 128 * 128 * 4 + 2 * kColCtaRows * kColLd * 4 + kColCtaRows * 136;
 
 __device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool valid) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
@@ -140,45 +141,50 @@ __device__ __forceinline__ void cp_async_wait_all() {
 
 struct ColStepArgs {
   const float (*Rs)[128];
-  float (*St)[129];
-  uint8_t (*Cs)[132];
+  float (*St)[kColLd];
+  uint8_t (*Cs)[136];
   const int* gs;
   const float* rinv;
   const float* scales;
   const int32_t* zeros;
   long long srow;  // row * ng
-  int lane, nb;
+  int r, q, nb;    // row within the CTA, column phase of this lane
+  unsigned src0;   // lane of phase 0 in this row's group
   bool active;
   float maxq, D0, Z0;
 };
 
-// One column step at block column off + J (J compile-time so that w[] stays in registers);
-// the sub-block's later columns (J+1 .. 31) are updated immediately.
+// One column step at block column off + J (J compile-time: owner phase J & 3, slot J >> 2).
 template <int J, bool UNIFORM>
-__device__ __forceinline__ void col_step(float (&w)[kColSub], const ColStepArgs& a, int off) {
+__device__ __forceinline__ void col_step(float (&w)[8], const ColStepArgs& a, int off) {
+  constexpr int TJ = J >> 2, QJ = J & 3;
   const int C = off + J;
   if (C < a.nb) {
+    const float wj = __shfl_sync(0xffffffffu, w[TJ], a.src0 + QJ);
     float Dj = a.D0, Zj = a.Z0;
     if (!UNIFORM && a.active) {
       const int gj = a.gs[C];
       Dj = a.scales[a.srow + gj];
       Zj = (float)a.zeros[a.srow + gj];
     }
-    const float u = __fdiv_rn(w[J], Dj);
+    const float u = __fdiv_rn(wj, Dj);
     const float cq = fminf(fmaxf(rintf(u) + Zj, 0.f), a.maxq);
-    const float q = __fmul_rn(Dj, cq - Zj);
-    const float eta = __fmul_rn(__fsub_rn(w[J], q), a.rinv[C]);
-    a.Cs[a.lane][C] = (uint8_t)cq;
-    a.St[a.lane][C] = eta;
-    w[J] = q;
-    const float* rrow = &a.Rs[C][off];
+    const float qv = __fmul_rn(Dj, cq - Zj);
+    const float eta = __fmul_rn(__fsub_rn(wj, qv), a.rinv[C]);
+    if (a.q == QJ) {
+      a.Cs[a.r][C] = (uint8_t)cq;
+      a.St[a.r][C] = eta;
+      w[TJ] = qv;
+    }
+    const float* rrow = &a.Rs[C][off + a.q];
+    if (a.q > QJ) w[TJ] = fmaf(-eta, rrow[4 * TJ], w[TJ]);
 #pragma unroll
-    for (int k = J + 1; k < kColSub; ++k) w[k] = fmaf(-eta, rrow[k], w[k]);
+    for (int t = TJ + 1; t < 8; ++t) w[t] = fmaf(-eta, rrow[4 * t], w[t]);
   }
 }
 
 template <bool UNIFORM, int... Js>
-__device__ __forceinline__ void col_steps(float (&w)[kColSub], const ColStepArgs& a, int off,
+__device__ __forceinline__ void col_steps(float (&w)[8], const ColStepArgs& a, int off,
                                           std::integer_sequence<int, Js...>) {
   (col_step<Js, UNIFORM>(w, a, off), ...);
 }
@@ -191,45 +197,44 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     uint8_t* __restrict__ codes, float* __restrict__ loss_part) {
   extern __shared__ __align__(16) unsigned char smem[];
   float(*Rs)[128] = reinterpret_cast<float(*)[128]>(smem);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* wbase = smem + 128 * 128 * 4 + warp * kColWarpSmem;
   // St: the W block on entry, then column by column η (scaled residual) replaces w
-  float(*St)[129] = reinterpret_cast<float(*)[129]>(wbase);
-  float(*Qs)[129] = reinterpret_cast<float(*)[129]>(wbase + 32 * 129 * 4);  // q per column
-  uint8_t(*Cs)[132] = reinterpret_cast<uint8_t(*)[132]>(wbase + 2 * 32 * 129 * 4);
+  float(*St)[kColLd] = reinterpret_cast<float(*)[kColLd]>(smem + 128 * 128 * 4);
+  float(*Qs)[kColLd] =
+      reinterpret_cast<float(*)[kColLd]>(smem + 128 * 128 * 4 + kColCtaRows * kColLd * 4);
+  uint8_t(*Cs)[136] =
+      reinterpret_cast<uint8_t(*)[136]>(smem + 128 * 128 * 4 + 2 * kColCtaRows * kColLd * 4);
   __shared__ int gs[128];
   __shared__ float rinv[128];
 
-  const int row0 = (blockIdx.x * kColWarps + warp) * 32;  // first row of this warp
-  const int row = row0 + lane;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row0 = blockIdx.x * kColCtaRows;
+  const int r = warp * 8 + (lane >> 2);  // row within the CTA
+  const int q = lane & 3;
+  const int row = row0 + r;
   const bool active = row < m;
-  const bool warp_active = row0 < m;
 
-  // asynchronous staging: R's diagonal block (upper triangle) and this warp's W rows
-  for (int e = threadIdx.x; e < 128 * 128; e += blockDim.x) {
+  for (int e = tid; e < 128 * 128; e += blockDim.x) {
     const int a = e >> 7, b = e & 127;
     const bool v = a < nb && b < nb && b >= a;
     cp_async4(&Rs[a][b], v ? R + (long long)(i + a) * d + i + b : R, v);
   }
-  for (int r = 0; r < 32; ++r) {
-    const int gr = row0 + r;
-    for (int t = lane; t < 128; t += 32) {
-      const bool v = gr < m && t < nb;
-      cp_async4(&St[r][t], v ? Wk + (long long)gr * d + i + t : Wk, v);
-    }
+  for (int e = tid; e < kColCtaRows * 128; e += blockDim.x) {
+    const int rr = e >> 7, t = e & 127;
+    const int gr = row0 + rr;
+    const bool v = gr < m && t < nb;
+    cp_async4(&St[rr][t], v ? Wk + (long long)gr * d + i + t : Wk, v);
   }
-  for (int a = threadIdx.x; a < 128; a += blockDim.x) gs[a] = (a < nb) ? gcol[i + a] : 0;
+  for (int a = tid; a < 128; a += blockDim.x) gs[a] = (a < nb) ? gcol[i + a] : 0;
   cp_async_wait_all();
   __syncthreads();
-  for (int a = threadIdx.x; a < 128; a += blockDim.x) rinv[a] = (a < nb) ? 1.f / Rs[a][a] : 0.f;
+  for (int a = tid; a < 128; a += blockDim.x) rinv[a] = (a < nb) ? 1.f / Rs[a][a] : 0.f;
   __syncthreads();
-  if (!warp_active) return;
 
   ColStepArgs args;
   args.Rs = Rs; args.St = St; args.Cs = Cs; args.gs = gs; args.rinv = rinv;
   args.scales = scales; args.zeros = zeros;
-  args.srow = (long long)row * ng;
-  args.lane = lane; args.nb = nb; args.active = active;
+  args.srow = (long long)(active ? row : 0) * ng;
+  args.r = r; args.q = q; args.nb = nb; args.src0 = lane & ~3u; args.active = active;
   args.maxq = (float)((1 << bits) - 1);
   args.D0 = 1.f; args.Z0 = 0.f;
   if (UNIFORM && active) {
@@ -239,42 +244,38 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
 #pragma unroll 1
   for (int sb = 0; sb < 128 / kColSub; ++sb) {
     const int off = sb * kColSub;
-    if (off < nb) {
-      float w[kColSub];
+    if (off >= nb) break;
+    float w[8];
 #pragma unroll
-      for (int t = 0; t < kColSub; ++t) w[t] = St[lane][off + t];
-      // residuals of the earlier sub-blocks: w -= η[0:off] R[0:off, off:off+32]
-      for (int j = 0; j < off; ++j) {
-        const float e = St[lane][j];
-        const float* rrow = &Rs[j][off];
+    for (int t = 0; t < 8; ++t) w[t] = St[r][off + q + 4 * t];
+    __syncwarp();
+    // residuals of the earlier sub-blocks: w -= η[0:off] R[0:off, my columns]
+    for (int j = 0; j < off; ++j) {
+      const float e = St[r][j];
+      const float* rrow = &Rs[j][off + q];
 #pragma unroll
-        for (int t = 0; t < kColSub; ++t) w[t] = fmaf(-e, rrow[t], w[t]);
-      }
-      col_steps<UNIFORM>(w, args, off, std::make_integer_sequence<int, kColSub>{});
+      for (int t = 0; t < 8; ++t) w[t] = fmaf(-e, rrow[4 * t], w[t]);
+    }
+    col_steps<UNIFORM>(w, args, off, std::make_integer_sequence<int, kColSub>{});
 #pragma unroll
-      for (int t = 0; t < kColSub; ++t) Qs[lane][off + t] = w[t];
+    for (int t = 0; t < 8; ++t) Qs[r][off + q + 4 * t] = w[t];
+    __syncwarp();
+  }
+  __syncthreads();
+  // E (scaled residuals), q, codes as row segments; loss partial Σ_rows η² per column
+  for (int rr = 0; rr < kColCtaRows; ++rr) {
+    const int gr = row0 + rr;
+    if (gr >= m) break;
+    for (int t = tid; t < nb; t += blockDim.x) {
+      E[(long long)gr * kColMax + t] = St[rr][t];
+      Wk[(long long)gr * d + i + t] = Qs[rr][t];
+      codes[(long long)gr * d + i + t] = Cs[rr][t];
     }
   }
-  __syncwarp();
-  // E (scaled residuals) and the per-column loss partial Σ_rows η² over this warp's rows
-  for (int r = 0; r < 32; ++r) {
-    const int gr = row0 + r;
-    if (gr >= m) break;
-    for (int t = lane; t < nb; t += 32) E[(long long)gr * kColMax + t] = St[r][t];
-  }
-  for (int t = lane; t < nb; t += 32) {
-    float s = 0.f;
-    for (int r = 0; r < 32 && row0 + r < m; ++r) s = fmaf(St[r][t], St[r][t], s);
-    loss_part[(long long)(row0 / 32) * d + i + t] = s;
-  }
-  __syncwarp();
-  for (int r = 0; r < 32; ++r) {
-    const int gr = row0 + r;
-    if (gr >= m) break;
-    for (int t = lane; t < nb; t += 32) {
-      Wk[(long long)gr * d + i + t] = Qs[r][t];
-      codes[(long long)gr * d + i + t] = Cs[r][t];
-    }
+  for (int t = tid; t < nb; t += blockDim.x) {
+    float sacc = 0.f;
+    for (int rr = 0; rr < kColCtaRows && row0 + rr < m; ++rr) sacc = fmaf(St[rr][t], St[rr][t], sacc);
+    loss_part[(long long)blockIdx.x * d + i + t] = sacc;
   }
 }
 
@@ -285,7 +286,7 @@ int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<false>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
-  const int blocks = (m + 32 * kColWarps - 1) / (32 * kColWarps);
+  const int blocks = (m + kColCtaRows - 1) / kColCtaRows;
   if (uniform_grid)
     k_colblock<true><<<blocks, 32 * kColWarps, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
                                                           gcol, bits, E, codes, loss_part);
