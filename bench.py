@@ -176,13 +176,26 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Maximum of a per-rank time over all ranks (NCCL: on the GPU; gloo: on the host)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Every rank quantizes its own, independently drawn layer."""
+    return 1 + rank
+
+
+def weak_scaling_value(world: int, m: int, d: int, per_step_s: float) -> float:
+    """Whole-job weights per second: every rank quantizes m x d weights per step, and the job
+    takes as long as its slowest rank."""
+    return world * m * d / per_step_s
 
 
 # ----------------------------------------------------------------------------- oracle leg
@@ -261,7 +274,7 @@ def run_ours(args):
 
     world, rank, local = dist_setup(args)
     spec = workload(args.scale, args.n_tokens)
-    seed = 1 + rank
+    seed = rank_seed(rank)
     dev = torch.device("cuda", torch.cuda.current_device())
     W = make_weight(spec, seed, dev)
     # the data do not depend on --chunk: 8192-token chunks are generated and regrouped
@@ -330,7 +343,7 @@ def run_ours(args):
     syrk_ms = sum(a.elapsed_time(b) for a, b in syrk_ev) / args.steps
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
     per_step_s = total_s / args.steps
-    value = world * spec.m * spec.d / per_step_s
+    value = weak_scaling_value(world, spec.m, spec.d, per_step_s)
 
     # roofline of the dominant kernel (Hessian accumulation): algorithmic flops per launch
     bf16_peak, hbm_peak, peak_src = measured_peaks()
@@ -375,7 +388,7 @@ def run_ours(args):
                 t_ev.append((a, b))
             barrier(world)
         e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in t_ev) / 1e3 / e2e_steps, world)
-        e2e = {"value": world * spec.m * spec.d / e2e_s, "unit": UNIT,
+        e2e = {"value": weak_scaling_value(world, spec.m, spec.d, e2e_s), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_s * 1e3}
 
