@@ -25,7 +25,7 @@ size_t prep_bytes(int64_t d) {
 size_t quant_bytes(int64_t m, int64_t d, bool general_perm) {
   size_t b = gptq::kStatusBytes + 256 * 10;
   b += 2 * d * sizeof(int32_t);                                  // gcol, inv
-  b += (size_t)m * gptq::kColMax * sizeof(float);                // E
+  b += (size_t)m * gptq::kSuperCols * sizeof(float);             // E of a super-block
   b += (size_t)((m + gptq::kColRows - 1) / gptq::kColRows) * d * sizeof(float);  // loss parts
   b += d * sizeof(float);                                        // loss in processing order
   if (general_perm) b += (size_t)m * d * (sizeof(float) + 1);    // W_work, codes (permuted)
@@ -191,7 +191,7 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   Carver cv(c);
   int32_t* gcol = cv.take<int32_t>(d);
   int32_t* inv = cv.take<int32_t>(d);
-  float* E = cv.take<float>((size_t)m * gptq::kColMax);
+  float* E = cv.take<float>((size_t)m * gptq::kSuperCols);
   float* loss_part = cv.take<float>((size_t)parts * d);
   float* loss_p = cv.take<float>(d);
   float* Wk = W_hat;
@@ -207,14 +207,26 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
     return rc;
   if ((rc = gptq::make_gcol(c, perm, di, group, gcol, general ? inv : nullptr))) return rc;
   if ((rc = gptq::init_work(c, W, w_dtype, mi, di, perm, dead, !general, Wk))) return rc;
+  // Two-level lazy blocks ([T] eq.(46); exact in exact arithmetic by eq.(47)-(49)): columns
+  // are quantized in tiles of bk <= 128; after a tile only the rest of its super-block of
+  // sb = 4 bk columns is updated, and after a super-block one GEMM with K = sb updates the
+  // remaining tail.
   const int bk = std::min(block, gptq::kColMax);
-  for (int i = 0; i < di; i += bk) {
-    const int nb = std::min(bk, di - i);
-    const bool uniform = (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
-    if ((rc = gptq::column_block(c, Wk, mi, di, i, nb, R, scales, zeros, ng, gcol, uniform, bits,
-                                 E, codes_p, loss_part)))
+  const int sb = bk * (gptq::kSuperCols / gptq::kColMax);
+  for (int s0 = 0; s0 < di; s0 += sb) {
+    const int s1 = std::min(di, s0 + sb);
+    for (int i = s0; i < s1; i += bk) {
+      const int nb = std::min(bk, s1 - i);
+      const bool uniform = (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
+      float* Et = E + (i - s0);
+      if ((rc = gptq::column_block(c, Wk, mi, di, i, nb, R, scales, zeros, ng, gcol, uniform,
+                                   bits, Et, gptq::kSuperCols, codes_p, loss_part)))
+        return rc;
+      if ((rc = gptq::trailing_update(c, Wk, mi, di, i, nb, i + nb, s1, Et, gptq::kSuperCols, R)))
+        return rc;
+    }
+    if ((rc = gptq::trailing_update(c, Wk, mi, di, s0, s1 - s0, s1, di, E, gptq::kSuperCols, R)))
       return rc;
-    if ((rc = gptq::trailing_update(c, Wk, mi, di, i, nb, E, R))) return rc;
   }
   if ((rc = gptq::loss_reduce(c, loss_part, parts, di, general ? loss_p : col_loss))) return rc;
   if (general &&

@@ -193,7 +193,7 @@ template <bool UNIFORM>
 __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     float* __restrict__ Wk, int m, int d, int i, int nb, const float* __restrict__ R,
     const float* __restrict__ scales, const int32_t* __restrict__ zeros, int ng,
-    const int32_t* __restrict__ gcol, int bits, float* __restrict__ E,
+    const int32_t* __restrict__ gcol, int bits, float* __restrict__ E, int ldE,
     uint8_t* __restrict__ codes, float* __restrict__ loss_part) {
   extern __shared__ __align__(16) unsigned char smem[];
   float(*Rs)[128] = reinterpret_cast<float(*)[128]>(smem);
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     const int gr = row0 + rr;
     if (gr >= m) break;
     for (int t = tid; t < nb; t += blockDim.x) {
-      E[(long long)gr * kColMax + t] = St[rr][t];
+      E[(long long)gr * ldE + t] = St[rr][t];
       Wk[(long long)gr * d + i + t] = Qs[rr][t];
       codes[(long long)gr * d + i + t] = Cs[rr][t];
     }
@@ -281,7 +281,8 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
 
 int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                  const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
-                 bool uniform_grid, int bits, float* E, uint8_t* codes, float* loss_part) {
+                 bool uniform_grid, int bits, float* E, int ldE, uint8_t* codes,
+                 float* loss_part) {
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<false>,
@@ -289,22 +290,21 @@ int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
   const int blocks = (m + kColCtaRows - 1) / kColCtaRows;
   if (uniform_grid)
     k_colblock<true><<<blocks, 32 * kColWarps, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
-                                                          gcol, bits, E, codes, loss_part);
+                                                          gcol, bits, E, ldE, codes, loss_part);
   else
     k_colblock<false><<<blocks, 32 * kColWarps, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
-                                                           gcol, bits, E, codes, loss_part);
+                                                           gcol, bits, E, ldE, codes, loss_part);
   GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
 }
 
-// a6: W[:, i+nb:] -= E R[i:i+nb, i+nb:]  ([T] eq.(46)), fp32 on CUDA cores.
-int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* E,
-                    const float* R) {
-  const int n = d - i - nb;
-  if (n <= 0) return GPTQ_OK;
+// a6: lazy update W[:, c0:c1] -= E[:, 0:k] R[i:i+k, c0:c1]  ([T] eq.(46)); fp32-accurate GEMM.
+int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int k, int c0, int c1,
+                    const float* E, int ldE, const float* R) {
+  const int n = c1 - c0;
+  if (n <= 0 || k <= 0) return GPTQ_OK;
   int rc;
-  GemmArgs g{m, n, nb, E, kColMax, 1, R + (long long)i * d + i + nb, d, 1,
-             Wk + i + nb, d, -1.f, 1.f, 0};
+  GemmArgs g{m, n, k, E, ldE, 1, R + (long long)i * d + c0, d, 1, Wk + c0, d, -1.f, 1.f, 0};
   if ((rc = gemm_f32(c, g))) return rc;
   return GPTQ_OK;
 }

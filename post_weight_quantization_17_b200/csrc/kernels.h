@@ -29,9 +29,10 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
               const uint8_t* dead, bool identity, float* Wk);
 int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                  const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
-                 bool uniform_grid, int bits, float* E, uint8_t* codes, float* loss_part);
-int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* E,
-                    const float* R);
+                 bool uniform_grid, int bits, float* E, int ldE, uint8_t* codes,
+                 float* loss_part);
+int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int k, int c0, int c1,
+                    const float* E, int ldE, const float* R);
 int loss_reduce(Ctx* c, const float* loss_part, int parts, int d, float* loss_p);
 int unpermute(Ctx* c, int m, int d, const int32_t* inv, const uint8_t* codes_p,
               const float* Wk, const float* loss_p, uint8_t* codes, float* W_hat,
@@ -43,5 +44,6 @@ int unpack_codes(Ctx* c, const uint32_t* packed, int m, int d, int bits, uint8_t
 
 constexpr int kColRows = 32;      // rows per column-block CTA (4 warps, 4 lanes per row)
 constexpr int kColMax = 128;      // columns per kernel block
+constexpr int kSuperCols = 512;   // columns per super-block of the two-level lazy update
 
 }  // namespace gptq
