@@ -31,6 +31,8 @@ struct Ctx {
   std::string last_error;
   long long timeout_cycles = 4000000000LL;  // bounded waits in the pipelined kernels
   unsigned long long launches = 0;          // kernels this context has launched
+  cudaStream_t side = nullptr;              // second stream of the factorization recursion
+  cudaEvent_t ev[2 * 64] = {};              // its per-level events
 };
 
 constexpr size_t kStatusBytes = 256;

@@ -90,6 +90,12 @@ int gptq_create(gptq_ctx** out, void* stream, void* workspace, size_t workspace_
 
 int gptq_destroy(gptq_ctx* h) {
   if (!h) return GPTQ_ERR_ARG;
+  if (h->c.side) {
+    cudaStreamSynchronize(h->c.side);
+    for (int k = 0; k < 2 * 64; ++k)
+      if (h->c.ev[k]) cudaEventDestroy(h->c.ev[k]);
+    cudaStreamDestroy(h->c.side);
+  }
   if (h->c.owns_ws) cudaFree(h->c.ws);
   delete h;
   return GPTQ_OK;

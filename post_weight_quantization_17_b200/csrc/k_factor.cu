@@ -13,7 +13,8 @@
 //   A - U12 U12^T = U11 U11^T -> (U11, R11) by recursion
 //   R12 = -R11 U12 R22
 // All off-diagonal work is fp32-accurate GEMM (tcgen05 3xTF32); blocks of <= 128 are factored and
-// inverted inside one CTA.  A non-positive or non-finite pivot raises GPTQ_ERR_NOT_PD /
+// inverted inside one CTA.  T2 = U12 R22 needs only the right subtree, so it runs on a second
+// stream beside the left subtree's factorization.  A non-positive or non-finite pivot raises GPTQ_ERR_NOT_PD /
 // GPTQ_ERR_NONFINITE in the device status word (the host retries with more damping).
 #include "kernels.h"
 #include "gemm_simt.cuh"
@@ -55,18 +56,41 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tx = tid & 15, ty = tid >> 4;
   if (tid == 0) bad = 0;
-  // asynchronous load of the block (all copies in flight), identity padding beyond n
-  for (int e = tid; e < FB * FB; e += FB_THREADS) {
-    const int i = e >> 7, k = e & 127;
-    if (i < n && k < n) {
-      const float* src = M + (long long)(s + min(i, k)) * ld + s + max(i, k);
-      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&A[i][k]));
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-    } else {
-      A[i][k] = (i == k) ? 1.f : 0.f;
+  // asynchronous load of the block's rows (all copies in flight; 16-byte copies when the rows
+  // are 16-byte aligned), identity padding beyond n; the lower triangle is then mirrored from
+  // the upper one in shared memory
+  const bool vec = ((reinterpret_cast<uintptr_t>(M + (long long)s * ld + s) & 15) == 0) &&
+                   (ld % 4 == 0) && (n % 4 == 0);
+  if (vec) {
+    for (int e = tid; e < FB * (FB / 4); e += FB_THREADS) {
+      const int i = e >> 5, k4 = (e & 31) * 4;
+      if (i < n && k4 < n) {
+        const float* src = M + (long long)(s + i) * ld + s + k4;
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&A[i][k4]));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+      } else {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) A[i][k4 + t] = (i == k4 + t) ? 1.f : 0.f;
+      }
+    }
+  } else {
+    for (int e = tid; e < FB * FB; e += FB_THREADS) {
+      const int i = e >> 7, k = e & 127;
+      if (i < n && k < n) {
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&A[i][k]));
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst),
+                     "l"(M + (long long)(s + i) * ld + s + k) : "memory");
+      } else {
+        A[i][k] = (i == k) ? 1.f : 0.f;
+      }
     }
   }
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  for (int e = tid; e < FB * FB; e += FB_THREADS) {
+    const int i = e >> 7, k = e & 127;
+    if (k < i) A[i][k] = A[k][i];
+  }
   __syncthreads();
 
   for (int P = FB / FP - 1; P >= 0; --P) {
@@ -251,9 +275,19 @@ __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ 
     }
     __syncthreads();
   }
-  for (int e = tid; e < n * n; e += FB_THREADS) {
-    const int i = e / n, k = e - i * n;
-    M[(long long)(s + i) * ld + s + k] = (k >= i) ? A[i][k] : 0.f;
+  // write R back by rows (the strict lower part of A is zero by now)
+  if (vec) {
+    for (int e = tid; e < FB * (FB / 4); e += FB_THREADS) {
+      const int i = e >> 5, k4 = (e & 31) * 4;
+      if (i < n && k4 < n)
+        *reinterpret_cast<float4*>(M + (long long)(s + i) * ld + s + k4) =
+            make_float4(A[i][k4], A[i][k4 + 1], A[i][k4 + 2], A[i][k4 + 3]);
+    }
+  } else {
+    for (int e = tid; e < FB * FB; e += FB_THREADS) {
+      const int i = e >> 7, k = e & 127;
+      if (i < n && k < n) M[(long long)(s + i) * ld + s + k] = A[i][k];
+    }
   }
   if (tid == 0 && bad) raise_error(st, bad, s);
 }
@@ -278,39 +312,76 @@ static int copy2d(Ctx* c, const float* src, long long lds, float* dst, long long
   return GPTQ_OK;
 }
 
-size_t factor_tmp_floats(int d) {
-  size_t h = (size_t)d / 2 + FB;
+// Scratch: for every recursion level, U12 and T2 of that level's node ([n1 x n2] each, with
+// n1 <= n/2 + FB and n2 <= n/2 at node size n).
+static size_t level_floats(int n) {
+  const size_t h = (size_t)n / 2 + FB;
   return h * h;
 }
 
-static int rec(Ctx* c, float* M, long long ld, int s, int e, float* tmp) {
+// Size of a node's left child: ceil(n/2) rounded up to whole blocks, so it is the larger child
+// (the right one has n - larger_child(n) <= n/2 columns) and smaller than n for n > FB.
+static int larger_child(int n) { return (((n + 1) / 2 + FB - 1) / FB) * FB; }
+
+size_t factor_tmp_floats(int d) {
+  size_t total = 0;
+  for (int n = d; n > FB; n = larger_child(n)) total += 2 * level_floats(n);
+  return total + 64;
+}
+
+struct FactorRun {
+  Ctx* c;
+  float* M;
+  long long ld;
+  float* tmp;              // level buffers, consecutive
+  cudaStream_t side;       // T2 = U12 R22 runs here, beside the left subtree
+  cudaEvent_t ev[2 * 64];  // per level: U12 ready, T2 ready
+};
+
+static int rec(FactorRun& f, int s, int e, int level, float* buf) {
+  Ctx* c = f.c;
+  const long long ld = f.ld;
+  float* M = f.M;
   const int n = e - s;
   if (n <= FB) {
     k_factor_base<<<1, FB_THREADS, FB_SMEM, c->stream>>>(M, ld, s, n, c->status);
     GPTQ_LAUNCH_CHECK(c);
     return GPTQ_OK;
   }
-  int n1 = ((n / 2 + FB - 1) / FB) * FB;
-  if (n1 >= n) n1 = n - FB;
+  const int n1 = larger_child(n);  // < n for n > FB
   const int mid = s + n1, n2 = e - mid;
-  int rc = rec(c, M, ld, mid, e, tmp);
+  float* U12 = buf;                                   // [n1 x n2]
+  float* T2 = buf + level_floats(n);                  // [n1 x n2]
+  float* next = buf + 2 * level_floats(n);
+  int rc = rec(f, mid, e, level + 1, next);
   if (rc) return rc;
-  float* Bblk = M + (long long)s * ld + mid;       // rows s..mid, cols mid..e
-  float* R22 = M + (long long)mid * ld + mid;
+  const float* Bblk = M + (long long)s * ld + mid;    // rows s..mid, cols mid..e (H_λ)
+  float* Rblk = M + (long long)s * ld + mid;          // becomes R12
+  const float* R22 = M + (long long)mid * ld + mid;
   float* Ablk = M + (long long)s * ld + s;
   // U12 = B R22^T  (opB(k,j) = R22[j][k], zero for k < j)
-  GemmArgs g{n1, n2, n2, Bblk, ld, 1, R22, 1, ld, tmp, n2, 1.f, 0.f, kBLower};
+  GemmArgs g{n1, n2, n2, Bblk, ld, 1, R22, 1, ld, U12, n2, 1.f, 0.f, kBLower};
   if ((rc = gemm_f32(c, g))) return rc;
-  if ((rc = copy2d(c, tmp, n2, Bblk, ld, n1, n2))) return rc;
   // A' = A - U12 U12^T  (upper tiles only)
-  GemmArgs g2{n1, n1, n2, tmp, n2, 1, tmp, 1, n2, Ablk, ld, -1.f, 1.f, kCUpper};
+  GemmArgs g2{n1, n1, n2, U12, n2, 1, U12, 1, n2, Ablk, ld, -1.f, 1.f, kCUpper};
   if ((rc = gemm_f32(c, g2))) return rc;
-  if ((rc = rec(c, M, ld, s, mid, tmp))) return rc;
-  // T2 = U12 R22  (R22(k,j) = 0 for k > j)
-  GemmArgs g3{n1, n2, n2, Bblk, ld, 1, R22, ld, 1, tmp, n2, 1.f, 0.f, kBUpper};
-  if ((rc = gemm_f32(c, g3))) return rc;
+  // T2 = U12 R22 (R22(k,j) = 0 for k > j) on the side stream, beside the left subtree
+  cudaEvent_t ev_u = f.ev[2 * level], ev_t = f.ev[2 * level + 1];
+  GPTQ_CUDA_CHECK(c, cudaEventRecord(ev_u, c->stream));
+  GPTQ_CUDA_CHECK(c, cudaStreamWaitEvent(f.side, ev_u, 0));
+  {
+    cudaStream_t main = c->stream;
+    c->stream = f.side;
+    GemmArgs g3{n1, n2, n2, U12, n2, 1, R22, ld, 1, T2, n2, 1.f, 0.f, kBUpper};
+    rc = gemm_f32(c, g3);
+    c->stream = main;
+    if (rc) return rc;
+  }
+  GPTQ_CUDA_CHECK(c, cudaEventRecord(ev_t, f.side));
+  if ((rc = rec(f, s, mid, level + 1, next))) return rc;
+  GPTQ_CUDA_CHECK(c, cudaStreamWaitEvent(c->stream, ev_t, 0));
   // R12 = -R11 T2  (R11(i,k) = 0 for k < i)
-  GemmArgs g4{n1, n2, n1, Ablk, ld, 1, tmp, n2, 1, Bblk, ld, -1.f, 0.f, kAUpper};
+  GemmArgs g4{n1, n2, n1, Ablk, ld, 1, T2, n2, 1, Rblk, ld, -1.f, 0.f, kAUpper};
   if ((rc = gemm_f32(c, g4))) return rc;
   // strict lower block of this level
   return copy2d(c, nullptr, 0, M + (long long)mid * ld + s, ld, n2, n1);
@@ -319,7 +390,19 @@ static int rec(Ctx* c, float* M, long long ld, int s, int e, float* tmp) {
 int factor_inverse(Ctx* c, float* M, int d, float* tmp) {
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_factor_base,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, FB_SMEM));
-  return rec(c, M, d, 0, d, tmp);
+  if (!c->side) {
+    GPTQ_CUDA_CHECK(c, cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking));
+    for (int k = 0; k < 2 * 64; ++k)
+      GPTQ_CUDA_CHECK(c, cudaEventCreateWithFlags(&c->ev[k], cudaEventDisableTiming));
+  }
+  FactorRun f;
+  f.c = c;
+  f.M = M;
+  f.ld = d;
+  f.tmp = tmp;
+  f.side = c->side;
+  for (int k = 0; k < 2 * 64; ++k) f.ev[k] = c->ev[k];
+  return rec(f, 0, d, 0, tmp);
 }
 
 }  // namespace gptq

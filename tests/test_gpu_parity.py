@@ -48,10 +48,12 @@ def test_layer_parity(ctx, name, spec, seed):
     print(name, f"H={herr:.2e}", {k: (f"{v:.2e}" if isinstance(v, float) else v) for k, v in res.items()})
 
 
-def test_factor_stage_isolated(ctx):
-    """Same fp32 H handed to both sides: R and H^-1 from the factorization alone."""
+@pytest.mark.parametrize("d", [700, 257, 1000])
+def test_factor_stage_isolated(ctx, d):
+    """Same fp32 H handed to both sides: R and H^-1 from the factorization alone (uneven
+    recursion splits included)."""
     from oracle import gptq_oracle as O
-    spec = CONFIGS[2][0].scaled(64, 700, 4000, chunk=4000)
+    spec = CONFIGS[2][0].scaled(64, d, 4000, chunk=4000)
     W, chunks = P.make_inputs(spec, 11)
     H32 = O.hessian_tokens(torch.cat(chunks).cpu().double().numpy()).astype(np.float32)
     gpu = P.gpu_run(ctx, spec, W, chunks, H32=H32)
