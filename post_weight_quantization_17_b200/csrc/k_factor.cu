@@ -26,7 +26,8 @@ constexpr int FP = 32;                  // panel width (one warp factors a panel
 constexpr int FB_THREADS = 256;
 // shared memory: A (the block, then U and R), the current panel, the diagonal inverses, T
 constexpr int FB_UP = 36;               // padded row of the warp-level panel buffers (16-B rows)
-constexpr int FB_SMEM = (FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
+constexpr int FB_LDA = FB + 4;          // padded row of A: 528 bytes, so rows are 16-byte aligned
+constexpr int FB_SMEM = (FB * FB_LDA + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
                          FP * (FB + 1) + 2 * FP * FB_UP) * 4;
 
 // Factor + invert the diagonal block M[s:s+n, s:s+n] (upper triangle read), n <= FB.
@@ -42,13 +43,13 @@ constexpr int FB_SMEM = (FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP *
 __global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ M, long long ld,
                                                              int s, int n, DeviceStatus* st) {
   extern __shared__ float fsm[];
-  float(*A)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(fsm);
-  float(*Pn)[FP + 1] = reinterpret_cast<float(*)[FP + 1]>(fsm + FB * (FB + 1));
+  float(*A)[FB_LDA] = reinterpret_cast<float(*)[FB_LDA]>(fsm);
+  float(*Pn)[FP + 1] = reinterpret_cast<float(*)[FP + 1]>(fsm + FB * FB_LDA);
   float(*Rd)[FP][FP + 1] =
-      reinterpret_cast<float(*)[FP][FP + 1]>(fsm + FB * (FB + 1) + (FB - FP) * (FP + 1));
+      reinterpret_cast<float(*)[FP][FP + 1]>(fsm + FB * FB_LDA + (FB - FP) * (FP + 1));
   float(*T)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(
-      fsm + FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1));
-  float* fsm_panel = fsm + FB * (FB + 1) + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
+      fsm + FB * FB_LDA + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1));
+  float* fsm_panel = fsm + FB * FB_LDA + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
                      FP * (FB + 1);
   float(*Uc)[FB_UP] = reinterpret_cast<float(*)[FB_UP]>(fsm_panel);  // Uc[j][l] = U_PP[l][j]
   float(*Ur)[FB_UP] = reinterpret_cast<float(*)[FB_UP]>(fsm_panel + FP * FB_UP);  // rows
