@@ -13,7 +13,7 @@
 //   A - U12 U12^T = U11 U11^T -> (U11, R11) by recursion
 //   R12 = -R11 U12 R22
 // All off-diagonal work is fp32-accurate GEMM (tcgen05 3xTF32); blocks of <= 128 are factored and
-// inverted inside one CTA.  T2 = U12 R22 needs only the right subtree, so it runs on a second
+// inverted inside one CTA, in registers.  T2 = U12 R22 needs only the right subtree, so it runs on a second
 // stream beside the left subtree's factorization.  A non-positive or non-finite pivot raises GPTQ_ERR_NOT_PD /
 // GPTQ_ERR_NONFINITE in the device status word (the host retries with more damping).
 #include "kernels.h"
@@ -22,275 +22,165 @@
 namespace gptq {
 
 constexpr int FB = 128;                 // diagonal block factored inside one CTA
-constexpr int FP = 32;                  // panel width (one warp factors a panel's diagonal)
-constexpr int FB_THREADS = 256;
-// shared memory: A (the block, then U and R), the current panel, the diagonal inverses, T
-constexpr int FB_UP = 36;               // padded row of the warp-level panel buffers (16-B rows)
-constexpr int FB_LDA = FB + 4;          // padded row of A: 528 bytes, so rows are 16-byte aligned
-constexpr int FB_SMEM = (FB * FB_LDA + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
-                         FP * (FB + 1) + 2 * FP * FB_UP) * 4;
+constexpr int FB_WARPS = FB / 8;        // warp w holds rows 8w .. 8w+7 (one pivot tile)
+constexpr int FB_THREADS = 32 * FB_WARPS;
+constexpr int FB_LDS = FB + 1;          // staging row stride (mirrored reads: 4-way conflicts)
+constexpr int FB_SMEM = FB * FB_LDS * 4;
+
+__device__ __forceinline__ float recip_sqrt(float p) {
+  // 1/sqrt(p): hardware estimate refined by one Newton-Raphson step y <- y (3 - p y^2) / 2
+  const float y = rsqrtf(p);
+  return y * fmaf(-0.5f * p * y, y, 1.5f);
+}
 
 // Factor + invert the diagonal block M[s:s+n, s:s+n] (upper triangle read), n <= FB.
 // Writes R = U^{-1} into the upper triangle and zeros below it.
 //
-// Blocked reverse Cholesky over four 32-column panels, last panel first:
-//   (a) one warp factors the panel's 32 x 32 diagonal block D = U_PP U_PP^T in registers
-//       (lane l holds row l; pivots and columns travel by shuffles) and inverts U_PP;
-//   (b) the rows above get their U panel U[0:p0, P] = A[0:p0, P] U_PP^{-T};
-//   (c) the rows above are updated, A[0:p0, 0:p0] -= U[0:p0, P] U[0:p0, P]^T.
-// Then R block row by block row, from the bottom: R[P, >P] = -R_PP (U[P, >P] R[>P, >P]).
-// Indices >= n are padded with the identity, which factors to itself without coupling.
-__global__ void __launch_bounds__(FB_THREADS) k_factor_base(float* __restrict__ M, long long ld,
-                                                             int s, int n, DeviceStatus* st) {
-  extern __shared__ float fsm[];
-  float(*A)[FB_LDA] = reinterpret_cast<float(*)[FB_LDA]>(fsm);
-  float(*Pn)[FP + 1] = reinterpret_cast<float(*)[FP + 1]>(fsm + FB * FB_LDA);
-  float(*Rd)[FP][FP + 1] =
-      reinterpret_cast<float(*)[FP][FP + 1]>(fsm + FB * FB_LDA + (FB - FP) * (FP + 1));
-  float(*T)[FB + 1] = reinterpret_cast<float(*)[FB + 1]>(
-      fsm + FB * FB_LDA + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1));
-  float* fsm_panel = fsm + FB * FB_LDA + (FB - FP) * (FP + 1) + (FB / FP) * FP * (FP + 1) +
-                     FP * (FB + 1);
-  float(*Uc)[FB_UP] = reinterpret_cast<float(*)[FB_UP]>(fsm_panel);  // Uc[j][l] = U_PP[l][j]
-  float(*Ur)[FB_UP] = reinterpret_cast<float(*)[FB_UP]>(fsm_panel + FP * FB_UP);  // rows
-  __shared__ int bad;
+// Row elimination on [H | I] from the last index: at step j the pivot row j is scaled by
+// 1/sqrt(pivot) and subtracted from every row i < j so that column j of H vanishes above the
+// diagonal.  The row operations form an upper-triangular E with E H lower triangular
+// (= U^T), hence E = U^{-1} = R, which is what the right half holds at the end.  For a row
+// i < j the live part of the left half is columns < j and that of the right half is columns
+// >= j, so each row is kept as ONE 128-wide register row: column c holds H for c < j and R for
+// c >= j.  When step j passes, column j switches from H (eliminated) to R (-m_i / sqrt(pivot)).
+// The multiplier m_i of row i is entry i of the scaled pivot row (the trailing block stays
+// exactly symmetric: both copies of an entry receive the same products).
+//
+// Registers: thread (warp w, lane l) holds rows 8w..8w+7, columns 4l..4l+3.  Pivots go by
+// tiles of 8 (one warp's rows), last tile first:
+//   phase 1  the owning warp eliminates its 8 rows among themselves (warp shuffles only) and
+//            publishes the 8 scaled pivot rows to a double-buffered shared tile;
+//   phase 2  every warp with rows above the tile applies them as a rank-8 update.  The 8
+//            columns of the tile switch to R during the tile: their final value is
+//            -sum_j m_i(j) r'_j[c] with r'_j[c] = 0 for c < j, so those entries restart from 0
+//            and the published rows carry the zeros.
+// The next tile's owner starts phase 1 as soon as its own phase 2 is done; warps whose rows
+// are final leave the loop and write them out while the rest continue, and the barrier counts
+// only the warps still working (every reader of a tile buffer takes part in the barrier that
+// precedes its next overwrite).  Indices >= n are padded with the identity.
+__global__ void __launch_bounds__(FB_THREADS, 1) k_factor_base(float* __restrict__ M, long long ld,
+                                                                int s, int n, DeviceStatus* st) {
+  extern __shared__ __align__(16) float fsm[];
+  float(*S)[FB_LDS] = reinterpret_cast<float(*)[FB_LDS]>(fsm);       // staging (load phase)
+  float(*tile)[8][FB] = reinterpret_cast<float(*)[8][FB]>(fsm);       // 2 x 8 pivot rows (after)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tx = tid & 15, ty = tid >> 4;
-  if (tid == 0) bad = 0;
-  // asynchronous load of the block's rows (all copies in flight; 16-byte copies when the rows
-  // are 16-byte aligned), identity padding beyond n; the lower triangle is then mirrored from
-  // the upper one in shared memory
-  const bool vec = ((reinterpret_cast<uintptr_t>(M + (long long)s * ld + s) & 15) == 0) &&
-                   (ld % 4 == 0) && (n % 4 == 0);
-  if (vec) {
-    for (int e = tid; e < FB * (FB / 4); e += FB_THREADS) {
-      const int i = e >> 5, k4 = (e & 31) * 4;
-      if (i < n && k4 < n) {
-        const float* src = M + (long long)(s + i) * ld + s + k4;
-        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&A[i][k4]));
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-      } else {
+  const int i0 = 8 * warp, c0 = 4 * lane;
+  // coalesced load of the upper triangle's row segments into shared memory
+  {
+    const float* base = M + (long long)s * ld + s;
+    const bool vec = ((reinterpret_cast<uintptr_t>(base) & 15) == 0) && (ld % 4 == 0);
+    float4 v[FB * FB / 4 / FB_THREADS];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) A[i][k4 + t] = (i == k4 + t) ? 1.f : 0.f;
+    for (int u = 0; u < FB * FB / 4 / FB_THREADS; ++u) {
+      const int e = tid + u * FB_THREADS, i = e >> 5, k = (e & 31) * 4;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < n && k + 3 >= i && k < n) {
+        const float* src = base + (long long)i * ld + k;
+        if (vec && k + 4 <= n) {
+          v[u] = *reinterpret_cast<const float4*>(src);
+        } else {
+          v[u].x = src[0];
+          if (k + 1 < n) v[u].y = src[1];
+          if (k + 2 < n) v[u].z = src[2];
+          if (k + 3 < n) v[u].w = src[3];
+        }
       }
     }
-  } else {
-    for (int e = tid; e < FB * FB; e += FB_THREADS) {
-      const int i = e >> 7, k = e & 127;
-      if (i < n && k < n) {
-        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&A[i][k]));
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst),
-                     "l"(M + (long long)(s + i) * ld + s + k) : "memory");
-      } else {
-        A[i][k] = (i == k) ? 1.f : 0.f;
-      }
+#pragma unroll
+    for (int u = 0; u < FB * FB / 4 / FB_THREADS; ++u) {
+      const int e = tid + u * FB_THREADS, i = e >> 5, k = (e & 31) * 4;
+      S[i][k] = v[u].x;
+      S[i][k + 1] = v[u].y;
+      S[i][k + 2] = v[u].z;
+      S[i][k + 3] = v[u].w;
     }
   }
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  for (int e = tid; e < FB * FB; e += FB_THREADS) {
-    const int i = e >> 7, k = e & 127;
-    if (k < i) A[i][k] = A[k][i];
-  }
-  __syncthreads();
-
-  for (int P = FB / FP - 1; P >= 0; --P) {
-    const int p0 = P * FP;
-    if (warp == 0) {
-      float dr[FP], u[FP], r[FP];
+  float x[8][4];
 #pragma unroll
-      for (int k = 0; k < FP; ++k) dr[k] = A[p0 + lane][p0 + k];
-      // (a) D = U_PP U_PP^T, eliminating from the last index.  Lane l keeps row l of D.  Column
-      // jj of U_PP is written to Uc[jj][:] and read back by every lane as float4 broadcasts.
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
-      for (int jj = FP - 1; jj >= 0; --jj) {
-        float piv = __shfl_sync(0xffffffffu, dr[jj], jj);
-        const bool good = (piv > 0.f) && isfinite(piv);
-        if (!good) {
-          if (lane == 0 && bad == 0) bad = isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE;
+    for (int t = 0; t < 4; ++t) {
+      const int i = i0 + a, c = c0 + t;
+      x[a][t] = (i < n && c < n) ? (c >= i ? S[i][c] : S[c][i]) : (i == c ? 1.f : 0.f);
+    }
+  __syncthreads();  // the staging area becomes the tile buffers
+  int bad = 0;
+  for (int jb = FB_WARPS - 1; jb >= warp; --jb) {
+    float(*tb)[FB] = tile[jb & 1];
+    if (warp == jb) {
+      // ---- phase 1: the tile's own rows, last first
+#pragma unroll
+      for (int a = 7; a >= 0; --a) {
+        const int j = 8 * jb + a;
+        const int jl = 2 * jb + (a >> 2);  // lane holding column j, as element a & 3
+        float piv = __shfl_sync(0xffffffffu, x[a][a & 3], jl);
+        if (!(piv > 0.f) || !isfinite(piv)) {
+          if (bad == 0) bad = isfinite(piv) ? GPTQ_ERR_NOT_PD : GPTQ_ERR_NONFINITE;
           piv = 1.f;
         }
-        const float rs = rsqrtf(piv);
-        const float uj = (lane < jj) ? dr[jj] * rs : (lane == jj ? piv * rs : 0.f);
-        u[jj] = uj;
-        Uc[jj][lane] = uj;
-        __syncwarp();
+        const float sc = recip_sqrt(piv);
+        float r[4];
 #pragma unroll
-        for (int k4 = 0; k4 < (jj + 3) / 4; ++k4) {
-          const float4 c4 = *reinterpret_cast<const float4*>(&Uc[jj][4 * k4]);
-          const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+        for (int t = 0; t < 4; ++t) r[t] = x[a][t] * sc;
+        if (lane == jl) r[a & 3] = sc;  // R_jj (the right half's 1, scaled)
+        // row j is final: R for c >= j, zero below the diagonal
 #pragma unroll
-          for (int t = 0; t < 4; ++t)
-            if (4 * k4 + t < jj) dr[4 * k4 + t] = fmaf(-uj, cv[t], dr[4 * k4 + t]);
+        for (int t = 0; t < 4; ++t) x[a][t] = (c0 + t < j) ? 0.f : r[t];
+        // published row: tile columns below j carry 0 (see phase 2)
+        const bool tcol = (lane >> 1) == jb;
+        *reinterpret_cast<float4*>(&tb[a][c0]) =
+            tcol ? make_float4(x[a][0], x[a][1], x[a][2], x[a][3])
+                 : make_float4(r[0], r[1], r[2], r[3]);
+#pragma unroll
+        for (int ap = 0; ap < a; ++ap) {
+          const float mm = __shfl_sync(0xffffffffu, r[ap & 3], 2 * jb + (ap >> 2));
+#pragma unroll
+          for (int t = 0; t < 4; ++t) x[ap][t] = fmaf(-mm, r[t], x[ap][t]);
+          if (lane == jl) x[ap][a & 3] = -mm * sc;
         }
       }
-      // rows of U_PP to Ur (lane l writes row l)
-#pragma unroll
-      for (int k = 0; k < FP; ++k) Ur[lane][k] = u[k];
-      __syncwarp();
-      // U_PP^{-1}: lane c computes column c, rows from the bottom.  Rows not yet computed are
-      // zero, so each dot product runs over the whole row (float4 broadcasts of U_PP's row i,
-      // four partial sums).
-#pragma unroll
-      for (int k = 0; k < FP; ++k) r[k] = 0.f;
-#pragma unroll
-      for (int i = FP - 1; i >= 0; --i) {
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k4 = (i + 1) / 4; k4 < FP / 4; ++k4) {
-          const float4 u4 = *reinterpret_cast<const float4*>(&Ur[i][4 * k4]);
-          const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t)
-            if (4 * k4 + t > i) part[t] = fmaf(uv[t], r[4 * k4 + t], part[t]);
-        }
-        const float inv = 1.f / Ur[i][i];
-        const float acc = (part[0] + part[1]) + (part[2] + part[3]);
-        r[i] = (lane == i) ? inv : (lane > i ? -acc * inv : 0.f);
-      }
-#pragma unroll
-      for (int i = 0; i < FP; ++i) Rd[P][i][lane] = r[i];
     }
-    __syncthreads();
-    if (p0 > 0) {
-      // (b) U panel of the rows above: Pn[i][c] = sum_k A[i][p0 + k] Rd[c][k] (Rd upper, its
-      //     lower part stored as zeros).  Thread (ty, tx): rows ty + 16 a, columns tx, tx + 16.
-      const int na = p0 / 16;
-      {
-        float acc[6][2];
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * (jb + 1)) : "memory");
+    if (warp < jb) {
+      // ---- phase 2: rank-8 update of this warp's rows
+      if ((lane >> 1) == jb) {
 #pragma unroll
-        for (int a = 0; a < 6; ++a) acc[a][0] = acc[a][1] = 0.f;
-#pragma unroll 4
-        for (int k = 0; k < FP; ++k) {
-          const float r0 = Rd[P][tx][k], r1 = Rd[P][tx + 16][k];
+        for (int a = 0; a < 8; ++a)
 #pragma unroll
-          for (int a = 0; a < 6; ++a)
-            if (a < na) {
-              const float x = A[ty + 16 * a][p0 + k];
-              acc[a][0] = fmaf(x, r0, acc[a][0]);
-              acc[a][1] = fmaf(x, r1, acc[a][1]);
-            }
-        }
-#pragma unroll
-        for (int a = 0; a < 6; ++a)
-          if (a < na) {
-            Pn[ty + 16 * a][tx] = acc[a][0];
-            Pn[ty + 16 * a][tx + 16] = acc[a][1];
-          }
+          for (int t = 0; t < 4; ++t) x[a][t] = 0.f;
       }
-      __syncthreads();
-      for (int e = tid; e < p0 * FP; e += FB_THREADS) {
-        const int i = e >> 5, c = e & 31;
-        A[i][p0 + c] = Pn[i][c];
+#pragma unroll
+      for (int a = 7; a >= 0; --a) {
+        const float4 v4 = *reinterpret_cast<const float4*>(&tb[a][c0]);
+        const float4 ma = *reinterpret_cast<const float4*>(&tb[a][i0]);
+        const float4 mb = *reinterpret_cast<const float4*>(&tb[a][i0 + 4]);
+        const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+        const float m[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+#pragma unroll
+        for (int ap = 0; ap < 8; ++ap)
+#pragma unroll
+          for (int t = 0; t < 4; ++t) x[ap][t] = fmaf(-m[ap], v[t], x[ap][t]);
       }
-      // (c) A[0:p0, 0:p0] -= Pn Pn^T; thread (ty, tx) owns rows ty + 16 a, columns tx + 16 b
-      {
-        float acc[6][6];
-#pragma unroll
-        for (int a = 0; a < 6; ++a)
-#pragma unroll
-          for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
-#pragma unroll 4
-        for (int c = 0; c < FP; ++c) {
-          float xa[6], xb[6];
-#pragma unroll
-          for (int a = 0; a < 6; ++a) {
-            xa[a] = (a < na) ? Pn[ty + 16 * a][c] : 0.f;
-            xb[a] = (a < na) ? Pn[tx + 16 * a][c] : 0.f;
-          }
-#pragma unroll
-          for (int a = 0; a < 6; ++a)
-#pragma unroll
-            for (int b = 0; b < 6; ++b) acc[a][b] = fmaf(xa[a], xb[b], acc[a][b]);
-        }
-#pragma unroll
-        for (int a = 0; a < 6; ++a)
-#pragma unroll
-          for (int b = 0; b < 6; ++b)
-            if (a < na && b < na) A[ty + 16 * a][tx + 16 * b] -= acc[a][b];
-      }
-      __syncthreads();
     }
   }
-  // R: diagonal blocks from the panel inverses; the strict lower part is zeroed so that the
-  // block products below can run over whole, uniform ranges
-  for (int e = tid; e < FB * FB; e += FB_THREADS) {
-    const int i = e >> 7, k = e & 127;
-    const int P = i / FP;
-    if (k < i) A[i][k] = 0.f;
-    else if (k < (P + 1) * FP) A[i][k] = Rd[P][i - P * FP][k - P * FP];
-  }
-  __syncthreads();
-  // block rows from the bottom: R[P, >P] = -R_PP (U[P, >P] R[>P, >P]).  Thread (ty, tx) owns
-  // rows ty, ty + 16 of the block row and columns c0 + tx + 16 b.
-  for (int P = FB / FP - 2; P >= 0; --P) {
-    const int p0 = P * FP, c0 = p0 + FP, nb = (FB - c0) / 16;
-    {
-      float acc[2][6];
+  if (bad && lane == 0) raise_error(st, bad, s);
+  // write the warp's rows of R (zeros below the diagonal are already in place)
+  const bool vec = ((reinterpret_cast<uintptr_t>(M + (long long)s * ld + s) & 15) == 0) &&
+                   (ld % 4 == 0) && (c0 + 4 <= n);
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
+  for (int a = 0; a < 8; ++a) {
+    const int i = i0 + a;
+    if (i >= n) break;
+    float* row = M + (long long)(s + i) * ld + s;
+    if (vec) {
+      *reinterpret_cast<float4*>(row + c0) = make_float4(x[a][0], x[a][1], x[a][2], x[a][3]);
+    } else {
 #pragma unroll
-        for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
-#pragma unroll 4
-      for (int l = c0; l < FB; ++l) {
-        const float u0 = A[p0 + ty][l], u1 = A[p0 + ty + 16][l];
-#pragma unroll
-        for (int b = 0; b < 6; ++b)
-          if (b < nb) {
-            const float rr = A[l][c0 + tx + 16 * b];
-            acc[0][b] = fmaf(u0, rr, acc[0][b]);
-            acc[1][b] = fmaf(u1, rr, acc[1][b]);
-          }
-      }
-#pragma unroll
-      for (int b = 0; b < 6; ++b)
-        if (b < nb) {
-          T[ty][c0 + tx + 16 * b] = acc[0][b];
-          T[ty + 16][c0 + tx + 16 * b] = acc[1][b];
-        }
-    }
-    __syncthreads();
-    {
-      float acc[2][6];
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
-#pragma unroll 4
-      for (int k = 0; k < FP; ++k) {
-        const float r0 = Rd[P][ty][k], r1 = Rd[P][ty + 16][k];
-#pragma unroll
-        for (int b = 0; b < 6; ++b)
-          if (b < nb) {
-            const float tt = T[k][c0 + tx + 16 * b];
-            acc[0][b] = fmaf(r0, tt, acc[0][b]);
-            acc[1][b] = fmaf(r1, tt, acc[1][b]);
-          }
-      }
-#pragma unroll
-      for (int b = 0; b < 6; ++b)
-        if (b < nb) {
-          A[p0 + ty][c0 + tx + 16 * b] = -acc[0][b];
-          A[p0 + ty + 16][c0 + tx + 16 * b] = -acc[1][b];
-        }
-    }
-    __syncthreads();
-  }
-  // write R back by rows (the strict lower part of A is zero by now)
-  if (vec) {
-    for (int e = tid; e < FB * (FB / 4); e += FB_THREADS) {
-      const int i = e >> 5, k4 = (e & 31) * 4;
-      if (i < n && k4 < n)
-        *reinterpret_cast<float4*>(M + (long long)(s + i) * ld + s + k4) =
-            make_float4(A[i][k4], A[i][k4 + 1], A[i][k4 + 2], A[i][k4 + 3]);
-    }
-  } else {
-    for (int e = tid; e < FB * FB; e += FB_THREADS) {
-      const int i = e >> 7, k = e & 127;
-      if (i < n && k < n) M[(long long)(s + i) * ld + s + k] = A[i][k];
+      for (int t = 0; t < 4; ++t)
+        if (c0 + t < n) row[c0 + t] = x[a][t];
     }
   }
-  if (tid == 0 && bad) raise_error(st, bad, s);
 }
 
 __global__ void k_copy2d(const float* __restrict__ src, long long lds, float* __restrict__ dst,

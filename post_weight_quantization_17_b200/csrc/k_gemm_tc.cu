@@ -6,7 +6,9 @@
 //
 // Each fp32 operand x is split as hi = tf32(x), lo = tf32(x - hi) (round to nearest) and the
 // product is hi*hi + hi*lo + lo*hi: three tcgen05.mma.kind::tf32 per k-step into one TMEM
-// accumulator (relative error ~2^-21 per product, against 2^-11 for plain TF32).  The tensor
+// accumulator (relative error ~2^-21 per product, against 2^-11 for plain TF32; clearing the
+// low bits instead of rounding would double the error that the factorization's conditioning
+// then amplifies).  The tensor
 // core's accumulation over many MMAs loses low bits, so partial sums of KP = 128 k-elements are
 // taken from TMEM and added in fp32 into a register accumulator by the epilogue warps.
 //   warp 0       TMA producer: A box 128 x 32, B box 128 x 32 (K-major) or 4 x (32 x 32)
@@ -59,10 +61,12 @@ __device__ __forceinline__ bool gt_tile(const GemmTcParams& p, int t, int& i0, i
   return true;
 }
 
-__device__ __forceinline__ uint32_t tf32_rna(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
+// Round an fp32 value to tf32 (10 explicit mantissa bits), to nearest with ties away from zero:
+// the format is sign-magnitude, so adding half a tf32 unit (bit 12) to the bit pattern and
+// clearing the 13 low bits rounds the magnitude; a mantissa carry moves into the exponent as it
+// should.  Integer ALU only (the conversion instruction runs on a narrower pipe).
+__device__ __forceinline__ float tf32_rna(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
 __global__ void __launch_bounds__(GT_THREADS, 1)
@@ -231,14 +235,14 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
           for (int c = ct; c < GT_TILE_BYTES / 16; c += 32 * GT_CONV_WARPS) {
             const float4 x = hi[c];
             float4 h, l;
-            h.x = __uint_as_float(tf32_rna(x.x));
-            h.y = __uint_as_float(tf32_rna(x.y));
-            h.z = __uint_as_float(tf32_rna(x.z));
-            h.w = __uint_as_float(tf32_rna(x.w));
-            l.x = __uint_as_float(tf32_rna(x.x - h.x));
-            l.y = __uint_as_float(tf32_rna(x.y - h.y));
-            l.z = __uint_as_float(tf32_rna(x.z - h.z));
-            l.w = __uint_as_float(tf32_rna(x.w - h.w));
+            h.x = tf32_rna(x.x);
+            h.y = tf32_rna(x.y);
+            h.z = tf32_rna(x.z);
+            h.w = tf32_rna(x.w);
+            l.x = tf32_rna(x.x - h.x);
+            l.y = tf32_rna(x.y - h.y);
+            l.z = tf32_rna(x.z - h.z);
+            l.w = tf32_rna(x.w - h.w);
             hi[c] = h;
             lo[c] = l;
           }
@@ -297,16 +301,25 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
         const bool vec = (jb + 64 <= p.N) && ((reinterpret_cast<uintptr_t>(crow + jb) & 15) == 0);
         if (vec) {
           float4* c4 = reinterpret_cast<float4*>(crow + jb);
+          // C is read in batches of eight float4 before any store, so that the loads overlap
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            float4 v = make_float4(p.alpha * m[4 * u], p.alpha * m[4 * u + 1],
-                                   p.alpha * m[4 * u + 2], p.alpha * m[4 * u + 3]);
+          for (int hb = 0; hb < 2; ++hb) {
+            float4 o[8];
             if (p.beta != 0.f) {
-              const float4 o = c4[u];
-              v.x = fmaf(p.beta, o.x, v.x); v.y = fmaf(p.beta, o.y, v.y);
-              v.z = fmaf(p.beta, o.z, v.z); v.w = fmaf(p.beta, o.w, v.w);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) o[u] = c4[8 * hb + u];
             }
-            c4[u] = v;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int e = 4 * (8 * hb + u);
+              float4 v = make_float4(p.alpha * m[e], p.alpha * m[e + 1], p.alpha * m[e + 2],
+                                     p.alpha * m[e + 3]);
+              if (p.beta != 0.f) {
+                v.x = fmaf(p.beta, o[u].x, v.x); v.y = fmaf(p.beta, o[u].y, v.y);
+                v.z = fmaf(p.beta, o[u].z, v.z); v.w = fmaf(p.beta, o[u].w, v.w);
+              }
+              c4[8 * hb + u] = v;
+            }
           }
         } else {
 #pragma unroll
@@ -321,6 +334,9 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       }
     }
   }
+  // the producer and MMA roles run on one lane of their warps: reconverge every warp before the
+  // CTA barrier, so that TMEM is released only after the epilogue has read it
+  __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {

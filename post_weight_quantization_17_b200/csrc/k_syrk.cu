@@ -241,6 +241,9 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
       }
     }
   }
+  // the producer and MMA roles run on one lane of their warps: reconverge every warp before the
+  // CTA barrier, so that TMEM is released only after the epilogue has read it
+  __syncwarp();
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {
