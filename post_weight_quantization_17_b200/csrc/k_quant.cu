@@ -114,20 +114,28 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 }
 
 // ------------------------------------------------------------------------------------------
-// a5: one block of up to 128 columns for 32 rows per CTA (4 warps, 8 rows per warp, 4 lanes
+// a5: one block of up to 128 columns for 32 rows per CTA (8 warps, 4 rows per warp, 8 lanes
 // per row).  The block is walked in four 32-column sub-blocks; in a sub-block lane q of a row
-// owns the columns q, q+4, ..., q+28 in registers.  A column step fetches the column's value
-// from its owner lane (width-4 shuffle), the 4 lanes run the sequential chain (divide, round,
-// clip, residual, η) side by side, and each lane updates only its own later columns
+// owns the 4 consecutive columns 4q .. 4q+3 in registers.  A column step fetches the column's
+// value from its owner lane (width-8 shuffle), the 8 lanes run the sequential chain (divide,
+// round, clip, residual, η) side by side, and each lane updates only its own later columns
 // ([T] eq.(42)).  A sub-block first receives the residuals of the sub-blocks before it
 // (E R, the lazy update of [T] eq.(46) at a finer grain, exact by eq.(47)-(49)).  R's block
 // and the W block are staged with asynchronous copies; outputs leave through shared memory
 // as coalesced row segments.
-constexpr int kColWarps = 4;
-constexpr int kColSub = 32;
+//
+// The quotient w/Δ is the IEEE (correctly rounded) one, computed from y = RN(1/Δ), taken once
+// per grid group: q0 = RN(w y), r = w - q0 Δ (exact, by FMA), u = RN(q0 + r y).  By
+// Markstein's theorem (IBM J. Res. Dev. 34(1), 1990: y within half an ulp of 1/Δ and q0 within
+// an ulp of w/Δ make RN(q0 + r y) = RN(w/Δ)) this is the same fp32 value as a division, at a
+// third of its latency on the column chain.
+constexpr int kColWarps = 8;
+constexpr int kColLanes = 8;                 // lanes per row
+constexpr int kColSub = 4 * kColLanes;       // sub-block width: 4 columns per lane
 constexpr int kColCtaRows = 32;
-constexpr int kColLd = 132;  // padded row of the staging buffers (conflict-free for 8 rows)
-constexpr int kColSmem = 128 * 128 * 4 + 2 * kColCtaRows * kColLd * 4 + kColCtaRows * 136;
+constexpr int kColLd = 132;  // padded row of the staging buffers (16-byte rows)
+constexpr int kColSmem = 128 * 128 * 4 + kColCtaRows * kColLd * 4 + kColWarps * 128 * 4;
+static_assert(kColCtaRows == kColWarps * 32 / kColLanes && kColCtaRows == kColRows, "rows per CTA");
 
 __device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool valid) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
@@ -135,58 +143,144 @@ __device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc, bool
                "r"(valid ? 4 : 0)
                : "memory");
 }
+// 16-byte copy of the first `bytes` (0..16) bytes, the rest zero-filled
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, int bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// y = RN(1/Δ) is used only while Δ lies in [2^-100, 2^100], where 1/Δ and the correction stay
+// normal; a CTA with any row outside that range takes the division itself.
+__device__ __forceinline__ bool quotient_fast(float delta) {
+  return delta >= 0x1p-100f && delta <= 0x1p100f;
+}
+template <bool FAST>
+__device__ __forceinline__ float quotient(float w, float delta, float y) {
+  if (!FAST) return __fdiv_rn(w, delta);
+  const float q0 = __fmul_rn(w, y);
+  const float r = fmaf(-q0, delta, w);
+  return fmaf(r, y, q0);
+}
+
 struct ColStepArgs {
   const float (*Rs)[128];
-  float (*St)[kColLd];
-  uint8_t (*Cs)[136];
   const int* gs;
   const float* rinv;
   const float* scales;
   const int32_t* zeros;
   long long srow;  // row * ng
-  int r, q, nb;    // row within the CTA, column phase of this lane
-  unsigned src0;   // lane of phase 0 in this row's group
+  int q;           // owner index of this lane
+  unsigned src0;   // lane of owner 0 in this row's group
   bool active;
-  float maxq, D0, Z0;
+  float maxq, D0, Z0, Y0;
 };
 
-// One column step at block column off + J (J compile-time: owner phase J & 3, slot J >> 2).
-template <int J, bool UNIFORM>
-__device__ __forceinline__ void col_step(float (&w)[8], const ColStepArgs& a, int off) {
-  constexpr int TJ = J >> 2, QJ = J & 3;
+// One column step at block column off + J (J compile-time: owner lane J >> 2, slot J & 3).
+// Columns past the block's end hold zeros with rinv = 0 and zero R rows, so their step is an
+// exact no-op and needs no branch.  The code offset c - z is clipped to [-z, maxq - z]
+// directly (integers in fp32: the same value as clipping c and subtracting z).
+template <int J, bool UNIFORM, bool FAST>
+__device__ __forceinline__ void col_step(float (&w)[4], float (&e4)[4], float (&c4)[4],
+                                         const ColStepArgs& a, int off) {
+  constexpr int TJ = J & 3, QJ = J >> 2;
   const int C = off + J;
-  if (C < a.nb) {
-    const float wj = __shfl_sync(0xffffffffu, w[TJ], a.src0 + QJ);
-    float Dj = a.D0, Zj = a.Z0;
-    if (!UNIFORM && a.active) {
-      const int gj = a.gs[C];
-      Dj = a.scales[a.srow + gj];
-      Zj = (float)a.zeros[a.srow + gj];
-    }
-    const float u = __fdiv_rn(wj, Dj);
-    const float cq = fminf(fmaxf(rintf(u) + Zj, 0.f), a.maxq);
-    const float qv = __fmul_rn(Dj, cq - Zj);
-    const float eta = __fmul_rn(__fsub_rn(wj, qv), a.rinv[C]);
-    if (a.q == QJ) {
-      a.Cs[a.r][C] = (uint8_t)cq;
-      a.St[a.r][C] = eta;
-      w[TJ] = qv;
-    }
-    const float* rrow = &a.Rs[C][off + a.q];
-    if (a.q > QJ) w[TJ] = fmaf(-eta, rrow[4 * TJ], w[TJ]);
+  const float wj = __shfl_sync(0xffffffffu, w[TJ], a.src0 + QJ);
+  float Dj = a.D0, Zj = a.Z0, Yj = a.Y0;
+  if (!UNIFORM && a.active) {
+    const int gj = a.gs[C];
+    Dj = a.scales[a.srow + gj];
+    Zj = (float)a.zeros[a.srow + gj];
+    if (FAST) Yj = __frcp_rn(Dj);
+  }
+  const float u = quotient<FAST>(wj, Dj, Yj);
+  const float co = fminf(fmaxf(rintf(u), -Zj), a.maxq - Zj);
+  const float qv = __fmul_rn(Dj, co);
+  const float eta = __fmul_rn(__fsub_rn(wj, qv), a.rinv[C]);
+  const float4 r4 = *reinterpret_cast<const float4*>(&a.Rs[C][off + 4 * a.q]);
+  const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
+  // later columns of this lane: all of them past the owner, the slots after TJ at the owner
+  const float e_hi = (a.q >= QJ) ? eta : 0.f;
+  const float e_lo = (a.q > QJ) ? eta : 0.f;
 #pragma unroll
-    for (int t = TJ + 1; t < 8; ++t) w[t] = fmaf(-eta, rrow[4 * t], w[t]);
+  for (int t = 0; t < 4; ++t) w[t] = fmaf(-(t > TJ ? e_hi : e_lo), rr[t], w[t]);
+  if (a.q == QJ) {
+    w[TJ] = qv;
+    e4[TJ] = eta;
+    c4[TJ] = co + Zj;
   }
 }
 
-template <bool UNIFORM, int... Js>
-__device__ __forceinline__ void col_steps(float (&w)[8], const ColStepArgs& a, int off,
+template <bool UNIFORM, bool FAST, int... Js>
+__device__ __forceinline__ void col_steps(float (&w)[4], float (&e4)[4], float (&c4)[4],
+                                          const ColStepArgs& a, int off,
                                           std::integer_sequence<int, Js...>) {
-  (col_step<Js, UNIFORM>(w, a, off), ...);
+  (col_step<Js, UNIFORM, FAST>(w, e4, c4, a, off), ...);
+}
+
+template <bool UNIFORM, bool FAST>
+__device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128],
+                                         const ColStepArgs& args, int r, int row, int nb, int d,
+                                         int i, int ldE, bool vec, float* __restrict__ Wk,
+                                         float* __restrict__ E, uint8_t* __restrict__ codes) {
+  const float(*Rs)[128] = args.Rs;
+  const int q = args.q, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll 1
+  for (int off = 0; off < nb; off += kColSub) {
+    float w[4], e4[4] = {0.f, 0.f, 0.f, 0.f}, c4[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const float4 w4 = *reinterpret_cast<const float4*>(&St[r][off + 4 * q]);
+      w[0] = w4.x; w[1] = w4.y; w[2] = w4.z; w[3] = w4.w;
+    }
+    // residuals of the earlier sub-blocks: w -= η[0:off] R[0:off, my columns], 8 at a time
+    for (int j = 0; j < off; j += 8) {
+      const float4 ea = *reinterpret_cast<const float4*>(&St[r][j]);
+      const float4 eb = *reinterpret_cast<const float4*>(&St[r][j + 4]);
+      const float e[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4 r4 = *reinterpret_cast<const float4*>(&Rs[j + u][off + 4 * q]);
+        w[0] = fmaf(-e[u], r4.x, w[0]);
+        w[1] = fmaf(-e[u], r4.y, w[1]);
+        w[2] = fmaf(-e[u], r4.z, w[2]);
+        w[3] = fmaf(-e[u], r4.w, w[3]);
+      }
+    }
+    col_steps<UNIFORM, FAST>(w, e4, c4, args, off, std::make_integer_sequence<int, kColSub>{});
+    // the sub-block's η for later sub-blocks; outputs straight from registers
+    __syncwarp();
+    *reinterpret_cast<float4*>(&St[r][off + 4 * q]) = make_float4(e4[0], e4[1], e4[2], e4[3]);
+    const int c = off + 4 * q;
+    if (args.active) {
+      if (vec && c + 4 <= nb) {
+        *reinterpret_cast<float4*>(E + (long long)row * ldE + c) =
+            make_float4(e4[0], e4[1], e4[2], e4[3]);
+        *reinterpret_cast<float4*>(Wk + (long long)row * d + i + c) =
+            make_float4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uchar4*>(codes + (long long)row * d + i + c) =
+            make_uchar4((uint8_t)c4[0], (uint8_t)c4[1], (uint8_t)c4[2], (uint8_t)c4[3]);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (c + t < nb) {
+            E[(long long)row * ldE + c + t] = e4[t];
+            Wk[(long long)row * d + i + c + t] = w[t];
+            codes[(long long)row * d + i + c + t] = (uint8_t)c4[t];
+          }
+      }
+    }
+    // Σ η² over the warp's 4 rows (lanes q, q+8, q+16, q+24 share columns)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float s2 = args.active ? e4[t] * e4[t] : 0.f;
+      s2 += __shfl_xor_sync(0xffffffffu, s2, 8);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, 16);
+      if (lane < kColLanes) lossw[warp][c + t] = s2;
+    }
+  }
 }
 
 template <bool UNIFORM>
@@ -197,84 +291,87 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     uint8_t* __restrict__ codes, float* __restrict__ loss_part) {
   extern __shared__ __align__(16) unsigned char smem[];
   float(*Rs)[128] = reinterpret_cast<float(*)[128]>(smem);
-  // St: the W block on entry, then column by column η (scaled residual) replaces w
+  // St: the W block on entry, then sub-block by sub-block η (scaled residual) replaces w
   float(*St)[kColLd] = reinterpret_cast<float(*)[kColLd]>(smem + 128 * 128 * 4);
-  float(*Qs)[kColLd] =
-      reinterpret_cast<float(*)[kColLd]>(smem + 128 * 128 * 4 + kColCtaRows * kColLd * 4);
-  uint8_t(*Cs)[136] =
-      reinterpret_cast<uint8_t(*)[136]>(smem + 128 * 128 * 4 + 2 * kColCtaRows * kColLd * 4);
+  float(*lossw)[128] =
+      reinterpret_cast<float(*)[128]>(smem + 128 * 128 * 4 + kColCtaRows * kColLd * 4);
   __shared__ int gs[128];
   __shared__ float rinv[128];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row0 = blockIdx.x * kColCtaRows;
-  const int r = warp * 8 + (lane >> 2);  // row within the CTA
-  const int q = lane & 3;
+  const int r = warp * (32 / kColLanes) + lane / kColLanes;  // row within the CTA
+  const int q = lane % kColLanes;
   const int row = row0 + r;
   const bool active = row < m;
 
-  for (int e = tid; e < 128 * 128; e += blockDim.x) {
-    const int a = e >> 7, b = e & 127;
-    const bool v = a < nb && b < nb && b >= a;
-    cp_async4(&Rs[a][b], v ? R + (long long)(i + a) * d + i + b : R, v);
-  }
-  for (int e = tid; e < kColCtaRows * 128; e += blockDim.x) {
-    const int rr = e >> 7, t = e & 127;
-    const int gr = row0 + rr;
-    const bool v = gr < m && t < nb;
-    cp_async4(&St[rr][t], v ? Wk + (long long)gr * d + i + t : Wk, v);
+  // R[i:i+nb, i:i+nb] and W[rows, i:i+nb], zero-filled beyond nb; 16-byte copies when the
+  // rows are 16-byte aligned
+  const bool vec = (d % 4 == 0) && (i % 4 == 0) && (ldE % 4 == 0) &&
+                   ((reinterpret_cast<uintptr_t>(R) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(Wk) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(E) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(codes) & 3) == 0);
+  if (vec) {
+    for (int e = tid; e < 128 * 32; e += blockDim.x) {
+      const int a = e >> 5, b = (e & 31) * 4;
+      const int bytes = (a < nb && b < nb) ? 4 * min(4, nb - b) : 0;
+      cp_async16(&Rs[a][b], bytes ? R + (long long)(i + a) * d + i + b : R, bytes);
+    }
+    for (int e = tid; e < kColCtaRows * 32; e += blockDim.x) {
+      const int rr = e >> 5, t = (e & 31) * 4;
+      const int gr = row0 + rr;
+      const int bytes = (gr < m && t < nb) ? 4 * min(4, nb - t) : 0;
+      cp_async16(&St[rr][t], bytes ? Wk + (long long)gr * d + i + t : Wk, bytes);
+    }
+  } else {
+    for (int e = tid; e < 128 * 128; e += blockDim.x) {
+      const int a = e >> 7, b = e & 127;
+      const bool v = a < nb && b < nb;
+      cp_async4(&Rs[a][b], v ? R + (long long)(i + a) * d + i + b : R, v);
+    }
+    for (int e = tid; e < kColCtaRows * 128; e += blockDim.x) {
+      const int rr = e >> 7, t = e & 127;
+      const int gr = row0 + rr;
+      const bool v = gr < m && t < nb;
+      cp_async4(&St[rr][t], v ? Wk + (long long)gr * d + i + t : Wk, v);
+    }
   }
   for (int a = tid; a < 128; a += blockDim.x) gs[a] = (a < nb) ? gcol[i + a] : 0;
   cp_async_wait_all();
   __syncthreads();
   for (int a = tid; a < 128; a += blockDim.x) rinv[a] = (a < nb) ? 1.f / Rs[a][a] : 0.f;
-  __syncthreads();
 
   ColStepArgs args;
-  args.Rs = Rs; args.St = St; args.Cs = Cs; args.gs = gs; args.rinv = rinv;
+  args.Rs = Rs; args.gs = gs; args.rinv = rinv;
   args.scales = scales; args.zeros = zeros;
   args.srow = (long long)(active ? row : 0) * ng;
-  args.r = r; args.q = q; args.nb = nb; args.src0 = lane & ~3u; args.active = active;
+  args.q = q; args.src0 = lane & ~(unsigned)(kColLanes - 1);
+  args.active = active;
   args.maxq = (float)((1 << bits) - 1);
-  args.D0 = 1.f; args.Z0 = 0.f;
-  if (UNIFORM && active) {
-    args.D0 = scales[args.srow + gs[0]];
-    args.Z0 = (float)zeros[args.srow + gs[0]];
-  }
-#pragma unroll 1
-  for (int sb = 0; sb < 128 / kColSub; ++sb) {
-    const int off = sb * kColSub;
-    if (off >= nb) break;
-    float w[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) w[t] = St[r][off + q + 4 * t];
-    __syncwarp();
-    // residuals of the earlier sub-blocks: w -= η[0:off] R[0:off, my columns]
-    for (int j = 0; j < off; ++j) {
-      const float e = St[r][j];
-      const float* rrow = &Rs[j][off + q];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) w[t] = fmaf(-e, rrow[4 * t], w[t]);
+  args.D0 = 1.f; args.Z0 = 0.f; args.Y0 = 1.f;
+  bool fast = true;
+  if (UNIFORM) {
+    if (active) {
+      args.D0 = scales[args.srow + gcol[i]];
+      args.Z0 = (float)zeros[args.srow + gcol[i]];
+      args.Y0 = __frcp_rn(args.D0);
+      fast = quotient_fast(args.D0);
     }
-    col_steps<UNIFORM>(w, args, off, std::make_integer_sequence<int, kColSub>{});
-#pragma unroll
-    for (int t = 0; t < 8; ++t) Qs[r][off + q + 4 * t] = w[t];
-    __syncwarp();
+  } else if (active) {
+    for (int t = q; t < nb; t += kColLanes) fast &= quotient_fast(scales[args.srow + gcol[i + t]]);
   }
+  fast = __syncthreads_and(fast);  // also publishes rinv and gs
+  if (fast)
+    col_walk<UNIFORM, true>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, codes);
+  else
+    col_walk<UNIFORM, false>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, codes);
   __syncthreads();
-  // E (scaled residuals), q, codes as row segments; loss partial Σ_rows η² per column
-  for (int rr = 0; rr < kColCtaRows; ++rr) {
-    const int gr = row0 + rr;
-    if (gr >= m) break;
-    for (int t = tid; t < nb; t += blockDim.x) {
-      E[(long long)gr * ldE + t] = St[rr][t];
-      Wk[(long long)gr * d + i + t] = Qs[rr][t];
-      codes[(long long)gr * d + i + t] = Cs[rr][t];
-    }
-  }
+  // loss partial Σ_rows η² per column, the 8 warps' sums in a fixed order
   for (int t = tid; t < nb; t += blockDim.x) {
     float sacc = 0.f;
-    for (int rr = 0; rr < kColCtaRows && row0 + rr < m; ++rr) sacc = fmaf(St[rr][t], St[rr][t], sacc);
+#pragma unroll
+    for (int w8 = 0; w8 < kColWarps; ++w8) sacc += lossw[w8][t];
     loss_part[(long long)blockIdx.x * d + i + t] = sacc;
   }
 }

@@ -42,7 +42,7 @@ int unpermute(Ctx* c, int m, int d, const int32_t* inv, const uint8_t* codes_p,
 int pack_codes(Ctx* c, const uint8_t* codes, int m, int d, int bits, uint32_t* packed);
 int unpack_codes(Ctx* c, const uint32_t* packed, int m, int d, int bits, uint8_t* codes);
 
-constexpr int kColRows = 32;      // rows per column-block CTA (4 warps, 4 lanes per row)
+constexpr int kColRows = 32;      // rows per column-block CTA (8 warps, 8 lanes per row)
 constexpr int kColMax = 128;      // columns per kernel block
 constexpr int kSuperCols = 512;   // columns per super-block of the two-level lazy update
 
