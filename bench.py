@@ -351,7 +351,8 @@ def run_ours(args):
     n_launch = len(chunks)
     achieved = syrk_flops / (syrk_ms / 1e3) / 1e12
     digest = kernel_source_digest(["post_weight_quantization_17_b200/csrc/k_syrk.cu",
-                                   "post_weight_quantization_17_b200/csrc/gemm_simt.cuh"])
+                                   "post_weight_quantization_17_b200/csrc/gemm_simt.cuh",
+                                   "post_weight_quantization_17_b200/csrc/tc_util.cuh"])
     roofline = {"kernel": "hessian_accumulate (S += X^T X)", "bound": "tensor",
                 "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
                 "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16 burst",

@@ -162,8 +162,118 @@ inline int gemm_simt(Ctx* c, const GemmArgs& g) {
   return GPTQ_OK;
 }
 
-// fp32-accurate GEMM: tcgen05 3xTF32 where TMA can take the operands, else CUDA cores
-// (k_gemm_tc.cu).
+// Small GEMMs (the factorization's two lowest recursion levels: up to 256 on a side) are
+// latency bound, so they take 32 x 32 tiles (2 x 2 outputs per thread, 32-deep k-slabs,
+// register prefetch of the next slab): many CTAs, no tensor-core setup, fp32 products.  From
+// 512 on a side, and for tall products such as the trailing update, the tensor path is as fast
+// or faster.
+constexpr int SBM = 32, SBK = 32;
+constexpr int kSmallGemmSide = 256;
+
+template <class TA, class TB>
+__global__ void __launch_bounds__(GTHREADS) k_gemm_small(GemmArgs g) {
+  constexpr int LA = SBM * SBK / GTHREADS;  // 4 elements of each operand per thread and slab
+  __shared__ __align__(16) float As[2][SBK][SBM + 4];  // As[k][i]
+  __shared__ __align__(16) float Bs[2][SBK][SBM + 4];  // Bs[k][j]
+  const int tid = threadIdx.x;
+  const int i0 = blockIdx.y * SBM, j0 = blockIdx.x * SBM;
+  if ((g.flags & kCUpper) && i0 > j0 + SBM - 1) return;
+  if ((g.flags & kCLower) && j0 > i0 + SBM - 1) return;
+  int kbeg = 0, kend = g.K;
+  if (g.flags & kAUpper) kbeg = max(kbeg, i0);
+  if (g.flags & kBLower) kbeg = max(kbeg, j0);
+  if (g.flags & kALower) kend = min(kend, i0 + SBM);
+  if (g.flags & kBUpper) kend = min(kend, j0 + SBM);
+
+  const TA* A = reinterpret_cast<const TA*>(g.A);
+  const TB* B = reinterpret_cast<const TB*>(g.B);
+  const bool a_kcontig = (g.sak == 1);
+  const bool b_ncontig = (g.sbj == 1);
+  float ra[LA], rb[LA];
+  // consecutive threads walk each operand's unit-stride dimension
+  auto a_idx = [&](int e, int& ii, int& kk) {
+    if (a_kcontig) { ii = e / SBK; kk = e % SBK; } else { kk = e / SBM; ii = e % SBM; }
+  };
+  auto b_idx = [&](int e, int& jj, int& kb) {
+    if (b_ncontig) { kb = e / SBM; jj = e % SBM; } else { jj = e / SBK; kb = e % SBK; }
+  };
+  auto load_slab = [&](int k0) {
+#pragma unroll
+    for (int r = 0; r < LA; ++r) {
+      int ii, kk, jj, kb;
+      a_idx(tid + r * GTHREADS, ii, kk);
+      const int gi = i0 + ii, gk = k0 + kk;
+      ra[r] = (gi < g.M && gk < kend && gk >= kbeg)
+                  ? to_f32<TA>(A[(long long)gi * g.sai + (long long)gk * g.sak]) : 0.f;
+      b_idx(tid + r * GTHREADS, jj, kb);
+      const int gj = j0 + jj, gkb = k0 + kb;
+      rb[r] = (gj < g.N && gkb < kend && gkb >= kbeg)
+                  ? to_f32<TB>(B[(long long)gkb * g.sbk + (long long)gj * g.sbj]) : 0.f;
+    }
+  };
+  auto store_slab = [&](int buf) {
+#pragma unroll
+    for (int r = 0; r < LA; ++r) {
+      int ii, kk, jj, kb;
+      a_idx(tid + r * GTHREADS, ii, kk);
+      As[buf][kk][ii] = ra[r];
+      b_idx(tid + r * GTHREADS, jj, kb);
+      Bs[buf][kb][jj] = rb[r];
+    }
+  };
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  kbeg = kbeg / SBK * SBK;
+  if (kbeg < kend) {
+    load_slab(kbeg);
+    store_slab(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = kbeg; k0 < kend; k0 += SBK) {
+      const bool more = k0 + SBK < kend;
+      if (more) load_slab(k0 + SBK);
+#pragma unroll
+      for (int kk = 0; kk < SBK; ++kk) {
+        const float2 a2 = *reinterpret_cast<const float2*>(&As[buf][kk][2 * ty]);
+        const float2 b2 = *reinterpret_cast<const float2*>(&Bs[buf][kk][2 * tx]);
+        acc[0][0] = fmaf(a2.x, b2.x, acc[0][0]);
+        acc[0][1] = fmaf(a2.x, b2.y, acc[0][1]);
+        acc[1][0] = fmaf(a2.y, b2.x, acc[1][0]);
+        acc[1][1] = fmaf(a2.y, b2.y, acc[1][1]);
+      }
+      if (more) {
+        store_slab(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const int gi = i0 + 2 * ty + a;
+    if (gi >= g.M) continue;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int gj = j0 + 2 * tx + b;
+      if (gj >= g.N) continue;
+      float* c = g.C + (long long)gi * g.ldc + gj;
+      const float v = g.alpha * acc[a][b];
+      *c = (g.beta == 0.f) ? v : fmaf(g.beta, *c, v);
+    }
+  }
+}
+
+template <class TA = float, class TB = float>
+inline int gemm_small(Ctx* c, const GemmArgs& g) {
+  if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
+  dim3 grid((g.N + SBM - 1) / SBM, (g.M + SBM - 1) / SBM);
+  k_gemm_small<TA, TB><<<grid, GTHREADS, 0, c->stream>>>(g);
+  GPTQ_LAUNCH_CHECK(c);
+  return GPTQ_OK;
+}
+
+// fp32-accurate GEMM: small ones on CUDA cores (gemm_small), else tcgen05 3xTF32 where TMA can
+// take the operands, else CUDA cores (k_gemm_tc.cu).
 int gemm_f32(Ctx* c, const GemmArgs& g);
 
 }  // namespace gptq

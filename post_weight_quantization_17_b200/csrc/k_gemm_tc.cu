@@ -409,10 +409,11 @@ int gemm_tc(Ctx* c, const GemmArgs& g) {
   return GPTQ_OK;
 }
 
-// fp32 GEMM entry used by the factorization and the trailing update: tensor cores where the
-// operands allow TMA, CUDA cores otherwise.
+// fp32 GEMM entry used by the factorization and the trailing update: small products on CUDA
+// cores with small tiles, tensor cores where the operands allow TMA, CUDA cores otherwise.
 int gemm_f32(Ctx* c, const GemmArgs& g) {
   if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
+  if (g.M <= kSmallGemmSide && g.N <= kSmallGemmSide) return gemm_small(c, g);
   if (gemm_tc_applies(g)) return gemm_tc(c, g);
   return gemm_simt(c, g);
 }

@@ -7,12 +7,14 @@
 // B[j, t] = X[t, 256 J + j].  Products of two 16-bit values are exact in fp32.
 //   warp 0      TMA producer: 64-token slabs of A (2 boxes) and B (4 boxes), 4-stage ring
 //   warp 1      MMA issuer: tcgen05.mma kind::f16, M=128 N=256 K=16, fp32 partial sums in TMEM
-//   warps 2..9  epilogue: every SY_KP tokens the TMEM partial is added (fp32, round to
+//   warps 2..9  epilogue: every SY_KP (512) tokens the TMEM partial is added (fp32, round to
 //               nearest) into a 128 x 256 accumulator held in the epilogue warps' registers
 //               (each thread: one row, 128 columns); at the end of the tile it goes to S.
 // The tensor core's own fp32 accumulation loses precision roughly in proportion to the number
-// of MMA steps it sums, so partial sums are kept short (256 tokens) and the long sum over all
-// tokens is done with IEEE adds.  Two TMEM partial buffers let the MMA run ahead of the adds.
+// of MMA steps it sums, so partial sums are kept short (512 tokens) and the long sum over all
+// tokens is done with IEEE adds (512-token partials give the same error as 256-token ones on 262144
+// tokens, measured; 1024 doubles it).  Two TMEM partial buffers let the MMA run ahead of the
+// adds.
 // Every wait is bounded; a wait that runs out records GPTQ_ERR_TIMEOUT and the CTA unwinds
 // (drains its own TMA copies, frees TMEM) instead of hanging.
 //
@@ -24,7 +26,7 @@
 namespace gptq {
 
 constexpr int SY_BM = 128, SY_BN = 256, SY_BK = 64, SY_STAGES = 4;
-constexpr int SY_KP = 256;                               // tokens per TMEM partial sum
+constexpr int SY_KP = 512;                               // tokens per TMEM partial sum
 constexpr int SY_KB_PER_PART = SY_KP / SY_BK;
 constexpr int SY_BOX_BYTES = SY_BK * 64 * 2;             // one 64 x 64 box of 16-bit values
 constexpr int SY_A_BYTES = (SY_BM / 64) * SY_BOX_BYTES;  // 16 KB
@@ -253,6 +255,267 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
 }
 
 // ------------------------------------------------------------------------------------------
+// The same statistic on CTA pairs (cluster of 2, tcgen05 cta_group::2): 256 x 256 output tiles
+// touching the lower triangle, M = N = 256 per MMA.  CTA r of the pair loads tile rows
+// 128 r .. 128 r + 127 (A) and tile columns 128 r .. 128 r + 127 (its half of B) into its own
+// shared memory; the tensor cores of both SMs read both halves of B, so each SM moves 32 KB
+// per 64-token stage for the work that took 48 KB on one SM (shared-memory bandwidth was the
+// single-SM limit).  Each CTA's TMEM receives its 128 rows of the tile and its own epilogue
+// warps fold them into S exactly as above.
+//   warp 0      both CTAs: TMA producer of its own halves (no multicast), 6-stage ring; the
+//               copies of both CTAs complete on the leader's (rank 0) stage barrier, which the
+//               leader arms for the bytes of both
+//   warp 1      leader: MMA issuer; commits arrive on the barriers of both CTAs
+//   warps 2..9  both CTAs: epilogue; a finished TMEM buffer is released to the leader by one
+//               arrive per warp (remote for the peer)
+// Every wait is bounded; both CTAs pass a cluster barrier before TMEM is freed or either exits
+// (the leader has then seen every stage of both CTAs land).
+constexpr int S2_BM = 128;                                // tile rows per CTA (256 per pair)
+constexpr int S2_BN = 256;                                // tile columns (128 per CTA's B half)
+constexpr int S2_STAGES = 6;
+constexpr int S2_A_BYTES = (S2_BM / 64) * SY_BOX_BYTES;   // 16 KB
+constexpr int S2_B_BYTES = (S2_BN / 128) * SY_BOX_BYTES;  // 16 KB: this CTA's 128 columns
+constexpr int S2_STAGE_BYTES = S2_A_BYTES + S2_B_BYTES;
+constexpr int S2_SMEM = S2_STAGES * S2_STAGE_BYTES + 1024 + 256;
+
+__device__ __forceinline__ void syrk2_tile_coords(int t, int& I, int& J) {
+  int i = 0;
+  for (;;) {
+    if (t <= i) {  // row-block i of 256 has tiles J = 0 .. i
+      I = i;
+      J = t;
+      return;
+    }
+    t -= i + 1;
+    ++i;
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
+    k_syrk_tc2(const __grid_constant__ CUtensorMap tmap, float* __restrict__ S, int d,
+               int n_tokens, int accumulate, int num_tiles, uint32_t idesc, DeviceStatus* st,
+               long long budget) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S2_STAGES * S2_STAGE_BYTES);
+  uint64_t* empty = full + S2_STAGES;
+  uint64_t* tfull = empty + S2_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = tc::cluster_rank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S2_STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(&tfull[a], 1);
+      tc::mbar_init(&tempty[a], 2 * SY_EPI_WARPS);
+    }
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) tc::prefetch_tmap(&tmap);
+  tc::cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  if (warp == 1) tc::tmem_alloc_pair(tmem_slot, 512);
+  tc::fence_before_sync();
+  tc::cluster_sync();  // TMEM allocated in both CTAs before the leader's first MMA
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int kblocks = (n_tokens + SY_BK - 1) / SY_BK;
+  const int nparts = (kblocks + SY_KB_PER_PART - 1) / SY_KB_PER_PART;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued[S2_STAGES] = {};
+      uint32_t issued_phase[S2_STAGES] = {};
+      const uint32_t leader_full = tc::map_to_rank(full, 0);
+      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+        int I, J;
+        syrk2_tile_coords(t, I, J);
+        const int ra = 256 * I + S2_BM * rank, rb = 256 * J + 128 * rank;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!tc::mbar_wait_cluster(&empty[stage], phase ^ 1, budget)) {
+            raise_error(st, GPTQ_ERR_TIMEOUT, 21);
+            *abort_flag = 1;
+            break;
+          }
+          uint8_t* sA = smem + stage * S2_STAGE_BYTES;
+          uint8_t* sB = sA + S2_A_BYTES;
+          if (rank == 0) tc::mbar_expect_tx(&full[stage], 2 * S2_STAGE_BYTES);
+          const uint32_t bar = leader_full + 8u * stage;
+          const int y = kb * SY_BK;
+          tc::tma_load_2d_pair(sA, &tmap, bar, ra, y);
+          tc::tma_load_2d_pair(sA + SY_BOX_BYTES, &tmap, bar, ra + 64, y);
+          tc::tma_load_2d_pair(sB, &tmap, bar, rb, y);
+          tc::tma_load_2d_pair(sB + SY_BOX_BYTES, &tmap, bar, rb + 64, y);
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == S2_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // drain: the leader's stage barriers count both CTAs' copies
+      if (rank == 0)
+        for (int s = 0; s < S2_STAGES; ++s)
+          if (issued[s] && !tc::mbar_wait_cluster(&full[s], issued_phase[s], budget))
+            raise_error(st, GPTQ_ERR_TIMEOUT, 22);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---- leader: MMA issuer for the pair
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, any = false;
+      for (int t = pair; t < num_tiles && ok && !*abort_flag; t += npairs) {
+        for (int p = 0; p < nparts && ok; ++p) {
+          if (!tc::mbar_wait_cluster(&tempty[acc], acc_phase ^ 1, budget)) {
+            raise_error(st, GPTQ_ERR_TIMEOUT, 23);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t d_tmem = tmem + acc * S2_BN;
+          const int kb1 = min(kblocks, (p + 1) * SY_KB_PER_PART);
+          for (int kb = p * SY_KB_PER_PART; kb < kb1; ++kb) {
+            if (!tc::mbar_wait_cluster(&full[stage], phase, budget)) {
+              raise_error(st, GPTQ_ERR_TIMEOUT, 24);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+            const uint32_t a0 = tc::smem_u32(smem + stage * S2_STAGE_BYTES);
+            const uint32_t b0 = a0 + S2_A_BYTES;
+            const bool first = (kb == p * SY_KB_PER_PART);
+#pragma unroll
+            for (int kk = 0; kk < SY_BK / 16; ++kk) {
+              const uint64_t ad = tc::sdesc_sw128(a0 + kk * 2048, SY_BOX_BYTES, 1024);
+              const uint64_t bd = tc::sdesc_sw128(b0 + kk * 2048, SY_BOX_BYTES, 1024);
+              tc::mma_f16_pair(d_tmem, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+            }
+            any = true;
+            tc::mma_commit_pair(&empty[stage]);
+            if (++stage == S2_STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (!ok) break;
+          tc::mma_commit_pair(&tfull[acc]);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1;
+          }
+        }
+      }
+      // every MMA of the pair has completed before either CTA may free TMEM or exit
+      if (any) {
+        tc::mma_commit_pair(drain);
+        if (!tc::mbar_wait(drain, 0, budget)) raise_error(st, GPTQ_ERR_TIMEOUT, 25);
+      }
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and the 128-column half h
+    const int q = warp & 3;
+    const int h = (warp - 2) / 4;
+    const int r = 32 * q + lane;
+    const uint32_t leader_tempty = tc::map_to_rank(tempty, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int t = pair; t < num_tiles && ok && !*abort_flag; t += npairs) {
+      int I, J;
+      syrk2_tile_coords(t, I, J);
+      float m[128];
+#pragma unroll
+      for (int u = 0; u < 128; ++u) m[u] = 0.f;
+      for (int p = 0; p < nparts; ++p) {
+        if (!tc::mbar_wait_cluster(&tfull[acc], acc_phase, budget)) {
+          raise_error(st, GPTQ_ERR_TIMEOUT, 27);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t base = tmem + acc * S2_BN + ((uint32_t)(32 * q) << 16) + h * 128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tc::tmem_ld32(base + cc * 32, v);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) m[cc * 32 + u] += __uint_as_float(v[u]);
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0)
+            tc::mbar_arrive(&tempty[acc]);
+          else
+            tc::mbar_arrive_remote(leader_tempty + 8u * acc);
+        }
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      const int gi = 256 * I + S2_BM * rank + r;
+      if (gi < d) {
+        float* srow = S + (long long)gi * d;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int gj0 = 256 * J + h * 128 + cc * 32;
+          if (gj0 > gi) continue;
+          if (gj0 + 31 <= gi && gj0 + 32 <= d) {
+            float4* p4 = reinterpret_cast<float4*>(srow + gj0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4 x = make_float4(m[cc * 32 + 4 * u], m[cc * 32 + 4 * u + 1],
+                                     m[cc * 32 + 4 * u + 2], m[cc * 32 + 4 * u + 3]);
+              if (accumulate) {
+                const float4 o = p4[u];
+                x.x += o.x; x.y += o.y; x.z += o.z; x.w += o.w;
+              }
+              p4[u] = x;
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const int gj = gj0 + u;
+              if (gj <= gi && gj < d) {
+                const float x = m[cc * 32 + u];
+                srow[gj] = accumulate ? srow[gj] + x : x;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::cluster_sync();  // no CTA frees TMEM or leaves while its pair may still touch it
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -280,13 +543,28 @@ int syrk_tc(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) GPTQ_SET_ERR(c, GPTQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  const uint32_t fmt = dtype == GPTQ_BF16 ? 1u : 0u;
+  if (d >= 256 && c->num_sms >= 2) {
+    // CTA pairs over 256 x 256 tiles
+    const int nI = (d + 255) / 256;
+    const int num_tiles = nI * (nI + 1) / 2;
+    const int grid = 2 * std::min(num_tiles, c->num_sms / 2);
+    GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_syrk_tc2,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM));
+    const uint32_t idesc = tc::idesc_f32acc(fmt, true, true, 2 * S2_BM, S2_BN);
+    k_syrk_tc2<<<grid, SY_THREADS, S2_SMEM, c->stream>>>(map, S, d, (int)n, overwrite ? 0 : 1,
+                                                         num_tiles, idesc, c->status,
+                                                         c->timeout_cycles);
+    GPTQ_LAUNCH_CHECK(c);
+    return GPTQ_OK;
+  }
   const int nI = (d + SY_BM - 1) / SY_BM;
   int num_tiles = 0;
   for (int i = 0; i < nI; ++i) num_tiles += i / 2 + 1;
   const int grid = std::min(num_tiles, c->num_sms);
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_syrk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           SY_SMEM));
-  const uint32_t idesc = tc::idesc_f32acc(dtype == GPTQ_BF16 ? 1u : 0u, true, true, SY_BM, SY_BN);
+  const uint32_t idesc = tc::idesc_f32acc(fmt, true, true, SY_BM, SY_BN);
   k_syrk_tc<<<grid, SY_THREADS, SY_SMEM, c->stream>>>(map, S, d, (int)n, overwrite ? 0 : 1,
                                                       num_tiles, idesc, c->status,
                                                       c->timeout_cycles);
