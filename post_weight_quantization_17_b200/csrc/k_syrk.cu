@@ -12,9 +12,9 @@
 //               (each thread: one row, 128 columns); at the end of the tile it goes to S.
 // The tensor core's own fp32 accumulation loses precision roughly in proportion to the number
 // of MMA steps it sums, so partial sums are kept short (512 tokens) and the long sum over all
-// tokens is done with IEEE adds (512-token partials give the same error as 256-token ones on 262144
-// tokens, measured; 1024 doubles it).  Two TMEM partial buffers let the MMA run ahead of the
-// adds.
+// tokens is done with IEEE adds.  Measured H error against fp64: <= 1.4e-6 with 512-token
+// partials on the parity cases (<= 7e-7 with 256, 1.2e-5 with 4096); 512 halves the hand-offs
+// between MMA and epilogue.  Two TMEM partial buffers let the MMA run ahead of the adds.
 // Every wait is bounded; a wait that runs out records GPTQ_ERR_TIMEOUT and the CTA unwinds
 // (drains its own TMA copies, frees TMEM) instead of hanging.
 //
