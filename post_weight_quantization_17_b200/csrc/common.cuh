@@ -6,6 +6,7 @@
 #include <stdint.h>
 #include <stdio.h>
 #include <string>
+#include <utility>
 
 #include "../../include/gptq.h"
 
@@ -57,6 +58,36 @@ __device__ __forceinline__ void raise_error(DeviceStatus* st, int code, int wher
   if (atomicCAS(&st->code, 0, code) == 0) st->where = where;
 }
 
+// ---- programmatic dependent launch
+// Every kernel is launched with programmatic stream serialization, so it may start while the
+// previous kernel of its stream is still running.  Before its first access to memory that the
+// previous kernel writes (or reads, for memory this kernel writes) it calls pdl_wait(), which
+// returns once that kernel has completed and its writes are visible, and only after that
+// pdl_release(), which lets the next kernel start its own set-up.  A kernel that has not waited
+// yet may therefore read data written two or more kernels back, never data of the kernel right
+// before it.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(Ctx* c, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                              size_t smem, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c->stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ++c->launches;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <class T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
@@ -82,8 +113,5 @@ template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16
                    cudaGetErrorString(_e), __FILE__, __LINE__);                 \
   } while (0)
 
-#define GPTQ_LAUNCH_CHECK(ctx)                                                  \
-  do {                                                                          \
-    (ctx)->launches++;                                                          \
-    GPTQ_CUDA_CHECK(ctx, cudaGetLastError());                                   \
-  } while (0)
+// Launches a kernel on the context's stream (programmatic dependent launch, counted).
+#define GPTQ_LAUNCH(ctx, ...) GPTQ_CUDA_CHECK(ctx, ::gptq::launch_pdl(ctx, __VA_ARGS__))

@@ -31,6 +31,8 @@ constexpr int GBK = 8, GTHREADS = 256;
 // 4 rows / 4 columns spaced BM/2 (BN/2) apart, so that the shared-memory reads are float4s.
 template <class TA, class TB, int BM, int BN>
 __global__ void __launch_bounds__(GTHREADS) k_gemm_simt(GemmArgs g) {
+  pdl_wait();
+  pdl_release();
   constexpr int TM = BM / 16, TN = BN / 16;          // 8 or 4
   constexpr int LA = BM * GBK / GTHREADS, LB = BN * GBK / GTHREADS;
   __shared__ __align__(16) float As[2][GBK][BM + 4];
@@ -153,12 +155,11 @@ inline int gemm_simt(Ctx* c, const GemmArgs& g) {
   const long long big = (long long)((g.N + 127) / 128) * ((g.M + 127) / 128);
   if (big >= 2LL * c->num_sms) {
     dim3 grid((g.N + 127) / 128, (g.M + 127) / 128);
-    k_gemm_simt<TA, TB, 128, 128><<<grid, GTHREADS, 0, c->stream>>>(g);
+    GPTQ_LAUNCH(c, k_gemm_simt<TA, TB, 128, 128>, grid, GTHREADS, 0, g);
   } else {
     dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
-    k_gemm_simt<TA, TB, 64, 64><<<grid, GTHREADS, 0, c->stream>>>(g);
+    GPTQ_LAUNCH(c, k_gemm_simt<TA, TB, 64, 64>, grid, GTHREADS, 0, g);
   }
-  GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
 }
 
@@ -172,6 +173,8 @@ constexpr int kSmallGemmSide = 256;
 
 template <class TA, class TB>
 __global__ void __launch_bounds__(GTHREADS) k_gemm_small(GemmArgs g) {
+  pdl_wait();
+  pdl_release();
   constexpr int LA = SBM * SBK / GTHREADS;  // 4 elements of each operand per thread and slab
   __shared__ __align__(16) float As[2][SBK][SBM + 4];  // As[k][i]
   __shared__ __align__(16) float Bs[2][SBK][SBM + 4];  // Bs[k][j]
@@ -267,8 +270,7 @@ template <class TA = float, class TB = float>
 inline int gemm_small(Ctx* c, const GemmArgs& g) {
   if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
   dim3 grid((g.N + SBM - 1) / SBM, (g.M + SBM - 1) / SBM);
-  k_gemm_small<TA, TB><<<grid, GTHREADS, 0, c->stream>>>(g);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_gemm_small<TA, TB>, grid, GTHREADS, 0, g);
   return GPTQ_OK;
 }
 

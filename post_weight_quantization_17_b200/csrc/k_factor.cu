@@ -60,6 +60,8 @@ __device__ __forceinline__ float recip_sqrt(float p) {
 // precedes its next overwrite).  Indices >= n are padded with the identity.
 __global__ void __launch_bounds__(FB_THREADS, 1) k_factor_base(float* __restrict__ M, long long ld,
                                                                 int s, int n, DeviceStatus* st) {
+  pdl_wait();
+  pdl_release();
   extern __shared__ __align__(16) float fsm[];
   float(*S)[FB_LDS] = reinterpret_cast<float(*)[FB_LDS]>(fsm);       // staging (load phase)
   float(*tile)[8][FB] = reinterpret_cast<float(*)[8][FB]>(fsm);       // 2 x 8 pivot rows (after)
@@ -185,6 +187,8 @@ __global__ void __launch_bounds__(FB_THREADS, 1) k_factor_base(float* __restrict
 
 __global__ void k_copy2d(const float* __restrict__ src, long long lds, float* __restrict__ dst,
                          long long ldd, int rows, int cols) {
+  pdl_wait();
+  pdl_release();
   long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   long long total = (long long)rows * cols;
   for (; e < total; e += (long long)gridDim.x * blockDim.x) {
@@ -198,8 +202,7 @@ static int copy2d(Ctx* c, const float* src, long long lds, float* dst, long long
   long long total = (long long)rows * cols;
   if (total <= 0) return GPTQ_OK;
   int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
-  k_copy2d<<<blocks, 256, 0, c->stream>>>(src, lds, dst, ldd, rows, cols);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_copy2d, blocks, 256, 0, src, lds, dst, ldd, rows, cols);
   return GPTQ_OK;
 }
 
@@ -235,8 +238,7 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   float* M = f.M;
   const int n = e - s;
   if (n <= FB) {
-    k_factor_base<<<1, FB_THREADS, FB_SMEM, c->stream>>>(M, ld, s, n, c->status);
-    GPTQ_LAUNCH_CHECK(c);
+    GPTQ_LAUNCH(c, k_factor_base, 1, FB_THREADS, FB_SMEM, M, ld, s, n, c->status);
     return GPTQ_OK;
   }
   const int n1 = larger_child(n);  // < n for n > FB

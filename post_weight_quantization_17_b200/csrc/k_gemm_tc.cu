@@ -106,6 +106,9 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // set-up above overlaps the previous kernel; its outputs are read only from here on
+  pdl_wait();
+  pdl_release();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -404,8 +407,7 @@ int gemm_tc(Ctx* c, const GemmArgs& g) {
   const int grid = std::min(p.num_tiles, c->num_sms);
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           GT_SMEM));
-  k_gemm_tc<<<grid, GT_THREADS, GT_SMEM, c->stream>>>(ma, mb, p, c->status, c->timeout_cycles);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_gemm_tc, grid, GT_THREADS, GT_SMEM, ma, mb, p, c->status, c->timeout_cycles);
   return GPTQ_OK;
 }
 

@@ -8,6 +8,8 @@ namespace gptq {
 
 __global__ void k_pack(const uint8_t* __restrict__ codes, int m, int d, int bits,
                        uint32_t* __restrict__ packed, int wpr) {
+  pdl_wait();
+  pdl_release();
   const int chunks = (d + 31) / 32;
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= (long long)m * chunks) return;
@@ -45,6 +47,8 @@ __global__ void k_pack(const uint8_t* __restrict__ codes, int m, int d, int bits
 
 __global__ void k_unpack(const uint32_t* __restrict__ packed, int m, int d, int bits,
                          uint8_t* __restrict__ codes, int wpr) {
+  pdl_wait();
+  pdl_release();
   const int chunks = (d + 31) / 32;
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= (long long)m * chunks) return;
@@ -70,16 +74,14 @@ __global__ void k_unpack(const uint32_t* __restrict__ packed, int m, int d, int 
 int pack_codes(Ctx* c, const uint8_t* codes, int m, int d, int bits, uint32_t* packed) {
   const int wpr = (int)(((long long)d * bits + 31) / 32);
   const long long threads = (long long)m * ((d + 31) / 32);
-  k_pack<<<(int)((threads + 255) / 256), 256, 0, c->stream>>>(codes, m, d, bits, packed, wpr);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_pack, (int)((threads + 255) / 256), 256, 0, codes, m, d, bits, packed, wpr);
   return GPTQ_OK;
 }
 
 int unpack_codes(Ctx* c, const uint32_t* packed, int m, int d, int bits, uint8_t* codes) {
   const int wpr = (int)(((long long)d * bits + 31) / 32);
   const long long threads = (long long)m * ((d + 31) / 32);
-  k_unpack<<<(int)((threads + 255) / 256), 256, 0, c->stream>>>(packed, m, d, bits, codes, wpr);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_unpack, (int)((threads + 255) / 256), 256, 0, packed, m, d, bits, codes, wpr);
   return GPTQ_OK;
 }
 

@@ -7,6 +7,8 @@ namespace gptq {
 // diag(H) = scale * diag(S); dead where it is exactly 0 (then replaced by 1).
 __global__ void k_diag(const float* __restrict__ S, int d, float scale, float* __restrict__ diagv,
                        uint8_t* __restrict__ dead, DeviceStatus* st) {
+  pdl_wait();
+  pdl_release();
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= d) return;
   float h = S[(long long)j * d + j] * scale;
@@ -17,14 +19,15 @@ __global__ void k_diag(const float* __restrict__ S, int d, float scale, float* _
 }
 
 int prep_diag(Ctx* c, const float* S, int d, float scale, float* diagv, uint8_t* dead) {
-  k_diag<<<(d + 255) / 256, 256, 0, c->stream>>>(S, d, scale, diagv, dead, c->status);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_diag, (d + 255) / 256, 256, 0, S, d, scale, diagv, dead, c->status);
   return GPTQ_OK;
 }
 
 // Deterministic fp64 sum of diag(H') (one CTA; the permutation does not change the mean).
 __global__ void __launch_bounds__(1024) k_mean(const float* __restrict__ diagv, int d,
                                                DeviceStatus* st) {
+  pdl_wait();
+  pdl_release();
   __shared__ double part[32];
   double acc = 0.0;
   for (int j = threadIdx.x; j < d; j += blockDim.x) acc += (double)diagv[j];
@@ -39,8 +42,7 @@ __global__ void __launch_bounds__(1024) k_mean(const float* __restrict__ diagv, 
 }
 
 int prep_mean(Ctx* c, const float* diagv, int d) {
-  k_mean<<<1, 1024, 0, c->stream>>>(diagv, d, c->status);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_mean, 1, 1024, 0, diagv, d, c->status);
   return GPTQ_OK;
 }
 
@@ -48,6 +50,8 @@ int prep_mean(Ctx* c, const float* diagv, int d) {
 // i.e. a stable sort by descending diag(H).
 __global__ void __launch_bounds__(256) k_rank(const float* __restrict__ diagv, int d,
                                               int32_t* __restrict__ perm) {
+  pdl_wait();
+  pdl_release();
   __shared__ float tile[1024];
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   const float v = (j < d) ? diagv[j] : 0.f;
@@ -68,14 +72,15 @@ __global__ void __launch_bounds__(256) k_rank(const float* __restrict__ diagv, i
 }
 
 __global__ void k_iota(int32_t* p, int d) {
+  pdl_wait();
+  pdl_release();
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j < d) p[j] = j;
 }
 
 int prep_perm(Ctx* c, const float* diagv, int d, int act_order, int32_t* perm) {
-  if (act_order) k_rank<<<(d + 255) / 256, 256, 0, c->stream>>>(diagv, d, perm);
-  else k_iota<<<(d + 255) / 256, 256, 0, c->stream>>>(perm, d);
-  GPTQ_LAUNCH_CHECK(c);
+  if (act_order) GPTQ_LAUNCH(c, k_rank, (d + 255) / 256, 256, 0, diagv, d, perm);
+  else GPTQ_LAUNCH(c, k_iota, (d + 255) / 256, 256, 0, perm, d);
   return GPTQ_OK;
 }
 
@@ -84,6 +89,8 @@ int prep_perm(Ctx* c, const float* diagv, int d, int act_order, int32_t* perm) {
 // transposed through shared memory.
 __global__ void k_build_identity(const float* __restrict__ S, int d, float scale,
                                  const float* __restrict__ diagv, float* __restrict__ Hp) {
+  pdl_wait();
+  pdl_release();
   __shared__ float lo[32][33];
   __shared__ float up[32][33];
   const int tr = blockIdx.y * 32, tc = blockIdx.x * 32;
@@ -109,6 +116,8 @@ __global__ void k_build_identity(const float* __restrict__ S, int d, float scale
 __global__ void k_build_perm(const float* __restrict__ S, int d, float scale,
                              const float* __restrict__ diagv, const int32_t* __restrict__ perm,
                              float* __restrict__ Hp) {
+  pdl_wait();
+  pdl_release();
   const int a = blockIdx.y;
   const int pa = perm[a];
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < d; b += gridDim.x * blockDim.x) {
@@ -127,17 +136,18 @@ int prep_build(Ctx* c, const float* S, int d, float scale, const float* diagv,
                const int32_t* perm, bool identity, float* Hp) {
   if (identity) {
     dim3 grid((d + 31) / 32, (d + 31) / 32), block(32, 8);
-    k_build_identity<<<grid, block, 0, c->stream>>>(S, d, scale, diagv, Hp);
+    GPTQ_LAUNCH(c, k_build_identity, grid, block, 0, S, d, scale, diagv, Hp);
   } else {
     dim3 grid((d + 255) / 256 < 8 ? (d + 255) / 256 : 8, d);
-    k_build_perm<<<grid, 256, 0, c->stream>>>(S, d, scale, diagv, perm, Hp);
+    GPTQ_LAUNCH(c, k_build_perm, grid, 256, 0, S, d, scale, diagv, perm, Hp);
   }
-  GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
 }
 
 __global__ void k_copy(const float* __restrict__ src, float* __restrict__ dst, size_t n,
                        bool vec) {
+  pdl_wait();
+  pdl_release();
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   size_t n4 = vec ? n / 4 : 0;
@@ -151,13 +161,14 @@ int prep_copy(Ctx* c, const float* src, float* dst, size_t count) {
   size_t work = vec ? count / 4 + 4 : count;
   int blocks = (int)std::min<size_t>((work + 255) / 256, (size_t)c->num_sms * 8);
   if (blocks < 1) blocks = 1;
-  k_copy<<<blocks, 256, 0, c->stream>>>(src, dst, count, vec);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_copy, blocks, 256, 0, src, dst, count, vec);
   return GPTQ_OK;
 }
 
 // λ = max(percdamp * mean(diag H'), 2^-23); H_λ = H' + λ I (in place on the diagonal).
 __global__ void k_damp(float* __restrict__ Hl, int d, float percdamp, DeviceStatus* st) {
+  pdl_wait();
+  pdl_release();
   const double mean = st->dsum;
   const double lam_d = fmax((double)percdamp * mean, 1.1920928955078125e-07);
   const float lam = (float)lam_d;
@@ -167,8 +178,7 @@ __global__ void k_damp(float* __restrict__ Hl, int d, float percdamp, DeviceStat
 }
 
 int prep_damp(Ctx* c, float* Hl, int d, float percdamp) {
-  k_damp<<<(d + 255) / 256, 256, 0, c->stream>>>(Hl, d, percdamp, c->status);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_damp, (d + 255) / 256, 256, 0, Hl, d, percdamp, c->status);
   return GPTQ_OK;
 }
 

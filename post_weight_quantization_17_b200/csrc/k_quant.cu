@@ -20,6 +20,8 @@ template <class T>
 __global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, int bits,
                           float* __restrict__ scales, int32_t* __restrict__ zeros,
                           DeviceStatus* st) {
+  pdl_wait();
+  pdl_release();
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= (long long)m * ng) return;
@@ -56,12 +58,11 @@ int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int gro
   const long long warps = (long long)m * ng;
   const int blocks = (int)((warps * 32 + 255) / 256);
   if (w_dtype == GPTQ_F16)
-    k_gridfit<__half><<<blocks, 256, 0, c->stream>>>((const __half*)W, m, d, g, ng, bits, scales, zeros, c->status);
+    GPTQ_LAUNCH(c, k_gridfit<__half>, blocks, 256, 0, (const __half*)W, m, d, g, ng, bits, scales, zeros, c->status);
   else if (w_dtype == GPTQ_BF16)
-    k_gridfit<__nv_bfloat16><<<blocks, 256, 0, c->stream>>>((const __nv_bfloat16*)W, m, d, g, ng, bits, scales, zeros, c->status);
+    GPTQ_LAUNCH(c, k_gridfit<__nv_bfloat16>, blocks, 256, 0, (const __nv_bfloat16*)W, m, d, g, ng, bits, scales, zeros, c->status);
   else
-    k_gridfit<float><<<blocks, 256, 0, c->stream>>>((const float*)W, m, d, g, ng, bits, scales, zeros, c->status);
-  GPTQ_LAUNCH_CHECK(c);
+    GPTQ_LAUNCH(c, k_gridfit<float>, blocks, 256, 0, (const float*)W, m, d, g, ng, bits, scales, zeros, c->status);
   return GPTQ_OK;
 }
 
@@ -69,6 +70,8 @@ int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int gro
 // permutation.
 __global__ void k_gcol(const int32_t* __restrict__ perm, int d, int group,
                        int32_t* __restrict__ gcol, int32_t* __restrict__ inv) {
+  pdl_wait();
+  pdl_release();
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= d) return;
   int p = perm ? perm[j] : j;
@@ -77,8 +80,7 @@ __global__ void k_gcol(const int32_t* __restrict__ perm, int d, int group,
 }
 
 int make_gcol(Ctx* c, const int32_t* perm, int d, int group, int32_t* gcol, int32_t* inv) {
-  k_gcol<<<(d + 255) / 256, 256, 0, c->stream>>>(perm, d, group, gcol, inv);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_gcol, (d + 255) / 256, 256, 0, perm, d, group, gcol, inv);
   return GPTQ_OK;
 }
 
@@ -87,6 +89,8 @@ template <class T>
 __global__ void k_init_work(const T* __restrict__ W, long long m, int d,
                             const int32_t* __restrict__ perm, const uint8_t* __restrict__ dead,
                             float* __restrict__ Wk) {
+  pdl_wait();
+  pdl_release();
   const long long total = m * d;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
@@ -104,12 +108,11 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
   const long long total = (long long)m * d;
   int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
   if (w_dtype == GPTQ_F16)
-    k_init_work<__half><<<blocks, 256, 0, c->stream>>>((const __half*)W, m, d, perm, dead, Wk);
+    GPTQ_LAUNCH(c, k_init_work<__half>, blocks, 256, 0, (const __half*)W, m, d, perm, dead, Wk);
   else if (w_dtype == GPTQ_BF16)
-    k_init_work<__nv_bfloat16><<<blocks, 256, 0, c->stream>>>((const __nv_bfloat16*)W, m, d, perm, dead, Wk);
+    GPTQ_LAUNCH(c, k_init_work<__nv_bfloat16>, blocks, 256, 0, (const __nv_bfloat16*)W, m, d, perm, dead, Wk);
   else
-    k_init_work<float><<<blocks, 256, 0, c->stream>>>((const float*)W, m, d, perm, dead, Wk);
-  GPTQ_LAUNCH_CHECK(c);
+    GPTQ_LAUNCH(c, k_init_work<float>, blocks, 256, 0, (const float*)W, m, d, perm, dead, Wk);
   return GPTQ_OK;
 }
 
@@ -312,17 +315,13 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
                    ((reinterpret_cast<uintptr_t>(Wk) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(E) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(codes) & 3) == 0);
+  // R was written before the previous kernel (the factorization, or an earlier block's
+  // kernels), so its copies start before the wait; the W block is the previous kernel's output
   if (vec) {
     for (int e = tid; e < 128 * 32; e += blockDim.x) {
       const int a = e >> 5, b = (e & 31) * 4;
       const int bytes = (a < nb && b < nb) ? 4 * min(4, nb - b) : 0;
       cp_async16(&Rs[a][b], bytes ? R + (long long)(i + a) * d + i + b : R, bytes);
-    }
-    for (int e = tid; e < kColCtaRows * 32; e += blockDim.x) {
-      const int rr = e >> 5, t = (e & 31) * 4;
-      const int gr = row0 + rr;
-      const int bytes = (gr < m && t < nb) ? 4 * min(4, nb - t) : 0;
-      cp_async16(&St[rr][t], bytes ? Wk + (long long)gr * d + i + t : Wk, bytes);
     }
   } else {
     for (int e = tid; e < 128 * 128; e += blockDim.x) {
@@ -330,6 +329,17 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
       const bool v = a < nb && b < nb;
       cp_async4(&Rs[a][b], v ? R + (long long)(i + a) * d + i + b : R, v);
     }
+  }
+  pdl_wait();
+  pdl_release();
+  if (vec) {
+    for (int e = tid; e < kColCtaRows * 32; e += blockDim.x) {
+      const int rr = e >> 5, t = (e & 31) * 4;
+      const int gr = row0 + rr;
+      const int bytes = (gr < m && t < nb) ? 4 * min(4, nb - t) : 0;
+      cp_async16(&St[rr][t], bytes ? Wk + (long long)gr * d + i + t : Wk, bytes);
+    }
+  } else {
     for (int e = tid; e < kColCtaRows * 128; e += blockDim.x) {
       const int rr = e >> 7, t = e & 127;
       const int gr = row0 + rr;
@@ -386,12 +396,11 @@ int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   const int blocks = (m + kColCtaRows - 1) / kColCtaRows;
   if (uniform_grid)
-    k_colblock<true><<<blocks, 32 * kColWarps, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
+    GPTQ_LAUNCH(c, k_colblock<true>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales, zeros, ng,
                                                           gcol, bits, E, ldE, codes, loss_part);
   else
-    k_colblock<false><<<blocks, 32 * kColWarps, kColSmem, c->stream>>>(Wk, m, d, i, nb, R, scales, zeros, ng,
+    GPTQ_LAUNCH(c, k_colblock<false>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales, zeros, ng,
                                                            gcol, bits, E, ldE, codes, loss_part);
-  GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
 }
 
@@ -409,6 +418,8 @@ int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int k, int c0, int c
 // col_loss[j] = ½ Σ_parts Σ_rows η²  (= Σ_rows ρ² / (2 R_jj²), [T] eq.(43))
 __global__ void k_loss_reduce(const float* __restrict__ part, int parts, int d,
                               float* __restrict__ out) {
+  pdl_wait();
+  pdl_release();
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= d) return;
   double s = 0.0;
@@ -417,8 +428,7 @@ __global__ void k_loss_reduce(const float* __restrict__ part, int parts, int d,
 }
 
 int loss_reduce(Ctx* c, const float* loss_part, int parts, int d, float* loss_p) {
-  k_loss_reduce<<<(d + 255) / 256, 256, 0, c->stream>>>(loss_part, parts, d, loss_p);
-  GPTQ_LAUNCH_CHECK(c);
+  GPTQ_LAUNCH(c, k_loss_reduce, (d + 255) / 256, 256, 0, loss_part, parts, d, loss_p);
   return GPTQ_OK;
 }
 
@@ -427,6 +437,8 @@ __global__ void k_unpermute(long long m, int d, const int32_t* __restrict__ inv,
                             const uint8_t* __restrict__ codes_p, const float* __restrict__ Wk,
                             const float* __restrict__ loss_p, uint8_t* __restrict__ codes,
                             float* __restrict__ W_hat, float* __restrict__ col_loss) {
+  pdl_wait();
+  pdl_release();
   const long long total = m * d;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
@@ -443,9 +455,8 @@ int unpermute(Ctx* c, int m, int d, const int32_t* inv, const uint8_t* codes_p, 
               const float* loss_p, uint8_t* codes, float* W_hat, float* col_loss) {
   const long long total = (long long)m * d;
   int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
-  k_unpermute<<<blocks, 256, 0, c->stream>>>(m, d, inv, codes_p, Wk, loss_p, codes, W_hat,
+  GPTQ_LAUNCH(c, k_unpermute, blocks, 256, 0, m, d, inv, codes_p, Wk, loss_p, codes, W_hat,
                                              col_loss);
-  GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
 }
 

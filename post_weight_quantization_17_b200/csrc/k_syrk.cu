@@ -83,6 +83,9 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // set-up above overlaps the previous kernel; its outputs are read only from here on
+  pdl_wait();
+  pdl_release();
   const int kblocks = (n_tokens + SY_BK - 1) / SY_BK;
   const int nparts = (kblocks + SY_KB_PER_PART - 1) / SY_KB_PER_PART;
 
@@ -329,6 +332,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
   tc::cluster_sync();  // TMEM allocated in both CTAs before the leader's first MMA
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // set-up above overlaps the previous kernel; its outputs are read only from here on
+  pdl_wait();
+  pdl_release();
   const int kblocks = (n_tokens + SY_BK - 1) / SY_BK;
   const int nparts = (kblocks + SY_KB_PER_PART - 1) / SY_KB_PER_PART;
 
@@ -552,10 +558,9 @@ int syrk_tc(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool
     GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_syrk_tc2,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM));
     const uint32_t idesc = tc::idesc_f32acc(fmt, true, true, 2 * S2_BM, S2_BN);
-    k_syrk_tc2<<<grid, SY_THREADS, S2_SMEM, c->stream>>>(map, S, d, (int)n, overwrite ? 0 : 1,
+    GPTQ_LAUNCH(c, k_syrk_tc2, grid, SY_THREADS, S2_SMEM, map, S, d, (int)n, overwrite ? 0 : 1,
                                                          num_tiles, idesc, c->status,
                                                          c->timeout_cycles);
-    GPTQ_LAUNCH_CHECK(c);
     return GPTQ_OK;
   }
   const int nI = (d + SY_BM - 1) / SY_BM;
@@ -565,10 +570,9 @@ int syrk_tc(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_syrk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           SY_SMEM));
   const uint32_t idesc = tc::idesc_f32acc(fmt, true, true, SY_BM, SY_BN);
-  k_syrk_tc<<<grid, SY_THREADS, SY_SMEM, c->stream>>>(map, S, d, (int)n, overwrite ? 0 : 1,
+  GPTQ_LAUNCH(c, k_syrk_tc, grid, SY_THREADS, SY_SMEM, map, S, d, (int)n, overwrite ? 0 : 1,
                                                       num_tiles, idesc, c->status,
                                                       c->timeout_cycles);
-  GPTQ_LAUNCH_CHECK(c);
   return GPTQ_OK;
 }
 
