@@ -17,6 +17,20 @@ namespace gptq {
 // a4: static min-max grid per (row, group of original columns), [T] §1.1 and §8.3.
 // One warp per (row, group); the range is extended to contain 0; fp32 arithmetic.
 template <class T>
+__device__ __forceinline__ void gridfit_finish(float mn, float mx, bool bad, int bits, int r,
+                                               float* scale, int32_t* zero, DeviceStatus* st) {
+  if (bad) raise_error(st, GPTQ_ERR_NONFINITE, r);
+  const float maxq = (float)((1 << bits) - 1);
+  float delta = (mx == mn) ? 1.f : __fdiv_rn(__fsub_rn(mx, mn), maxq);
+  float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, delta)), 0.f), maxq);
+  *scale = delta;
+  *zero = (int32_t)z;
+}
+
+// One warp per (row, 4 consecutive groups) when groups are 128 wide in 16-bit W: each lane
+// loads its 4 elements of all 4 groups up front (8 bytes each) and the four reductions run
+// side by side.  Otherwise one warp per (row, group).
+template <class T>
 __global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, int bits,
                           float* __restrict__ scales, int32_t* __restrict__ zeros,
                           DeviceStatus* st) {
@@ -24,6 +38,52 @@ __global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, 
   pdl_release();
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
+  const bool quad = (g == 128) && (d % 512 == 0) && (sizeof(T) == 2) &&
+                    ((reinterpret_cast<uintptr_t>(W) & 7) == 0);
+  if (quad) {
+    const int nq = ng / 4;
+    if (warp >= (long long)m * nq) return;
+    const int r = (int)(warp / nq), k0 = 4 * (int)(warp % nq);
+    const T* row = W + (long long)r * d + (long long)k0 * 128 + 4 * lane;
+    uint2 raw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) raw[u] = *reinterpret_cast<const uint2*>(row + u * 128);
+    float mn[4], mx[4];
+    bool bad = false;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const T* e = reinterpret_cast<const T*>(&raw[u]);
+      mn[u] = 0.f;
+      mx[u] = 0.f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float v = to_f32<T>(e[t]);
+        bad |= !isfinite(v);
+        mn[u] = fminf(mn[u], v);
+        mx[u] = fmaxf(mx[u], v);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        mn[u] = fminf(mn[u], __shfl_xor_sync(0xffffffffu, mn[u], o));
+        mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], o));
+      }
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane < 4) {
+      float a = mn[0], b = mx[0];
+#pragma unroll
+      for (int u = 1; u < 4; ++u)
+        if (lane == u) {
+          a = mn[u];
+          b = mx[u];
+        }
+      const long long o = (long long)r * ng + k0 + lane;
+      gridfit_finish<T>(a, b, bad && lane == 0, bits, r, scales + o, zeros + o, st);
+    }
+    return;
+  }
   if (warp >= (long long)m * ng) return;
   const int r = (int)(warp / ng), k = (int)(warp % ng);
   const int c0 = k * g, c1 = min(d, c0 + g);
@@ -41,28 +101,28 @@ __global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, 
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
   bad = __any_sync(0xffffffffu, bad);
-  if (lane == 0) {
-    if (bad) raise_error(st, GPTQ_ERR_NONFINITE, r);
-    const float maxq = (float)((1 << bits) - 1);
-    float delta = (mx == mn) ? 1.f : __fdiv_rn(__fsub_rn(mx, mn), maxq);
-    float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, delta)), 0.f), maxq);
-    scales[(long long)r * ng + k] = delta;
-    zeros[(long long)r * ng + k] = (int32_t)z;
-  }
+  if (lane == 0)
+    gridfit_finish<T>(mn, mx, bad, bits, r, scales + (long long)r * ng + k,
+                      zeros + (long long)r * ng + k, st);
 }
 
 int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int group,
              float* scales, int32_t* zeros) {
   const int g = (group == -1) ? d : group;
   const int ng = (d + g - 1) / g;
-  const long long warps = (long long)m * ng;
+  const bool quad = (g == 128) && (d % 512 == 0) && (w_dtype != GPTQ_F32) &&
+                    ((reinterpret_cast<uintptr_t>(W) & 7) == 0);
+  const long long warps = (long long)m * (quad ? ng / 4 : ng);
   const int blocks = (int)((warps * 32 + 255) / 256);
   if (w_dtype == GPTQ_F16)
-    GPTQ_LAUNCH(c, k_gridfit<__half>, blocks, 256, 0, (const __half*)W, m, d, g, ng, bits, scales, zeros, c->status);
+    GPTQ_LAUNCH(c, k_gridfit<__half>, blocks, 256, 0, (const __half*)W, m, d, g, ng, bits, scales,
+                zeros, c->status);
   else if (w_dtype == GPTQ_BF16)
-    GPTQ_LAUNCH(c, k_gridfit<__nv_bfloat16>, blocks, 256, 0, (const __nv_bfloat16*)W, m, d, g, ng, bits, scales, zeros, c->status);
+    GPTQ_LAUNCH(c, k_gridfit<__nv_bfloat16>, blocks, 256, 0, (const __nv_bfloat16*)W, m, d, g, ng,
+                bits, scales, zeros, c->status);
   else
-    GPTQ_LAUNCH(c, k_gridfit<float>, blocks, 256, 0, (const float*)W, m, d, g, ng, bits, scales, zeros, c->status);
+    GPTQ_LAUNCH(c, k_gridfit<float>, blocks, 256, 0, (const float*)W, m, d, g, ng, bits, scales,
+                zeros, c->status);
   return GPTQ_OK;
 }
 
@@ -84,35 +144,55 @@ int make_gcol(Ctx* c, const int32_t* perm, int d, int group, int32_t* gcol, int3
   return GPTQ_OK;
 }
 
-// working copy in processing order: Wk[r][j] = dead[π_j] ? 0 : W[r][π_j]  ([T] §10)
+// working copy in processing order: Wk[r][j] = dead[π_j] ? 0 : W[r][π_j]  ([T] §10).
+// Grid: x over groups of 4 columns, y strided over rows (no index division).
 template <class T>
 __global__ void k_init_work(const T* __restrict__ W, long long m, int d,
                             const int32_t* __restrict__ perm, const uint8_t* __restrict__ dead,
                             float* __restrict__ Wk) {
   pdl_wait();
   pdl_release();
-  const long long total = m * d;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    long long r = e / d;
-    int j = (int)(e - r * d);
-    int src = perm ? perm[j] : j;
-    float v = to_f32<T>(W[r * d + src]);
-    if (dead && dead[src]) v = 0.f;
-    Wk[e] = v;
+  const int j0 = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (j0 >= d) return;
+  const bool vec = !perm && (j0 + 4 <= d) && (d % 4 == 0) && (sizeof(T) == 2) &&
+                   ((reinterpret_cast<uintptr_t>(W) & 7) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(Wk) & 15) == 0);
+  int src[4];
+  bool keep[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int j = min(j0 + t, d - 1);
+    src[t] = perm ? perm[j] : j;
+    keep[t] = !(dead && dead[src[t]]);
+  }
+  for (long long r = blockIdx.y; r < m; r += gridDim.y) {
+    const T* wr = W + r * d;
+    float* out = Wk + r * d + j0;
+    if (vec) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(wr + j0);
+      const T* e = reinterpret_cast<const T*>(&raw);
+      *reinterpret_cast<float4*>(out) =
+          make_float4(keep[0] ? to_f32<T>(e[0]) : 0.f, keep[1] ? to_f32<T>(e[1]) : 0.f,
+                      keep[2] ? to_f32<T>(e[2]) : 0.f, keep[3] ? to_f32<T>(e[3]) : 0.f);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (j0 + t < d) out[t] = keep[t] ? to_f32<T>(wr[src[t]]) : 0.f;
+    }
   }
 }
 
 int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* perm,
               const uint8_t* dead, bool, float* Wk) {
-  const long long total = (long long)m * d;
-  int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
+  const int gx = (d + 4 * 256 - 1) / (4 * 256);
+  const int gy = std::max(1, std::min(m, (c->num_sms * 16 + gx - 1) / gx));
+  const dim3 grid(gx, gy);
   if (w_dtype == GPTQ_F16)
-    GPTQ_LAUNCH(c, k_init_work<__half>, blocks, 256, 0, (const __half*)W, m, d, perm, dead, Wk);
+    GPTQ_LAUNCH(c, k_init_work<__half>, grid, 256, 0, (const __half*)W, (long long)m, d, perm, dead, Wk);
   else if (w_dtype == GPTQ_BF16)
-    GPTQ_LAUNCH(c, k_init_work<__nv_bfloat16>, blocks, 256, 0, (const __nv_bfloat16*)W, m, d, perm, dead, Wk);
+    GPTQ_LAUNCH(c, k_init_work<__nv_bfloat16>, grid, 256, 0, (const __nv_bfloat16*)W, (long long)m, d, perm, dead, Wk);
   else
-    GPTQ_LAUNCH(c, k_init_work<float>, blocks, 256, 0, (const float*)W, m, d, perm, dead, Wk);
+    GPTQ_LAUNCH(c, k_init_work<float>, grid, 256, 0, (const float*)W, (long long)m, d, perm, dead, Wk);
   return GPTQ_OK;
 }
 
@@ -432,31 +512,30 @@ int loss_reduce(Ctx* c, const float* loss_part, int parts, int d, float* loss_p)
   return GPTQ_OK;
 }
 
-// a7: back to original column order ([T] §10: undo the column permutation).
+// a7: back to original column order ([T] §10: undo the column permutation).  Grid: x over
+// columns, y strided over rows.
 __global__ void k_unpermute(long long m, int d, const int32_t* __restrict__ inv,
                             const uint8_t* __restrict__ codes_p, const float* __restrict__ Wk,
                             const float* __restrict__ loss_p, uint8_t* __restrict__ codes,
                             float* __restrict__ W_hat, float* __restrict__ col_loss) {
   pdl_wait();
   pdl_release();
-  const long long total = m * d;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    long long r = e / d;
-    int k = (int)(e - r * d);
-    long long src = r * d + inv[k];
-    codes[e] = codes_p[src];
-    W_hat[e] = Wk[src];
-    if (r == 0) col_loss[k] = loss_p[inv[k]];
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= d) return;
+  const int src = inv[k];
+  if (blockIdx.y == 0) col_loss[k] = loss_p[src];
+  for (long long r = blockIdx.y; r < m; r += gridDim.y) {
+    codes[r * d + k] = codes_p[r * d + src];
+    W_hat[r * d + k] = Wk[r * d + src];
   }
 }
 
 int unpermute(Ctx* c, int m, int d, const int32_t* inv, const uint8_t* codes_p, const float* Wk,
               const float* loss_p, uint8_t* codes, float* W_hat, float* col_loss) {
-  const long long total = (long long)m * d;
-  int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
-  GPTQ_LAUNCH(c, k_unpermute, blocks, 256, 0, m, d, inv, codes_p, Wk, loss_p, codes, W_hat,
-                                             col_loss);
+  const int gx = (d + 255) / 256;
+  const int gy = std::max(1, std::min(m, (c->num_sms * 16 + gx - 1) / gx));
+  GPTQ_LAUNCH(c, k_unpermute, dim3(gx, gy), 256, 0, (long long)m, d, inv, codes_p, Wk, loss_p,
+              codes, W_hat, col_loss);
   return GPTQ_OK;
 }
 

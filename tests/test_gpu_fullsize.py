@@ -13,7 +13,7 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 import post_weight_quantization_17_b200 as G  # noqa: E402
 from oracle import gptq_oracle as O  # noqa: E402
 from tests import _parity as P  # noqa: E402
-from workloads.synth import CONFIGS, XSource, make_weight  # noqa: E402
+from workloads.synth import BLOCK7B_SHARED_INPUT, CONFIGS, XSource, make_weight  # noqa: E402
 
 
 def _oracle_hessian(chunks, d):
@@ -58,7 +58,15 @@ def _run_full(spec, seed, n_rows=48):
     res["R"] = P.rel_fro(Rg, prep["R"])
     res["Hinv"] = P.rel_fro(Rg.T @ Rg, prep["G"])
     assert res["R"] <= P.TOL_HINV and res["Hinv"] <= P.TOL_HINV, res
-    # sampled rows
+    res.update(_check_rows(spec, W, b, prep, seed, n_rows))
+    ctx.close()
+    return res
+
+
+def _check_rows(spec, W, b, prep, seed, n_rows):
+    """Grid (bit-exact), codes (decision replay against the oracle's own R), Ŵ and packed words
+    of `n_rows` sampled rows."""
+    res = {}
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(spec.m, size=n_rows, replace=False))
     Wn = W.float().cpu().double().numpy()[rows]
@@ -81,7 +89,6 @@ def _run_full(spec, seed, n_rows=48):
     assert res["W_hat"] <= P.TOL_WHAT, res
     packed = b.packed.cpu().numpy().view(np.uint32)[rows]
     assert np.array_equal(packed, O.pack(codes, spec.bits))
-    ctx.close()
     return res
 
 
@@ -93,3 +100,140 @@ def test_q_proj_4096_full_size():
 def test_down_proj_11008_actorder_3bit_full_size():
     res = _run_full(CONFIGS[3][0], seed=2, n_rows=24)
     print("down_proj full size:", {k: f"{v:.3e}" if isinstance(v, float) else v for k, v in res.items()})
+
+
+def test_block7b_full_size():
+    """Config 4: one 7B decoder block, seven matrices over four calibration inputs (q/k/v share
+    one H and one R, gate/up share one), N = 65536 tokens per input, at full size."""
+    dev = torch.device("cuda")
+    specs = {s.name.split("_")[0]: s for s in CONFIGS[4]}
+    for gi, (gname, members) in enumerate(BLOCK7B_SHARED_INPUT.items()):
+        first = specs[members[0]]
+        d, seed = first.d, 30 + gi
+        X = XSource(first, seed, dev).full()
+        ctx = G.Context(m_max=max(specs[n].m for n in members), d_max=d, act_order=False)
+        S = torch.empty(d, d, device=dev)
+        R = torch.empty(d, d, device=dev)
+        perm = torch.empty(d, dtype=torch.int32, device=dev)
+        dead = torch.empty(d, dtype=torch.uint8, device=dev)
+        n = G.gptq_hessian_accumulate(ctx, X, S, 0)
+        S_gpu = torch.tril(S).cpu().double().numpy() * (2.0 / n)
+        G.gptq_prepare_hinv(ctx, S, n, first.percdamp, False, R, perm, dead)
+        G.gptq_sync_status(ctx)
+        H = _oracle_hessian([X], d)
+        del X
+        res = {"H": P.rel_fro(S_gpu, np.tril(H))}
+        del S_gpu
+        prep = O.prepare_with_retry(H, first.percdamp, False)
+        Rg = R.cpu().double().numpy()
+        res["R"] = P.rel_fro(Rg, prep["R"])
+        res["Hinv"] = P.rel_fro(Rg.T @ Rg, prep["G"])
+        del Rg
+        assert res["H"] <= P.TOL_H and res["R"] <= P.TOL_HINV and res["Hinv"] <= P.TOL_HINV, (gname, res)
+        print(f"{gname} d={d}:", {k: f"{v:.3e}" for k, v in res.items()})
+        for k, name in enumerate(members):
+            spec = specs[name]
+            W = make_weight(spec, seed * 10 + k, dev)
+            b = G.LayerBuffers(spec.m, d, spec.bits, spec.group, dev)
+            G.gptq_quantize_layer(ctx, W, R, None, dead, spec.bits, spec.group, spec.block, False,
+                                  b.scales, b.zeros, b.codes, b.W_hat, b.col_loss)
+            G.gptq_pack(ctx, b.codes, spec.bits, b.packed)
+            G.gptq_sync_status(ctx)
+            r = _check_rows(spec, W, b, prep, seed * 10 + k, 12)
+            print(f"  {name} {spec.m}x{d}:", {k2: f"{v:.3e}" if isinstance(v, float) else v
+                                             for k2, v in r.items()})
+            del b, W
+        ctx.close()
+        del S, R
+        torch.cuda.empty_cache()
+
+
+def test_fc2_175b_full_size():
+    """Config 5 at full size: W 12288 x 49152, X 49152 x 65536 streamed in eight 8192-token
+    chunks, H 49152^2 fp32 on the device, 4- and 2-bit.  The fp64 oracle cannot form or invert
+    H at this size in seconds, so the checks are: H on sampled entries against fp64 sums over the
+    same bf16 bytes; the factor through the identity R H_λ R^T = I on sampled entries (it holds
+    at any size); grid and packed words bit-exact against the oracle on sampled rows; Ŵ exactly
+    Δ(c - z).  Decision parity of the column loop is covered at the same recipe's reduced
+    shapes in test_gpu_parity.py."""
+    dev = torch.device("cuda")
+    spec4, spec2 = CONFIGS[5]
+    d, m = spec4.d, spec4.m
+    rng = np.random.default_rng(5)
+    cols = np.sort(rng.choice(d, size=12, replace=False))
+    cols_t = torch.as_tensor(cols, device=dev)
+    ctx = G.Context(m_max=m, d_max=d, act_order=False)
+    S = torch.empty(d, d, device=dev)
+    n = 0
+    xs = []
+    for chunk in XSource(spec4, 4, dev).chunks():
+        n = G.gptq_hessian_accumulate(ctx, chunk, S, n)
+        xs.append(chunk.index_select(1, cols_t).float().cpu().double().numpy())
+        del chunk
+    G.gptq_sync_status(ctx)
+    assert n == spec4.n_tokens
+    Xc = np.concatenate(xs)
+    H_o = (2.0 / n) * (Xc.T @ Xc)                       # fp64 over the same bytes
+    Sl = S.index_select(0, cols_t).index_select(1, cols_t).cpu().double().numpy()
+    lo = np.tril(np.ones((len(cols), len(cols)), bool))
+    H_g = np.where(lo, Sl, Sl.T) * (2.0 / n)            # S holds the lower triangle
+    res = {"H_sampled": P.rel_fro(H_g, H_o)}
+    assert res["H_sampled"] <= P.TOL_H, res
+    # symmetric copy of H for the factorization identity (prepare overwrites S)
+    Hs = torch.tril(S)
+    Hs += torch.tril(Hs, -1).T
+    Hs *= 2.0 / n
+    R = torch.empty(d, d, device=dev)
+    perm = torch.empty(d, dtype=torch.int32, device=dev)
+    dead = torch.empty(d, dtype=torch.uint8, device=dev)
+    lam, retries = G.gptq_prepare_hinv(ctx, S, n, spec4.percdamp, False, R, perm, dead)
+    del S
+    torch.cuda.empty_cache()
+    assert int(dead.sum()) == 0 and retries == 0
+    # R H_λ R^T = I (R = U^{-1}, H_λ = U U^T): fp64 products in row blocks
+    pick = torch.as_tensor(np.sort(rng.choice(d, size=6, replace=False)), device=dev)
+    Ra = R.index_select(0, pick).double()               # [6, d]
+    Y = torch.zeros(len(pick), d, dtype=torch.float64, device=dev)
+    for r0 in range(0, d, 4096):
+        Hb = Hs[r0:r0 + 4096].double()
+        Hb[:, r0:r0 + 4096].diagonal().add_(lam)
+        Y += Ra[:, r0:r0 + 4096] @ Hb
+        del Hb
+    M = (Y @ Ra.T).cpu().numpy()
+    res["RHRt_minus_I"] = float(np.abs(M - np.eye(len(pick))).max())
+    assert res["RHRt_minus_I"] <= 1e-3, res
+    del Hs, Y, Ra
+    torch.cuda.empty_cache()
+    rows = np.sort(rng.choice(m, size=16, replace=False))
+    for spec in (spec4, spec2):
+        W = make_weight(spec, 4, dev)
+        ng = -(-d // spec.group)
+        scales = torch.empty(m, ng, device=dev)
+        zeros = torch.empty(m, ng, dtype=torch.int32, device=dev)
+        codes = torch.empty(m, d, dtype=torch.uint8, device=dev)
+        W_hat = torch.empty(m, d, device=dev)
+        col_loss = torch.empty(d, device=dev)
+        packed = torch.empty(m, G.words_per_row(d, spec.bits), dtype=torch.int32, device=dev)
+        G.gptq_quantize_layer(ctx, W, R, None, dead, spec.bits, spec.group, spec.block, False,
+                              scales, zeros, codes, W_hat, col_loss)
+        G.gptq_pack(ctx, codes, spec.bits, packed)
+        G.gptq_sync_status(ctx)
+        rt = torch.as_tensor(rows, device=dev)
+        Wn = W.index_select(0, rt).float().cpu().double().numpy()
+        sc, ze = O.fit_grid(Wn, spec.bits, spec.group)
+        assert np.array_equal(scales.index_select(0, rt).cpu().numpy(), sc)
+        assert np.array_equal(zeros.index_select(0, rt).cpu().numpy(), ze)
+        c_s = codes.index_select(0, rt).cpu().numpy()
+        assert int(c_s.max()) <= (1 << spec.bits) - 1
+        gidx = np.arange(d) // spec.group
+        q = (sc[:, gidx] * (c_s.astype(np.int64) - ze[:, gidx]).astype(np.float32)).astype(np.float32)
+        assert np.array_equal(q, W_hat.index_select(0, rt).cpu().numpy()), "W_hat is not Δ(c - z)"
+        assert np.array_equal(packed.index_select(0, rt).cpu().numpy().view(np.uint32),
+                              O.pack(c_s, spec.bits))
+        cl = col_loss.cpu().numpy()
+        assert np.all(np.isfinite(cl)) and np.all(cl >= 0)
+        res[f"{spec.bits}bit_rows_checked"] = len(rows)
+        del W, scales, zeros, codes, W_hat, packed
+        torch.cuda.empty_cache()
+    ctx.close()
+    print("fc2 full size:", {k: f"{v:.3e}" if isinstance(v, float) else v for k, v in res.items()})
