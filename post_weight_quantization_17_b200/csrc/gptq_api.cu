@@ -22,6 +22,13 @@ size_t prep_bytes(int64_t d) {
   return b;
 }
 
+// tf32 halves of E and of one super-block's slice of R for the pair tail GEMM (optional: a
+// workspace without room for them runs the tail update on the single-CTA GEMM)
+size_t pair_bytes(int64_t m, int64_t d) {
+  return 256 * 4 + 2 * (size_t)m * gptq::kSuperCols * sizeof(float) +
+         2 * (size_t)gptq::kSuperCols * (size_t)((d + 3) / 4 * 4) * sizeof(float);
+}
+
 size_t quant_bytes(int64_t m, int64_t d, bool general_perm) {
   size_t b = gptq::kStatusBytes + 256 * 10;
   b += 2 * d * sizeof(int32_t);                                  // gcol, inv
@@ -29,6 +36,7 @@ size_t quant_bytes(int64_t m, int64_t d, bool general_perm) {
   b += (size_t)((m + gptq::kColRows - 1) / gptq::kColRows) * d * sizeof(float);  // loss parts
   b += d * sizeof(float);                                        // loss in processing order
   if (general_perm) b += (size_t)m * d * (sizeof(float) + 1);    // W_work, codes (permuted)
+  b += pair_bytes(m, d);                                         // optional: pair tail GEMM
   return b;
 }
 
@@ -208,6 +216,13 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   }
   if (!cv.ok())
     GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "quantize_layer: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
+  const int ldr = (di + 3) / 4 * 4;
+  float* Ehi = cv.take<float>((size_t)m * gptq::kSuperCols);
+  float* Elo = cv.take<float>((size_t)m * gptq::kSuperCols);
+  float* Rhi = cv.take<float>((size_t)gptq::kSuperCols * ldr);
+  float* Rlo = cv.take<float>((size_t)gptq::kSuperCols * ldr);
+  const bool pair_ws = cv.ok();
+  if (!pair_ws) Ehi = Elo = Rhi = Rlo = nullptr;
   int rc;
   if (!grid_given && (rc = gptq::grid_fit(c, W, w_dtype, mi, di, bits, group, scales, zeros)))
     return rc;
@@ -226,13 +241,25 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
       const bool uniform = (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
       float* Et = E + (i - s0);
       if ((rc = gptq::column_block(c, Wk, mi, di, i, nb, R, scales, zeros, ng, gcol, uniform,
-                                   bits, Et, gptq::kSuperCols, codes_p, loss_part)))
+                                   bits, Et, Ehi ? Ehi + (i - s0) : nullptr,
+                                   Elo ? Elo + (i - s0) : nullptr, gptq::kSuperCols, codes_p,
+                                   loss_part)))
         return rc;
       if ((rc = gptq::trailing_update(c, Wk, mi, di, i, nb, i + nb, s1, Et, gptq::kSuperCols, R)))
         return rc;
     }
-    if ((rc = gptq::trailing_update(c, Wk, mi, di, s0, s1 - s0, s1, di, E, gptq::kSuperCols, R)))
+    // tail: W[:, s1:] -= E R[s0:s1, s1:], on CTA pairs with split operands where it applies
+    const int tn = di - s1, tk = s1 - s0;
+    if (tn > 0 && pair_ws && gptq::gemm_pair_applies(mi, tn, tk, Ehi, gptq::kSuperCols, Rhi, ldr,
+                                                     c->num_sms)) {
+      if ((rc = gptq::split_tf32(c, R + (long long)s0 * di + s1, di, tk, tn, Rhi, Rlo, ldr)))
+        return rc;
+      if ((rc = gptq::gemm_pair(c, mi, tn, tk, Ehi, Elo, gptq::kSuperCols, Rhi, Rlo, ldr, Wk + s1,
+                                di, -1.f, 1.f)))
+        return rc;
+    } else if ((rc = gptq::trailing_update(c, Wk, mi, di, s0, tk, s1, di, E, gptq::kSuperCols, R))) {
       return rc;
+    }
   }
   if ((rc = gptq::loss_reduce(c, loss_part, parts, di, general ? loss_p : col_loss))) return rc;
   if (general &&

@@ -61,14 +61,6 @@ __device__ __forceinline__ bool gt_tile(const GemmTcParams& p, int t, int& i0, i
   return true;
 }
 
-// Round an fp32 value to tf32 (10 explicit mantissa bits), to nearest with ties away from zero:
-// the format is sign-magnitude, so adding half a tf32 unit (bit 12) to the bit pattern and
-// clearing the 13 low bits rounds the magnitude; a mantissa carry moves into the exponent as it
-// should.  Integer ALU only (the conversion instruction runs on a narrower pipe).
-__device__ __forceinline__ float tf32_rna(float x) {
-  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
-}
-
 __global__ void __launch_bounds__(GT_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               GemmTcParams p, DeviceStatus* st, long long budget) {
@@ -238,14 +230,14 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
           for (int c = ct; c < GT_TILE_BYTES / 16; c += 32 * GT_CONV_WARPS) {
             const float4 x = hi[c];
             float4 h, l;
-            h.x = tf32_rna(x.x);
-            h.y = tf32_rna(x.y);
-            h.z = tf32_rna(x.z);
-            h.w = tf32_rna(x.w);
-            l.x = tf32_rna(x.x - h.x);
-            l.y = tf32_rna(x.y - h.y);
-            l.z = tf32_rna(x.z - h.z);
-            l.w = tf32_rna(x.w - h.w);
+            h.x = tc::tf32_rna(x.x);
+            h.y = tc::tf32_rna(x.y);
+            h.z = tc::tf32_rna(x.z);
+            h.w = tc::tf32_rna(x.w);
+            l.x = tc::tf32_rna(x.x - h.x);
+            l.y = tc::tf32_rna(x.y - h.y);
+            l.z = tc::tf32_rna(x.z - h.z);
+            l.w = tc::tf32_rna(x.w - h.w);
             hi[c] = h;
             lo[c] = l;
           }

@@ -8,6 +8,7 @@
 // W[:, i+nb:] -= E R[i:i+nb, i+nb:] (eq.(46)).
 #include "kernels.h"
 #include "gemm_simt.cuh"
+#include "tc_util.cuh"
 
 #include <utility>
 
@@ -308,7 +309,8 @@ template <bool UNIFORM, bool FAST>
 __device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128],
                                          const ColStepArgs& args, int r, int row, int nb, int d,
                                          int i, int ldE, bool vec, float* __restrict__ Wk,
-                                         float* __restrict__ E, uint8_t* __restrict__ codes) {
+                                         float* __restrict__ E, float* __restrict__ Ehi,
+                                         float* __restrict__ Elo, uint8_t* __restrict__ codes) {
   const float(*Rs)[128] = args.Rs;
   const int q = args.q, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll 1
@@ -338,9 +340,22 @@ __device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128
     *reinterpret_cast<float4*>(&St[r][off + 4 * q]) = make_float4(e4[0], e4[1], e4[2], e4[3]);
     const int c = off + 4 * q;
     if (args.active) {
+      // η's tf32 halves for the pair GEMM of the tail update, when it is used
+      float eh[4], el[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        eh[t] = tc::tf32_rna(e4[t]);
+        el[t] = tc::tf32_rna(e4[t] - eh[t]);
+      }
       if (vec && c + 4 <= nb) {
         *reinterpret_cast<float4*>(E + (long long)row * ldE + c) =
             make_float4(e4[0], e4[1], e4[2], e4[3]);
+        if (Ehi) {
+          *reinterpret_cast<float4*>(Ehi + (long long)row * ldE + c) =
+              make_float4(eh[0], eh[1], eh[2], eh[3]);
+          *reinterpret_cast<float4*>(Elo + (long long)row * ldE + c) =
+              make_float4(el[0], el[1], el[2], el[3]);
+        }
         *reinterpret_cast<float4*>(Wk + (long long)row * d + i + c) =
             make_float4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uchar4*>(codes + (long long)row * d + i + c) =
@@ -350,6 +365,10 @@ __device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128
         for (int t = 0; t < 4; ++t)
           if (c + t < nb) {
             E[(long long)row * ldE + c + t] = e4[t];
+            if (Ehi) {
+              Ehi[(long long)row * ldE + c + t] = eh[t];
+              Elo[(long long)row * ldE + c + t] = el[t];
+            }
             Wk[(long long)row * d + i + c + t] = w[t];
             codes[(long long)row * d + i + c + t] = (uint8_t)c4[t];
           }
@@ -370,8 +389,9 @@ template <bool UNIFORM>
 __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     float* __restrict__ Wk, int m, int d, int i, int nb, const float* __restrict__ R,
     const float* __restrict__ scales, const int32_t* __restrict__ zeros, int ng,
-    const int32_t* __restrict__ gcol, int bits, float* __restrict__ E, int ldE,
-    uint8_t* __restrict__ codes, float* __restrict__ loss_part) {
+    const int32_t* __restrict__ gcol, int bits, float* __restrict__ E, float* __restrict__ Ehi,
+    float* __restrict__ Elo, int ldE, uint8_t* __restrict__ codes,
+    float* __restrict__ loss_part) {
   extern __shared__ __align__(16) unsigned char smem[];
   float(*Rs)[128] = reinterpret_cast<float(*)[128]>(smem);
   // St: the W block on entry, then sub-block by sub-block η (scaled residual) replaces w
@@ -394,6 +414,8 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
                    ((reinterpret_cast<uintptr_t>(R) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(Wk) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(E) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(Ehi) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(Elo) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(codes) & 3) == 0);
   // R was written before the previous kernel (the factorization, or an earlier block's
   // kernels), so its copies start before the wait; the W block is the previous kernel's output
@@ -453,9 +475,9 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
   }
   fast = __syncthreads_and(fast);  // also publishes rinv and gs
   if (fast)
-    col_walk<UNIFORM, true>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, codes);
+    col_walk<UNIFORM, true>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, Ehi, Elo, codes);
   else
-    col_walk<UNIFORM, false>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, codes);
+    col_walk<UNIFORM, false>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, Ehi, Elo, codes);
   __syncthreads();
   // loss partial Σ_rows η² per column, the 8 warps' sums in a fixed order
   for (int t = tid; t < nb; t += blockDim.x) {
@@ -468,22 +490,23 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
 
 int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                  const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
-                 bool uniform_grid, int bits, float* E, int ldE, uint8_t* codes,
-                 float* loss_part) {
+                 bool uniform_grid, int bits, float* E, float* Ehi, float* Elo, int ldE,
+                 uint8_t* codes, float* loss_part) {
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<false>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   const int blocks = (m + kColCtaRows - 1) / kColCtaRows;
   if (uniform_grid)
-    GPTQ_LAUNCH(c, k_colblock<true>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales, zeros, ng,
-                                                          gcol, bits, E, ldE, codes, loss_part);
+    GPTQ_LAUNCH(c, k_colblock<true>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales,
+                zeros, ng, gcol, bits, E, Ehi, Elo, ldE, codes, loss_part);
   else
-    GPTQ_LAUNCH(c, k_colblock<false>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales, zeros, ng,
-                                                           gcol, bits, E, ldE, codes, loss_part);
+    GPTQ_LAUNCH(c, k_colblock<false>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales,
+                zeros, ng, gcol, bits, E, Ehi, Elo, ldE, codes, loss_part);
   return GPTQ_OK;
 }
 
+// ------------------------------------------------------------------------------------------
 // a6: lazy update W[:, c0:c1] -= E[:, 0:k] R[i:i+k, c0:c1]  ([T] eq.(46)); fp32-accurate GEMM.
 int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int k, int c0, int c1,
                     const float* E, int ldE, const float* R) {

@@ -27,10 +27,20 @@ int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int gro
 int make_gcol(Ctx* c, const int32_t* perm, int d, int group, int32_t* gcol, int32_t* inv);
 int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* perm,
               const uint8_t* dead, bool identity, float* Wk);
+// E (and, if not null, its tf32 halves Ehi / Elo) receive the block's scaled residuals.
 int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                  const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
-                 bool uniform_grid, int bits, float* E, int ldE, uint8_t* codes,
-                 float* loss_part);
+                 bool uniform_grid, int bits, float* E, float* Ehi, float* Elo, int ldE,
+                 uint8_t* codes, float* loss_part);
+// Tail update on CTA pairs with operands split into tf32 halves (k_gemm_pair.cu):
+// C = alpha A B + beta C, A [M, K] (lda), B [K, N] (ldb), both row-major.
+bool gemm_pair_applies(int M, int N, int K, const float* Ah, long long lda, const float* Bh,
+                       long long ldb, int num_sms);
+int gemm_pair(Ctx* c, int M, int N, int K, const float* Ah, const float* Al, long long lda,
+              const float* Bh, const float* Bl, long long ldb, float* C, long long ldc, float alpha,
+              float beta);
+int split_tf32(Ctx* c, const float* src, long long lds, int rows, int cols, float* hi, float* lo,
+               long long ldd);
 int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int k, int c0, int c1,
                     const float* E, int ldE, const float* R);
 int loss_reduce(Ctx* c, const float* loss_part, int parts, int d, float* loss_p);

@@ -216,6 +216,21 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, ui
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+__device__ __forceinline__ void mma_tf32_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Round an fp32 value to tf32 (10 explicit mantissa bits), to nearest with ties away from zero:
+// the format is sign-magnitude, so adding half a tf32 unit (bit 12) to the bit pattern and
+// clearing the 13 low bits rounds the magnitude; a mantissa carry moves into the exponent as it
+// should.  Integer ALU only.
+__device__ __forceinline__ float tf32_rna(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
 // Arrives on `bar` in both CTAs of the pair once every pair MMA issued so far has completed.
 __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
   asm volatile(

@@ -25,6 +25,9 @@ SMALL = [
     ("block7b_down_shape", CONFIGS[4][6].scaled(72, 256, 1500), 3),
     ("fc2_shape_2bit", CONFIGS[5][1].scaled(130, 256, 2048, chunk=512), 4),
     ("fc2_shape_4bit", CONFIGS[5][0].scaled(40, 200, 900, chunk=300), 9),
+    # m >= 256 and tails past the first super-block: the split-operand pair GEMM (ragged rows,
+    # a 588-column tail) and, for the last 76 columns, the single-CTA GEMM
+    ("pair_tail_ragged", CONFIGS[2][0].scaled(300, 1100, 2500, chunk=1000), 10),
     ("ragged_all", LayerSpec("ragged", 77, 333, 1001, bits=4, group=128, block=128,
                              act_order=False, x_kind="lowrank_t3", x_rank=40, chunk=333), 5),
     ("ragged_actorder_rowgrid", LayerSpec("ragged2", 33, 197, 517, bits=3, group=-1, block=64,
