@@ -21,8 +21,7 @@ Precision: fp64 everywhere, except where floating point decides an integer.  The
 round-half-to-even), which is the precision the CUDA kernels take them in, and Δ is rounded to
 fp32 because it is a stored fp32 artifact.
 
-Readings where the pages leave a step open are listed in the design doc; the ones that show up in
-code are commented where they are used.  Every function here is pinned by a ``-m "not gpu"``
+Readings where the pages leave a step open are commented where they show up in the code.  Every function here is pinned by a ``-m "not gpu"``
 test (worked examples, closed forms, invariants, library special cases, brute force).
 """
 from __future__ import annotations
@@ -235,7 +234,26 @@ def _group_of_column(orig_cols, d: int, group: int):
     return np.asarray(orig_cols) // int(group)
 
 
-def gptq_explicit(Wp, G, scale, zero, gcol, bits: int):
+def _dynamic_refit(W, j: int, dyn: int, bits: int, scale, zero):
+    """Dynamic groups ([T] §8.3 and §8.4 remark): at a group start j (j % g == 0) the grid of
+    processing group j // g is fitted per row, by the same min-max rule as `fit_grid`, on the
+    CURRENT working weights of that group's columns W[:, j : j+g] (every earlier column's
+    compensation already applied).  Reading: the pages leave the moment open beyond "at the
+    start of each group"; the fit sees the group's columns exactly as column j is about to be
+    quantized."""
+    if dyn > 0 and j % dyn == 0:
+        sc, ze = fit_grid(W[:, j:j + dyn], bits, -1)
+        scale[:, j // dyn] = sc[:, 0]
+        zero[:, j // dyn] = ze[:, 0]
+
+
+def dynamic_grid_arrays(m: int, d: int, dyn: int):
+    """Empty per-(row, processing group) grid arrays for dynamic groups of size dyn."""
+    ng = -(-d // dyn)
+    return np.zeros((m, ng), np.float32), np.zeros((m, ng), np.int32)
+
+
+def gptq_explicit(Wp, G, scale, zero, gcol, bits: int, dynamic: int = 0):
     """Unblocked GPTQ with explicit inverse updates, column by column in processing order.
 
     For j = 0..d-1 over all rows at once (F = {j..d-1}): quantize column j ([T] eq.(36));
@@ -244,7 +262,9 @@ def gptq_explicit(Wp, G, scale, zero, gcol, bits: int):
     ([T] eq.(41)); downdate G by eq.(27).
 
     Wp: working weights [m, d] in processing order (dead columns already zero).
-    gcol: grid index used at processing position j.  Returns (codes, Q, col_loss, R_rows).
+    gcol: grid index used at processing position j.  dynamic = g > 0: the grid is refitted at
+    every group start by `_dynamic_refit` and written into scale / zero (gcol must be j // g).
+    Returns (codes, Q, col_loss, R_rows).
     """
     W = np.array(Wp, dtype=np.float64, copy=True)
     G = np.array(G, dtype=np.float64, copy=True)
@@ -254,6 +274,7 @@ def gptq_explicit(Wp, G, scale, zero, gcol, bits: int):
     loss = np.zeros(d, np.float64)
     Rrows = np.zeros((d, d), np.float64)
     for j in range(d):
+        _dynamic_refit(W, j, dynamic, bits, scale, zero)
         c, q, _ = quantize(W[:, j], scale[:, gcol[j]], zero[:, gcol[j]], bits)
         rho = W[:, j] - q
         gjj = G[j, j]
@@ -267,13 +288,18 @@ def gptq_explicit(Wp, G, scale, zero, gcol, bits: int):
     return codes, Q, loss, Rrows
 
 
-def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int):
+def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int, dynamic: int = 0):
     """GPTQ in Cholesky form with lazy block updates: [W] Algorithm 1 / [T] §10 pseudo-code.
 
     For each block [i, i2): for j in the block quantize column j, η = ρ / R_jj, record
     ρ² / (2 R_jj²) ([T] eq.(43)), update the block's remaining columns by eq.(42) and keep η
     in E; after the block apply W[:, i2:] -= E R[i:i2, i2:] ([T] eq.(46)).
+    dynamic = g > 0 refits at group starts as in `gptq_explicit`; the group's columns are then
+    current only if every group starts on a block start or lies inside one block
+    (g % block == 0 or block % g == 0), which is required.
     Returns (codes, Q, col_loss)."""
+    if dynamic > 0 and dynamic % block != 0 and block % dynamic != 0:
+        raise ValueError("dynamic groups must start on block starts or lie inside a block")
     W = np.array(Wp, dtype=np.float64, copy=True)
     R = np.asarray(R, np.float64)
     m, d = W.shape
@@ -284,6 +310,7 @@ def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int):
         i2 = min(i + block, d)
         E = np.zeros((m, i2 - i), np.float64)
         for j in range(i, i2):
+            _dynamic_refit(W, j, dynamic, bits, scale, zero)
             c, q, _ = quantize(W[:, j], scale[:, gcol[j]], zero[:, gcol[j]], bits)
             rho = W[:, j] - q
             eta = rho / R[j, j]
@@ -296,7 +323,8 @@ def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int):
     return codes, Q, loss
 
 
-def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: float = 1e-3):
+def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: float = 1e-3,
+                    dynamic: int = 0):
     """Check another implementation's codes against this recursion, decision by decision.
 
     Runs the unblocked Cholesky-form recursion ([T] eq.(42)) in fp64 on the same inputs, but at
@@ -308,6 +336,9 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
 
     Along the replayed decisions it also records Ŵ (replay_Q) and the per-column loss
     Σ_r ρ² / (2 R_jj²) ([T] eq.(43)), which are the oracle's values for those decisions.
+
+    dynamic = g > 0: the grid is refitted at group starts from the replay's own working
+    weights (scale / zero are overwritten), as in `gptq_explicit`.
 
     Returns dict(n, identical, in_band, violations, max_excess, replay_Q, replay_loss,
     rows_with_flips).
@@ -323,6 +354,7 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
     loss = np.zeros(d, np.float64)
     flipped = np.zeros(m, bool)
     for j in range(d):
+        _dynamic_refit(W, j, dynamic, bits, scale, zero)
         delta = np.asarray(scale[:, gcol[j]], np.float32)
         z = np.asarray(zero[:, gcol[j]], np.int64)
         c_o, _, u = quantize(W[:, j], delta, z, bits)
@@ -357,7 +389,7 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
 # --------------------------------------------------------------------------------------------
 def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 0.01,
                act_order: bool = False, method: str = "explicit", grid=None,
-               eps: float = FP32_EPS, perm=None):
+               eps: float = FP32_EPS, perm=None, dynamic: bool = False):
     """The layer-wise hot path of [T] §10, end to end on one layer.
 
     1. grid: fitted on the original W before anything else (static groups), unless given;
@@ -366,25 +398,35 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     4. the column recursion: `method` = "explicit" (eq.(22)/(26)) or "lazy" (eq.(42)/(46));
     5. un-permute codes, Ŵ and the per-column loss back to original column order.
 
+    dynamic=True (group > 0): dynamic groups ([T] §8.3): the grid of processing group j // g is
+    refitted at its start from the current working weights (step 1 is skipped), and the
+    returned scale / zero are indexed by processing group; group_id[π_j] = j // g maps each
+    original column to its group ([T] §8.3, §8.4 table).
+
     Returns a dict with codes [m,d] int64, W_hat [m,d], scale, zero, col_loss [d], perm, dead,
-    lam, G, R, H_lambda, Wp (the permuted working copy fed to the recursion), gcol.
+    lam, G, R, H_lambda, Wp (the permuted working copy fed to the recursion), gcol, group_id.
     """
     W = np.asarray(W, np.float64)
     m, d = W.shape
-    if grid is None:
+    if dynamic and group <= 0:
+        raise ValueError("dynamic groups need group > 0")
+    prep = prepare_with_retry(H, percdamp, act_order, eps, perm=perm)
+    perm, dead = prep["perm"], prep["dead"]
+    if dynamic:
+        scale, zero = dynamic_grid_arrays(m, d, group)
+    elif grid is None:
         scale, zero = fit_grid(W, bits, group)
     else:
         scale, zero = (np.asarray(grid[0], np.float32), np.asarray(grid[1], np.int32))
-    prep = prepare_with_retry(H, percdamp, act_order, eps, perm=perm)
-    perm, dead = prep["perm"], prep["dead"]
     Wwork = W.copy()
     Wwork[:, dead] = 0.0
     Wp = Wwork[:, perm]
-    gcol = _group_of_column(perm, d, group)
+    dyn = int(group) if dynamic else 0
+    gcol = np.arange(d) // dyn if dynamic else _group_of_column(perm, d, group)
     if method == "explicit":
-        codes_p, Q_p, loss_p, _ = gptq_explicit(Wp, prep["G"], scale, zero, gcol, bits)
+        codes_p, Q_p, loss_p, _ = gptq_explicit(Wp, prep["G"], scale, zero, gcol, bits, dyn)
     elif method == "lazy":
-        codes_p, Q_p, loss_p = gptq_lazy(Wp, prep["R"], scale, zero, gcol, bits, block)
+        codes_p, Q_p, loss_p = gptq_lazy(Wp, prep["R"], scale, zero, gcol, bits, block, dyn)
     else:
         raise ValueError(method)
     codes = np.empty_like(codes_p)
@@ -393,9 +435,12 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     codes[:, perm] = codes_p
     W_hat[:, perm] = Q_p
     col_loss[perm] = loss_p
+    group_id = np.empty(d, np.int64)
+    group_id[perm] = gcol
     return dict(codes=codes, W_hat=W_hat, scale=scale, zero=zero, col_loss=col_loss,
                 perm=perm, dead=dead, lam=prep["lam"], G=prep["G"], R=prep["R"],
-                H_lambda=prep["H_lambda"], retries=prep["retries"], Wp=Wp, gcol=gcol)
+                H_lambda=prep["H_lambda"], retries=prep["retries"], Wp=Wp, gcol=gcol,
+                group_id=group_id)
 
 
 def is_valid_act_order(perm, H, rtol: float = 1e-5) -> bool:

@@ -386,3 +386,78 @@ def test_pack_layout_definition():
         c = rng.integers(0, 2 ** bits, size=(3, 37))
         assert np.array_equal(O.unpack(O.pack(c, bits), 37, bits), c)
         assert O.pack(c, bits).shape[1] == O.words_per_row(37, bits)
+
+
+# ---------------------------------------------------------------- dynamic groups ([T] §8.3)
+def test_dynamic_one_group_is_the_row_grid():
+    """A single dynamic group covering the row is fitted at j = 0 on the untouched working
+    weights, i.e. it is the static row grid: identical results."""
+    W, X = _layer(8, 24, 100, 21)
+    H = O.hessian(X)
+    ref = O.gptq_layer(W, H, 4, -1, method="explicit")
+    dyn = O.gptq_layer(W, H, 4, 24, method="explicit", dynamic=True)
+    assert np.array_equal(dyn["codes"], ref["codes"])
+    assert np.array_equal(dyn["W_hat"], ref["W_hat"])
+    assert np.array_equal(dyn["scale"], ref["scale"]) and np.array_equal(dyn["zero"], ref["zero"])
+    assert np.array_equal(dyn["group_id"], np.zeros(24, np.int64))
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+def test_dynamic_diagonal_hessian_is_rtn_on_processing_groups(act_order):
+    """With a diagonal H nothing is compensated, so the working weights never change: each
+    dynamic group is the static min-max fit of its processing-order columns and the codes are
+    round-to-nearest on that grid.  group_id maps original columns to processing groups."""
+    W, _ = _layer(9, 24, 10, 22)
+    dg = np.random.default_rng(2).uniform(0.5, 2.0, 24)
+    H = np.diag(dg)
+    out = O.gptq_layer(W, H, 3, 8, method="explicit", act_order=act_order, dynamic=True)
+    perm = out["perm"]
+    if act_order:
+        assert np.array_equal(perm, np.argsort(-dg, kind="stable"))
+    Wp = W[:, perm]
+    sc, ze = O.fit_grid(Wp, 3, 8)
+    assert np.array_equal(out["scale"], sc) and np.array_equal(out["zero"], ze)
+    c, q = O.quantize_rtn(Wp, sc, ze, 3, 8)
+    assert np.array_equal(out["codes"][:, perm], c) and np.allclose(out["W_hat"][:, perm], q)
+    assert np.array_equal(out["group_id"][perm], np.arange(24) // 8)
+
+
+@pytest.mark.parametrize("group,blocks", [(4, [1, 2, 4, 8, 12]), (8, [4, 8, 16])])
+def test_dynamic_lazy_equals_unblocked(group, blocks):
+    """Lazy blocks give the unblocked result when every group starts on a block start or lies
+    inside one block ([T] eq.(47)-(49) with the grid refitted from current weights)."""
+    W, X = _layer(10, 40, 160, 23)
+    H = O.hessian(X)
+    ref = O.gptq_layer(W, H, 4, group, method="explicit", act_order=True, dynamic=True)
+    for block in blocks:
+        out = O.gptq_layer(W, H, 4, group, block=block, method="lazy", act_order=True,
+                           dynamic=True)
+        assert np.array_equal(out["codes"], ref["codes"]), block
+        assert np.array_equal(out["zero"], ref["zero"]), block
+        assert np.allclose(out["scale"], ref["scale"], rtol=1e-6), block
+        assert np.allclose(out["W_hat"], ref["W_hat"], rtol=1e-6, atol=1e-9), block
+    with pytest.raises(ValueError):
+        O.gptq_layer(W, H, 4, 8, block=3, method="lazy", dynamic=True)
+
+
+def test_dynamic_grid_moves_with_compensation():
+    """With cross-column compensation the second group's grid is fitted on compensated weights,
+    so it differs from the static fit of the original weights (the heuristic the pages warn
+    about, [T] §8.4 remark), while the first group's does not."""
+    W, X = _layer(6, 16, 80, 24)
+    H = O.hessian(X)
+    dyn = O.gptq_layer(W, H, 4, 8, method="explicit", dynamic=True)
+    sc, ze = O.fit_grid(W, 4, 8)
+    assert np.array_equal(dyn["scale"][:, 0], sc[:, 0])
+    assert not np.array_equal(dyn["scale"][:, 1], sc[:, 1])
+
+
+def test_dynamic_replay_accepts_self():
+    W, X = _layer(12, 32, 120, 25)
+    H = O.hessian(X)
+    out = O.gptq_layer(W, H, 4, 8, method="lazy", block=16, act_order=True, dynamic=True)
+    codes_p = out["codes"][:, out["perm"]]
+    sc, ze = O.dynamic_grid_arrays(12, 32, 8)
+    rep = O.decision_replay(out["Wp"], out["R"], sc, ze, out["gcol"], 4, codes_p, dynamic=8)
+    assert rep["identical"] == rep["n"] and rep["violations"] == 0
+    assert np.array_equal(ze, out["zero"]) and np.allclose(sc, out["scale"], rtol=1e-6)
