@@ -109,7 +109,7 @@ int gptq_prepare_hinv(gptq_ctx* ctx, float* S, int64_t n_total, int64_t d, float
                       float* damp_used, int* retries);
 
 /* Column-by-column quantization with lazy block updates, [W] Algorithm 1, [T] §9.2-9.3
- * eq.(42)-(46) and §10; quantizer [T] eq.(36); static groups [T] §8.3.
+ * eq.(42)-(46) and §10; quantizer [T] eq.(36); static and dynamic groups [T] §8.3.
  *   W        [m, d] weights of type w_dtype (GPTQ_F16 / GPTQ_BF16 / GPTQ_F32), ORIGINAL
  *            column order; not modified.
  *   R, perm, dead  as produced by gptq_prepare_hinv for this layer's H.
@@ -119,9 +119,16 @@ int gptq_prepare_hinv(gptq_ctx* ctx, float* S, int64_t n_total, int64_t d, float
  *   block    lazy block size B >= 1.  Blocks of up to 128 columns are run as given; a larger
  *            B is run as 128-column blocks, which gives the same result in exact arithmetic
  *            ([T] eq.(47)-(49)).
- *   grid_given 0: fit a min-max grid on the original W (range extended to contain 0,
- *            Δ = (max - min) / (2^b - 1), z = clip(rint(-min / Δ)); all-zero range -> Δ = 1)
- *            and write it to scales/zeros; 1: read scales/zeros as the fixed grid.
+ *   grid_given 0: static groups: fit a min-max grid on the original W (range extended to
+ *            contain 0, Δ = (max - min) / (2^b - 1), z = clip(rint(-min / Δ)); all-zero range
+ *            -> Δ = 1) and write it to scales/zeros; 1: read scales/zeros as the fixed grid;
+ *            2: dynamic groups ([T] §8.3): group k holds PROCESSING positions k g .. k g + g - 1
+ *            and its grid is fitted by the same rule, per row, at the group's start from the
+ *            current working weights (all earlier columns' compensation applied); scales/zeros
+ *            are written and indexed by processing group, and original column π_j belongs to
+ *            group j / g (the deployment metadata group_id[π_j] = j / g, from perm).  Needs
+ *            group == 32 (with min(block, 128) a multiple of 32) or group == 128 (with
+ *            block >= 128); otherwise ARG.
  *   scales   [m, n_g] fp32, zeros [m, n_g] int32 (in or out, see grid_given).
  *   codes    [m, d] uint8 out, W_hat [m, d] fp32 out (= Δ (c - z)), col_loss [d] fp32 out
  *            (Σ_rows ρ² / (2 R_jj²), [T] eq.(43)); all in ORIGINAL column order.

@@ -324,7 +324,7 @@ def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int, dynamic: int = 0)
 
 
 def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: float = 1e-3,
-                    dynamic: int = 0):
+                    dynamic: int = 0, other_zero=None):
     """Check another implementation's codes against this recursion, decision by decision.
 
     Runs the unblocked Cholesky-form recursion ([T] eq.(42)) in fp64 on the same inputs, but at
@@ -338,10 +338,14 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
     Σ_r ρ² / (2 R_jj²) ([T] eq.(43)), which are the oracle's values for those decisions.
 
     dynamic = g > 0: the grid is refitted at group starts from the replay's own working
-    weights (scale / zero are overwritten), as in `gptq_explicit`.
+    weights (scale / zero are overwritten), as in `gptq_explicit`.  With `other_zero` (the other
+    implementation's zero points, [m, n_groups]) the integer zero point is a decision too: the
+    replay follows the other's z, accepting a difference iff the two are adjacent and the
+    replay's pre-round value -x_min / Δ lies within `band` of the boundary between them; Δ
+    stays the replay's own.
 
     Returns dict(n, identical, in_band, violations, max_excess, replay_Q, replay_loss,
-    rows_with_flips).
+    rows_with_flips, grid_in_band, grid_violations).
     """
     W = np.array(Wp, dtype=np.float64, copy=True)
     R = np.asarray(R, np.float64)
@@ -353,8 +357,25 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
     Qr = np.zeros((m, d), np.float64)
     loss = np.zeros(d, np.float64)
     flipped = np.zeros(m, bool)
+    grid_in_band = grid_violations = 0
     for j in range(d):
         _dynamic_refit(W, j, dynamic, bits, scale, zero)
+        if dynamic > 0 and other_zero is not None and j % dynamic == 0:
+            k = j // dynamic
+            z_o = np.asarray(zero[:, k], np.int64)
+            z_g = np.asarray(other_zero, np.int64)[:, k]
+            zdiff = z_o != z_g
+            if np.any(zdiff):
+                # the pre-round value of z as fit_grid forms it (fp32)
+                x_min = np.minimum(W[:, j:j + dynamic].astype(np.float32).min(axis=1),
+                                   np.float32(0.0))
+                t = (-x_min / np.asarray(scale[:, k], np.float32)).astype(np.float32)
+                lo = np.minimum(z_o, z_g)[zdiff]
+                dist = np.abs(t[zdiff].astype(np.float64) - (lo + 0.5))
+                ok = (np.abs(z_o - z_g)[zdiff] == 1) & (dist <= band)
+                grid_in_band += int(np.sum(ok))
+                grid_violations += int(np.sum(~ok))
+            zero[:, k] = z_g
         delta = np.asarray(scale[:, gcol[j]], np.float32)
         z = np.asarray(zero[:, gcol[j]], np.int64)
         c_o, _, u = quantize(W[:, j], delta, z, bits)
@@ -381,7 +402,8 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
         W[:, j:] -= np.outer(eta, R[j, j:])
         Qr[:, j] = q
     return dict(n=m * d, identical=identical, in_band=in_band, violations=violations,
-                max_excess=max_excess, replay_Q=Qr, replay_loss=loss, rows_with_flips=flipped)
+                max_excess=max_excess, replay_Q=Qr, replay_loss=loss, rows_with_flips=flipped,
+                grid_in_band=grid_in_band, grid_violations=grid_violations)
 
 
 # --------------------------------------------------------------------------------------------

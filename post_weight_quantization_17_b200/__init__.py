@@ -158,8 +158,9 @@ def gptq_prepare_hinv(ctx: Context, S, n_total: int, percdamp: float, act_order:
 
 
 def gptq_quantize_layer(ctx: Context, W, R, perm, dead, bits: int, group: int, block: int,
-                        grid_given: bool, scales, zeros, codes, W_hat, col_loss):
-    """perm / dead may be None (identity order / no dead features)."""
+                        grid_given, scales, zeros, codes, W_hat, col_loss):
+    """perm / dead may be None (identity order / no dead features).  grid_given: False / 0 fit a
+    static grid, True / 1 use the given one, 2 dynamic groups (see include/gptq.h)."""
     m, d = W.shape
     _dev(W, name="W")
     for t, dt, nm in ((R, torch.float32, "R"), (scales, torch.float32, "scales"),
@@ -168,7 +169,7 @@ def gptq_quantize_layer(ctx: Context, W, R, perm, dead, bits: int, group: int, b
         _dev(t, dt, nm)
     rc = _lib.gptq_quantize_layer(ctx.handle, _ptr(W), _DTYPE_CODE[W.dtype], m, d, _ptr(R),
                                   _ptr(perm), _ptr(dead), bits, group, block,
-                                  1 if grid_given else 0, _ptr(scales), _ptr(zeros), _ptr(codes),
+                                  int(grid_given), _ptr(scales), _ptr(zeros), _ptr(codes),
                                   _ptr(W_hat), _ptr(col_loss))
     ctx.check(rc, "gptq_quantize_layer")
 
@@ -183,7 +184,7 @@ def gptq_quantize_layer_noalloc(W, R, perm, dead, bits: int, group: int, block: 
     s = stream if stream is not None else torch.cuda.current_stream(W.device)
     return int(_lib.gptq_quantize_layer_noalloc(
         ctypes.c_void_p(s.cuda_stream), _ptr(W), _DTYPE_CODE[W.dtype], m, d, _ptr(R), _ptr(perm),
-        _ptr(dead), bits, group, block, 1 if grid_given else 0, _ptr(scales), _ptr(zeros),
+        _ptr(dead), bits, group, block, int(grid_given), _ptr(scales), _ptr(zeros),
         _ptr(codes), _ptr(W_hat), _ptr(col_loss)))
 
 

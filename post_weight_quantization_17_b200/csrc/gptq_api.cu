@@ -194,9 +194,17 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   Ctx* c = &h->c;
   if (!W || !R || !scales || !zeros || !codes || !W_hat || !col_loss || !valid_dtype(w_dtype) ||
       m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || (long long)m * d > (1LL << 40) ||
-      bits < 1 || bits > 8 || !(group == -1 || group > 0) || block < 1)
+      bits < 1 || bits > 8 || !(group == -1 || group > 0) || block < 1 || grid_given < 0 ||
+      grid_given > 2)
     GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "quantize_layer: bad argument (m=%lld d=%lld bits=%d group=%d block=%d)",
                  (long long)m, (long long)d, bits, group, block);
+  // dynamic groups: a group is one 32-column sub-block or one 128-column block of the column
+  // kernel, so that the grid is fitted on columns that are all current at its start
+  const int dyn = (grid_given == 2) ? group : 0;
+  if (dyn && !((dyn == 32 && std::min(block, gptq::kColMax) % 32 == 0) ||
+               (dyn == 128 && block >= gptq::kColMax)))
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "quantize_layer: dynamic groups need group 32 (block a multiple of 32) or 128 (block >= 128), got group=%d block=%d",
+                 group, block);
   const int mi = (int)m, di = (int)d;
   const bool general = perm != nullptr;
   const int g = (group == -1) ? di : group;
@@ -224,9 +232,9 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   const bool pair_ws = cv.ok();
   if (!pair_ws) Ehi = Elo = Rhi = Rlo = nullptr;
   int rc;
-  if (!grid_given && (rc = gptq::grid_fit(c, W, w_dtype, mi, di, bits, group, scales, zeros)))
+  if (grid_given == 0 && (rc = gptq::grid_fit(c, W, w_dtype, mi, di, bits, group, scales, zeros)))
     return rc;
-  if ((rc = gptq::make_gcol(c, perm, di, group, gcol, general ? inv : nullptr))) return rc;
+  if ((rc = gptq::make_gcol(c, perm, di, group, dyn != 0, gcol, general ? inv : nullptr))) return rc;
   if ((rc = gptq::init_work(c, W, w_dtype, mi, di, perm, dead, !general, Wk))) return rc;
   // Two-level lazy blocks ([T] eq.(46); exact in exact arithmetic by eq.(47)-(49)): columns
   // are quantized in tiles of bk <= 128; after a tile only the rest of its super-block of
@@ -238,10 +246,10 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
     const int s1 = std::min(di, s0 + sb);
     for (int i = s0; i < s1; i += bk) {
       const int nb = std::min(bk, s1 - i);
-      const bool uniform = (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
+      const bool uniform = dyn || (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
       float* Et = E + (i - s0);
       if ((rc = gptq::column_block(c, Wk, mi, di, i, nb, R, scales, zeros, ng, gcol, uniform,
-                                   bits, Et, Ehi ? Ehi + (i - s0) : nullptr,
+                                   dyn, bits, Et, Ehi ? Ehi + (i - s0) : nullptr,
                                    Elo ? Elo + (i - s0) : nullptr, gptq::kSuperCols, codes_p,
                                    loss_part)))
         return rc;

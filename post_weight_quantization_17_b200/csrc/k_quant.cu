@@ -127,21 +127,22 @@ int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int gro
   return GPTQ_OK;
 }
 
-// grid index of each processing position (static groups: floor(π_j / g)) and the inverse
-// permutation.
-__global__ void k_gcol(const int32_t* __restrict__ perm, int d, int group,
+// grid index of each processing position (static groups: floor(π_j / g); dynamic groups:
+// j / g) and the inverse permutation.
+__global__ void k_gcol(const int32_t* __restrict__ perm, int d, int group, int dynamic,
                        int32_t* __restrict__ gcol, int32_t* __restrict__ inv) {
   pdl_wait();
   pdl_release();
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= d) return;
   int p = perm ? perm[j] : j;
-  gcol[j] = (group == -1) ? 0 : p / group;
+  gcol[j] = (group == -1) ? 0 : (dynamic ? j : p) / group;
   if (inv) inv[p] = j;
 }
 
-int make_gcol(Ctx* c, const int32_t* perm, int d, int group, int32_t* gcol, int32_t* inv) {
-  GPTQ_LAUNCH(c, k_gcol, (d + 255) / 256, 256, 0, perm, d, group, gcol, inv);
+int make_gcol(Ctx* c, const int32_t* perm, int d, int group, bool dynamic, int32_t* gcol,
+              int32_t* inv) {
+  GPTQ_LAUNCH(c, k_gcol, (d + 255) / 256, 256, 0, perm, d, group, dynamic ? 1 : 0, gcol, inv);
   return GPTQ_OK;
 }
 
@@ -250,6 +251,24 @@ __device__ __forceinline__ float quotient(float w, float delta, float y) {
   return fmaf(r, y, q0);
 }
 
+// The min-max fit of the static grid (the fp32 arithmetic of k_gridfit) from a row's range.
+__device__ __forceinline__ void fit_from_range(float mn, float mx, float maxq, float& delta,
+                                               float& z) {
+  mn = fminf(mn, 0.f);
+  mx = fmaxf(mx, 0.f);
+  delta = (mx == mn) ? 1.f : __fdiv_rn(__fsub_rn(mx, mn), maxq);
+  z = fminf(fmaxf(rintf(__fdiv_rn(-mn, delta)), 0.f), maxq);
+}
+
+// min and max over the 8 lanes that hold one row
+__device__ __forceinline__ void row_range(float& mn, float& mx) {
+#pragma unroll
+  for (int o = 1; o < kColLanes; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+}
+
 struct ColStepArgs {
   const float (*Rs)[128];
   const int* gs;
@@ -310,7 +329,9 @@ __device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128
                                          const ColStepArgs& args, int r, int row, int nb, int d,
                                          int i, int ldE, bool vec, float* __restrict__ Wk,
                                          float* __restrict__ E, float* __restrict__ Ehi,
-                                         float* __restrict__ Elo, uint8_t* __restrict__ codes) {
+                                         float* __restrict__ Elo, uint8_t* __restrict__ codes,
+                                         int dyn, int ng, float* __restrict__ dscales,
+                                         int32_t* __restrict__ dzeros) {
   const float(*Rs)[128] = args.Rs;
   const int q = args.q, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll 1
@@ -334,7 +355,23 @@ __device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128
         w[3] = fmaf(-e[u], r4.w, w[3]);
       }
     }
-    col_steps<UNIFORM, FAST>(w, e4, c4, args, off, std::make_integer_sequence<int, kColSub>{});
+    ColStepArgs sa = args;
+    if (dyn == kColSub) {
+      // dynamic group = this sub-block: its grid is fitted per row from the current weights
+      // (every earlier column's compensation is in w now)
+      float mn = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
+      float mx = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
+      row_range(mn, mx);
+      float dlt, zz;
+      fit_from_range(mn, mx, args.maxq, dlt, zz);
+      sa.D0 = dlt;
+      sa.Z0 = zz;
+      if (q == 0 && args.active) {
+        dscales[args.srow + (i + off) / kColSub] = dlt;
+        dzeros[args.srow + (i + off) / kColSub] = (int32_t)zz;
+      }
+    }
+    col_steps<UNIFORM, FAST>(w, e4, c4, sa, off, std::make_integer_sequence<int, kColSub>{});
     // the sub-block's η for later sub-blocks; outputs straight from registers
     __syncwarp();
     *reinterpret_cast<float4*>(&St[r][off + 4 * q]) = make_float4(e4[0], e4[1], e4[2], e4[3]);
@@ -388,8 +425,9 @@ __device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128
 template <bool UNIFORM>
 __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     float* __restrict__ Wk, int m, int d, int i, int nb, const float* __restrict__ R,
-    const float* __restrict__ scales, const int32_t* __restrict__ zeros, int ng,
-    const int32_t* __restrict__ gcol, int bits, float* __restrict__ E, float* __restrict__ Ehi,
+    float* __restrict__ scales, int32_t* __restrict__ zeros, int ng,
+    const int32_t* __restrict__ gcol, int dyn, int bits, float* __restrict__ E,
+    float* __restrict__ Ehi,
     float* __restrict__ Elo, int ldE, uint8_t* __restrict__ codes,
     float* __restrict__ loss_part) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -463,7 +501,30 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
   args.maxq = (float)((1 << bits) - 1);
   args.D0 = 1.f; args.Z0 = 0.f; args.Y0 = 1.f;
   bool fast = true;
-  if (UNIFORM) {
+  if (UNIFORM && dyn == 128) {
+    // dynamic group = this kernel block: its grid is fitted per row from the staged block,
+    // which holds the current weights (zeros beyond nb leave the range, which contains 0, as is)
+    float mn = 0.f, mx = 0.f;
+#pragma unroll
+    for (int sb = 0; sb < 128 / kColSub; ++sb) {
+      const float4 v = *reinterpret_cast<const float4*>(&St[r][sb * kColSub + 4 * q]);
+      mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
+      mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+    }
+    row_range(mn, mx);
+    float dlt, zz;
+    fit_from_range(mn, mx, args.maxq, dlt, zz);
+    args.D0 = dlt;
+    args.Z0 = zz;
+    args.Y0 = __frcp_rn(dlt);
+    fast = quotient_fast(dlt);
+    if (q == 0 && active) {
+      scales[args.srow + i / 128] = dlt;
+      zeros[args.srow + i / 128] = (int32_t)zz;
+    }
+  } else if (UNIFORM && dyn == kColSub) {
+    fast = false;  // each sub-block fits its own grid inside the walk; Δ is divided by
+  } else if (UNIFORM) {
     if (active) {
       args.D0 = scales[args.srow + gcol[i]];
       args.Z0 = (float)zeros[args.srow + gcol[i]];
@@ -475,9 +536,11 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
   }
   fast = __syncthreads_and(fast);  // also publishes rinv and gs
   if (fast)
-    col_walk<UNIFORM, true>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, Ehi, Elo, codes);
+    col_walk<UNIFORM, true>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, Ehi, Elo, codes,
+                          dyn, ng, scales, zeros);
   else
-    col_walk<UNIFORM, false>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, Ehi, Elo, codes);
+    col_walk<UNIFORM, false>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, Ehi, Elo, codes,
+                          dyn, ng, scales, zeros);
   __syncthreads();
   // loss partial Σ_rows η² per column, the 8 warps' sums in a fixed order
   for (int t = tid; t < nb; t += blockDim.x) {
@@ -488,21 +551,20 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
   }
 }
 
-int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
-                 const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
-                 bool uniform_grid, int bits, float* E, float* Ehi, float* Elo, int ldE,
-                 uint8_t* codes, float* loss_part) {
+int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R, float* scales,
+                 int32_t* zeros, int ng, const int32_t* gcol, bool uniform_grid, int dyn, int bits,
+                 float* E, float* Ehi, float* Elo, int ldE, uint8_t* codes, float* loss_part) {
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<false>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
   const int blocks = (m + kColCtaRows - 1) / kColCtaRows;
-  if (uniform_grid)
+  if (uniform_grid || dyn)
     GPTQ_LAUNCH(c, k_colblock<true>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales,
-                zeros, ng, gcol, bits, E, Ehi, Elo, ldE, codes, loss_part);
+                zeros, ng, gcol, dyn, bits, E, Ehi, Elo, ldE, codes, loss_part);
   else
     GPTQ_LAUNCH(c, k_colblock<false>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales,
-                zeros, ng, gcol, bits, E, Ehi, Elo, ldE, codes, loss_part);
+                zeros, ng, gcol, 0, bits, E, Ehi, Elo, ldE, codes, loss_part);
   return GPTQ_OK;
 }
 

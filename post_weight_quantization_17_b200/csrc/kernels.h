@@ -24,13 +24,17 @@ int factor_inverse(Ctx* c, float* M, int d, float* tmp);
 // ---- a4-a7 quantization
 int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int group,
              float* scales, int32_t* zeros);
-int make_gcol(Ctx* c, const int32_t* perm, int d, int group, int32_t* gcol, int32_t* inv);
+// grid index of each processing position: static groups floor(π_j / g), dynamic groups j / g
+int make_gcol(Ctx* c, const int32_t* perm, int d, int group, bool dynamic, int32_t* gcol,
+              int32_t* inv);
 int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* perm,
               const uint8_t* dead, bool identity, float* Wk);
 // E (and, if not null, its tf32 halves Ehi / Elo) receive the block's scaled residuals.
+// dyn = 32 or 128: dynamic groups of that many processing positions, whose grid the kernel
+// fits and writes to scales/zeros; 0: the grid is read from scales/zeros.
 int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
-                 const float* scales, const int32_t* zeros, int ng, const int32_t* gcol,
-                 bool uniform_grid, int bits, float* E, float* Ehi, float* Elo, int ldE,
+                 float* scales, int32_t* zeros, int ng, const int32_t* gcol,
+                 bool uniform_grid, int dyn, int bits, float* E, float* Ehi, float* Elo, int ldE,
                  uint8_t* codes, float* loss_part);
 // Tail update on CTA pairs with operands split into tf32 halves (k_gemm_pair.cu):
 // C = alpha A B + beta C, A [M, K] (lda), B [K, N] (ldb), both row-major.

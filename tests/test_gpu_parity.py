@@ -1,5 +1,7 @@
 """GPU parity: the C-ABI path against the fp64 oracle on the same seeded inputs, at sizes the
 oracle finishes in seconds that still span several tiles and ragged tails."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -49,6 +51,88 @@ def test_layer_parity(ctx, name, spec, seed):
     H, herr = P.check_hessian(gpu, Xt)
     res = P.check_layer(gpu, Wn, H, spec)
     print(name, f"H={herr:.2e}", {k: (f"{v:.2e}" if isinstance(v, float) else v) for k, v in res.items()})
+
+
+STATIC_MORE = [
+    # 32-column groups with 2 bits: several grids inside one column-kernel block
+    ("static_g32_2bit", dataclasses.replace(
+        CONFIGS[5][1].scaled(130, 256, 2048, chunk=512), group=32), 12),
+    # 8-column groups under act-order: the per-column grid lookup of the general path
+    ("static_g8_actorder", dataclasses.replace(
+        CONFIGS[3][0].scaled(64, 200, 1500, chunk=500), group=8, bits=4), 13),
+]
+
+
+@pytest.mark.parametrize("name,spec,seed", STATIC_MORE, ids=[c[0] for c in STATIC_MORE])
+def test_static_small_groups_parity(ctx, name, spec, seed):
+    W, chunks = P.make_inputs(spec, seed)
+    gpu = P.gpu_run(ctx, spec, W, chunks)
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    H, herr = P.check_hessian(gpu, Xt)
+    res = P.check_layer(gpu, P.to_np64(W), H, spec)
+    print(name, f"H={herr:.2e}", {k: (f"{v:.2e}" if isinstance(v, float) else v) for k, v in res.items()})
+
+
+@pytest.mark.parametrize("act_order", [False, True])
+def test_given_symmetric_grid_parity(ctx, act_order):
+    """grid_given = 1: a caller-chosen grid (here symmetric, z = 2^(b-1), Δ = 2 max|w| / maxq
+    per row and group of 128) is used as is and returned untouched."""
+    spec = dataclasses.replace(CONFIGS[2][0].scaled(96, 384, 2000, chunk=1000),
+                               act_order=act_order)
+    W, chunks = P.make_inputs(spec, 14)
+    Wn = P.to_np64(W)
+    maxq = 2 ** spec.bits - 1
+    amax = np.abs(Wn.astype(np.float32)).reshape(96, -1, 128).max(axis=2)
+    scales = np.where(amax > 0, 2 * amax / np.float32(maxq), 1).astype(np.float32)
+    zeros = np.full(scales.shape, (maxq + 1) // 2, np.int32)
+    gpu = P.gpu_run(ctx, spec, W, chunks, grid=(scales, zeros))
+    assert np.array_equal(gpu["scales"], scales) and np.array_equal(gpu["zeros"], zeros)
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    H, _ = P.check_hessian(gpu, Xt)
+    res = P.check_layer(gpu, Wn, H, spec, grid=(scales, zeros))
+    print("given_grid", act_order, res)
+
+
+DYNAMIC = [
+    # g = 128: one grid per kernel block, fitted from the staged block; ragged last group
+    ("dyn128_qproj_shape", CONFIGS[2][0].scaled(160, 600, 3000, chunk=1024), 1, 128),
+    # g = 32: one grid per sub-block, with act-order and 3 bits; ragged rows and last group
+    ("dyn32_downproj_actorder", dataclasses.replace(
+        CONFIGS[3][0].scaled(77, 300, 2000, chunk=700), group=32), 2, 128),
+    # g = 32 inside 64-column blocks; 2 bits
+    ("dyn32_block64_2bit", dataclasses.replace(
+        CONFIGS[5][1].scaled(130, 256, 2048, chunk=512), group=32, block=64), 4, 64),
+    # g = 128 under blocks of 256 (the kernel still walks 128-column blocks); m >= 256 reaches
+    # the pair tail GEMM
+    ("dyn128_block256_pair_tail", dataclasses.replace(
+        CONFIGS[2][0].scaled(300, 1100, 2500, chunk=1000), block=256), 10, 256),
+]
+
+
+@pytest.mark.parametrize("name,spec,seed,block", DYNAMIC, ids=[c[0] for c in DYNAMIC])
+def test_dynamic_groups_parity(ctx, name, spec, seed, block):
+    """grid_given = 2: each processing group's grid is fitted on the GPU from the current
+    working weights at its start ([T] §8.3), against the oracle's dynamic recursion."""
+    W, chunks = P.make_inputs(spec, seed)
+    gpu = P.gpu_run(ctx, spec, W, chunks, block=block, grid_given=2)
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    H, herr = P.check_hessian(gpu, Xt)
+    res = P.check_layer(gpu, P.to_np64(W), H, spec, block=block, dynamic=True)
+    print(name, f"H={herr:.2e}", {k: (f"{v:.2e}" if isinstance(v, float) else v) for k, v in res.items()})
+
+
+def test_dynamic_groups_rejects_unsupported(ctx):
+    """Dynamic groups other than 32 / 128, or a group that a column block would split, are
+    argument errors reported by the library, not silently static."""
+    import post_weight_quantization_17_b200 as G
+    spec = CONFIGS[2][0].scaled(64, 256, 512, chunk=512)
+    W, chunks = P.make_inputs(spec, 3)
+    for group, block in ((64, 128), (128, 64), (32, 48)):
+        bufs = G.LayerBuffers(64, 256, 4, group, W.device)
+        bufs.R.copy_(torch.eye(256))
+        with pytest.raises(RuntimeError):
+            G.gptq_quantize_layer(ctx, W, bufs.R, None, bufs.dead, 4, group, block, 2, bufs.scales,
+                                  bufs.zeros, bufs.codes, bufs.W_hat, bufs.col_loss)
 
 
 @pytest.mark.parametrize("d", [700, 257, 1000])

@@ -461,3 +461,32 @@ def test_dynamic_replay_accepts_self():
     rep = O.decision_replay(out["Wp"], out["R"], sc, ze, out["gcol"], 4, codes_p, dynamic=8)
     assert rep["identical"] == rep["n"] and rep["violations"] == 0
     assert np.array_equal(ze, out["zero"]) and np.allclose(sc, out["scale"], rtol=1e-6)
+
+
+def test_dynamic_replay_zero_point_decisions():
+    """With the other side's zero points given, the replay counts a differing z as in band only
+    when it is adjacent and -x_min / Δ sits on the rounding boundary: a row fitted on
+    [-1, 5] with 4 bits has Δ = 0.4 and -x_min / Δ = 2.5 exactly, so z = 2 (the oracle's
+    ties-to-even) and z = 3 are both correct; a z moved by one anywhere else is a violation."""
+    W, _ = _layer(4, 16, 10, 26)
+    W[0, :] = np.linspace(-1.0, 5.0, 16)
+    H = np.diag(np.linspace(1.0, 2.0, 16))
+    out = O.gptq_layer(W, H, 4, 16, method="explicit", dynamic=True)
+    assert out["zero"][0, 0] == 2 and out["scale"][0, 0] == np.float32(0.4)
+    codes_p = out["codes"][:, out["perm"]]
+
+    def replay(other_zero):
+        sc, ze = O.dynamic_grid_arrays(4, 16, 16)
+        return O.decision_replay(out["Wp"], out["R"], sc, ze, out["gcol"], 4, codes_p,
+                                 dynamic=16, other_zero=other_zero)
+
+    rep = replay(out["zero"])
+    assert rep["grid_in_band"] == 0 and rep["grid_violations"] == 0 and rep["violations"] == 0
+    tie = out["zero"].copy()
+    tie[0, 0] = 3
+    rep = replay(tie)
+    assert rep["grid_in_band"] == 1 and rep["grid_violations"] == 0
+    bad = out["zero"].copy()
+    bad[1, 0] += 1 if bad[1, 0] < 15 else -1
+    rep = replay(bad)
+    assert rep["grid_violations"] == 1
