@@ -32,6 +32,9 @@ METRIC = "GPTQ weights quantized/sec per layer (4-bit g128) on 1 B200; % of roof
 UNIT = "weights/s"
 
 
+GRID_MODES = {"static": 0, "dynamic": 2}  # the library's grid_given argument
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -43,6 +46,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scale", type=float, default=1.0,
                     help="shrink the layer (tests only); the bench line is for 1.0")
+    ap.add_argument("--grid", choices=sorted(GRID_MODES), default="static",
+                    help="static groups (the default line) or dynamic groups (grid refitted per "
+                         "processing group on the GPU)")
     ap.add_argument("--n-tokens", type=int, default=0,
                     help="calibration tokens (profiling captures only; the bench line uses all)")
     return ap.parse_args()
@@ -60,9 +66,12 @@ def workload(scale: float, n_tokens: int = 0):
     return spec
 
 
-def workload_config(spec, chunk):
+def workload_config(spec, chunk, grid="static"):
     return {"workload": f"q_proj {spec.m}x{spec.d} fp16 W, N={spec.n_tokens} bf16 tokens, "
-                        f"{spec.bits}-bit g{spec.group}, block {spec.block}",
+                        f"{spec.bits}-bit g{spec.group}" +
+                        (" (dynamic groups)" if grid == "dynamic" else "") +
+                        f", block {spec.block}",
+            "grid": grid,
             "m": spec.m, "d": spec.d, "n_tokens": spec.n_tokens, "bits": spec.bits,
             "group": spec.group, "block": spec.block, "act_order": spec.act_order,
             "chunk_tokens": min(chunk, spec.n_tokens),
@@ -205,7 +214,7 @@ def weak_scaling_value(world: int, m: int, d: int, per_step_s: float) -> float:
 
 
 # ----------------------------------------------------------------------------- oracle leg
-def oracle_sample(spec, seed: int, n_tok: int, rows: int):
+def oracle_sample(spec, seed: int, n_tok: int, rows: int, grid: str = "static"):
     """The CPU oracle on a bounded sample of the layer: H from `n_tok` tokens at full d,
     preparation at full d, lazy-block quantization of `rows` rows.  Returns (seconds for the
     sample, seconds extrapolated to the whole layer, description)."""
@@ -222,10 +231,15 @@ def oracle_sample(spec, seed: int, n_tok: int, rows: int):
     t1 = time.perf_counter()
     prep = O.prepare_with_retry(H, spec.percdamp, spec.act_order)
     t2 = time.perf_counter()
-    sc, ze = O.fit_grid(W, spec.bits, spec.group)
     Wp = W[:, prep["perm"]]
-    gcol = (prep["perm"] // spec.group) if spec.group != -1 else np.zeros(spec.d, int)
-    O.gptq_lazy(Wp, prep["R"], sc, ze, gcol, spec.bits, spec.block)
+    if grid == "dynamic":
+        sc, ze = O.dynamic_grid_arrays(rows, spec.d, spec.group)
+        O.gptq_lazy(Wp, prep["R"], sc, ze, np.arange(spec.d) // spec.group, spec.bits,
+                    spec.block, dynamic=spec.group)
+    else:
+        sc, ze = O.fit_grid(W, spec.bits, spec.group)
+        gcol = (prep["perm"] // spec.group) if spec.group != -1 else np.zeros(spec.d, int)
+        O.gptq_lazy(Wp, prep["R"], sc, ze, gcol, spec.bits, spec.block)
     t3 = time.perf_counter()
     full = (t1 - t0) * (spec.n_tokens / n_tok) + (t2 - t1) + (t3 - t2) * (spec.m / rows)
     desc = (f"H from {n_tok} of {spec.n_tokens} tokens (time x{spec.n_tokens / n_tok:g}), "
@@ -249,12 +263,12 @@ def run_reference(args):
     spec = workload(args.scale, args.n_tokens)
     n_tok, rows = min(2048, spec.n_tokens), min(16, spec.m)
     for _ in range(args.warmup):
-        oracle_sample(spec, 1, n_tok, rows)
+        oracle_sample(spec, 1, n_tok, rows, args.grid)
     fulls = []
     desc = ""
     t_start = time.perf_counter()
     for _ in range(args.steps):
-        _, full, desc = oracle_sample(spec, 1, n_tok, rows)
+        _, full, desc = oracle_sample(spec, 1, n_tok, rows, args.grid)
         fulls.append(full)
     wall = time.perf_counter() - t_start
     per_layer = sum(fulls) / len(fulls)
@@ -263,7 +277,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_layer * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(spec, args.chunk),
+            "config": workload_config(spec, args.chunk, args.grid),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores_used(),
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -316,7 +330,8 @@ def run_ours(args):
         G.gptq_prepare_hinv(ctx, bufs.S, n, spec.percdamp, spec.act_order, bufs.R, bufs.perm,
                             bufs.dead)
         G.gptq_quantize_layer(ctx, W, bufs.R, bufs.perm if spec.act_order else None, bufs.dead,
-                              spec.bits, spec.group, spec.block, False, bufs.scales, bufs.zeros,
+                              spec.bits, spec.group, spec.block, GRID_MODES[args.grid],
+                              bufs.scales, bufs.zeros,
                               bufs.codes, bufs.W_hat, bufs.col_loss)
         G.gptq_pack(ctx, bufs.codes, spec.bits, bufs.packed)
 
@@ -411,7 +426,8 @@ def run_ours(args):
                 G.gptq_prepare_hinv(ctx, bufs.S, n_total, spec.percdamp, spec.act_order, bufs.R,
                                     bufs.perm, bufs.dead)
                 G.gptq_quantize_layer(ctx, W, bufs.R, bufs.perm if spec.act_order else None,
-                                      bufs.dead, spec.bits, spec.group, spec.block, False,
+                                      bufs.dead, spec.bits, spec.group, spec.block,
+                                      GRID_MODES[args.grid],
                                       bufs.scales, bufs.zeros, bufs.codes, bufs.W_hat,
                                       bufs.col_loss)
                 G.gptq_pack(ctx, bufs.codes, spec.bits, bufs.packed)
@@ -429,7 +445,7 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_tok, rows = min(131072, spec.n_tokens), min(3072, spec.m)
-        sample_s, full_s, desc = oracle_sample(spec, seed, n_tok, rows)
+        sample_s, full_s, desc = oracle_sample(spec, seed, n_tok, rows, args.grid)
         cpu = {"value": spec.m * spec.d / full_s, "unit": UNIT, "cores": cores_used(),
                "kind": "oracle", "sample": desc, "sample_seconds": sample_s}
 
@@ -439,7 +455,7 @@ def run_ours(args):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16 products, f32 accumulate/factor/quantize",
                 "data": "synthetic (seeded; workloads/synth.py)",
-                "config": workload_config(spec, args.chunk),
+                "config": workload_config(spec, args.chunk, args.grid),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
                 "gpu_launches": launches, "gpu_launches_per_step": launches / args.steps,
                 "step_ms_min": min(step_ms), "step_ms_max": max(step_ms)}

@@ -129,6 +129,13 @@ int gptq_prepare_hinv(gptq_ctx* ctx, float* S, int64_t n_total, int64_t d, float
  *            group j / g (the deployment metadata group_id[π_j] = j / g, from perm).  Needs
  *            group == 32 (with min(block, 128) a multiple of 32) or group == 128 (with
  *            block >= 128); otherwise ARG.
+ *            3: static groups with a symmetric grid (the pages name symmetric grids beside the
+ *            min-max fit, [T] §1.1): per (row, group) M = max |w| over the original columns,
+ *            Δ = 2M / (2^b - 1) (M = 0 -> Δ = 1), z = 2^(b-1); written to scales/zeros.
+ *            4: static groups with the ternary grid {-Δ, 0, +Δ} of the pages' extreme case
+ *            ([W] section "extreme quantization: 2-bit and ternary", used there with g = 8):
+ *            bits must be 2;
+ *            Δ = M (M = 0 -> Δ = 1), z = 1, and codes lie in 0..2 (2 bits each when packed).
  *   scales   [m, n_g] fp32, zeros [m, n_g] int32 (in or out, see grid_given).
  *   codes    [m, d] uint8 out, W_hat [m, d] fp32 out (= Δ (c - z)), col_loss [d] fp32 out
  *            (Σ_rows ρ² / (2 R_jj²), [T] eq.(43)); all in ORIGINAL column order.

@@ -88,9 +88,37 @@ def fit_grid(W, bits: int, group: int):
     return scale, zero
 
 
-def quantize(w, delta, zero, bits: int):
+def fit_grid_symmetric(W, maxq: int, group: int):
+    """Static symmetric grid per row or per (row, group of original columns): the grid is
+    centred on 0, the choice [T] §1.1 names beside the min-max fit ("real quantizers also
+    handle symmetric grids").  With maxq = 2 it is the ternary grid {-Δ, 0, +Δ} of [W]'s
+    section "extreme quantization: 2-bit and ternary".
+
+    Readings: M = max |w| over the group; Δ = 2M / maxq (so the codes span [-M, M]); M = 0 gives
+    Δ = 1; z = (maxq + 1) // 2 (= 2^(b-1) for maxq = 2^b - 1, 1 for the ternary grid).  fp32
+    arithmetic as in `fit_grid`.  Returns scale [m, n_g] float32 and zero [m, n_g] int32.
+    """
+    W32 = np.asarray(W, dtype=np.float32)
+    m, d = W32.shape
+    g = d if group == -1 else int(group)
+    ng = -(-d // g)
+    scale = np.empty((m, ng), np.float32)
+    zero = np.full((m, ng), (int(maxq) + 1) // 2, np.int32)
+    for k in range(ng):
+        M = np.abs(W32[:, k * g:min(d, (k + 1) * g)]).max(axis=1)
+        delta = ((np.float32(2.0) * M) / np.float32(maxq)).astype(np.float32)
+        scale[:, k] = np.where(M == 0, np.float32(1.0), delta)
+    return scale, zero
+
+
+def _code_max(bits: int, maxq=None) -> int:
+    """Largest code: 2^b - 1, unless a grid with fewer levels (the ternary grid: 2) is used."""
+    return int(2 ** bits - 1 if maxq is None else maxq)
+
+
+def quantize(w, delta, zero, bits: int, maxq=None):
     """Affine quantizer of [T] §1.1 / eq.(36): c = clip(round(w/Δ) + z, 0, 2^b - 1),
-    q = Δ (c - z).
+    q = Δ (c - z).  `maxq` replaces 2^b - 1 for a grid with fewer levels than 2^b.
 
     The decision is taken in fp32 (w rounded to fp32, IEEE fp32 division, round half to even);
     q is the fp32 product Δ (c - z), returned as fp64.  Returns (c int64, q fp64, u) where
@@ -99,17 +127,18 @@ def quantize(w, delta, zero, bits: int):
     w32 = np.asarray(w, dtype=np.float64).astype(np.float32)
     d32 = np.asarray(delta, dtype=np.float32)
     u = (w32 / d32).astype(np.float32)
-    c = np.clip(np.rint(u).astype(np.float64) + np.asarray(zero, np.float64), 0, 2 ** bits - 1)
+    c = np.clip(np.rint(u).astype(np.float64) + np.asarray(zero, np.float64), 0,
+                _code_max(bits, maxq))
     q = (d32 * (c - zero).astype(np.float32)).astype(np.float32)
     return c.astype(np.int64), q.astype(np.float64), u
 
 
-def quantize_rtn(W, scale, zero, bits: int, group: int):
+def quantize_rtn(W, scale, zero, bits: int, group: int, maxq=None):
     """Round-to-nearest of the original W on the same grid ([T] eq.(68) baseline)."""
     W = np.asarray(W, np.float64)
     m, d = W.shape
     gcol = _group_of_column(np.arange(d), d, group)
-    c, q, _ = quantize(W, scale[:, gcol], zero[:, gcol], bits)
+    c, q, _ = quantize(W, scale[:, gcol], zero[:, gcol], bits, maxq)
     return c, q
 
 
@@ -253,7 +282,7 @@ def dynamic_grid_arrays(m: int, d: int, dyn: int):
     return np.zeros((m, ng), np.float32), np.zeros((m, ng), np.int32)
 
 
-def gptq_explicit(Wp, G, scale, zero, gcol, bits: int, dynamic: int = 0):
+def gptq_explicit(Wp, G, scale, zero, gcol, bits: int, dynamic: int = 0, maxq=None):
     """Unblocked GPTQ with explicit inverse updates, column by column in processing order.
 
     For j = 0..d-1 over all rows at once (F = {j..d-1}): quantize column j ([T] eq.(36));
@@ -275,7 +304,7 @@ def gptq_explicit(Wp, G, scale, zero, gcol, bits: int, dynamic: int = 0):
     Rrows = np.zeros((d, d), np.float64)
     for j in range(d):
         _dynamic_refit(W, j, dynamic, bits, scale, zero)
-        c, q, _ = quantize(W[:, j], scale[:, gcol[j]], zero[:, gcol[j]], bits)
+        c, q, _ = quantize(W[:, j], scale[:, gcol[j]], zero[:, gcol[j]], bits, maxq)
         rho = W[:, j] - q
         gjj = G[j, j]
         loss[j] = float(np.sum(step_loss(G, j, rho)))
@@ -288,7 +317,7 @@ def gptq_explicit(Wp, G, scale, zero, gcol, bits: int, dynamic: int = 0):
     return codes, Q, loss, Rrows
 
 
-def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int, dynamic: int = 0):
+def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int, dynamic: int = 0, maxq=None):
     """GPTQ in Cholesky form with lazy block updates: [W] Algorithm 1 / [T] §10 pseudo-code.
 
     For each block [i, i2): for j in the block quantize column j, η = ρ / R_jj, record
@@ -311,7 +340,7 @@ def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int, dynamic: int = 0)
         E = np.zeros((m, i2 - i), np.float64)
         for j in range(i, i2):
             _dynamic_refit(W, j, dynamic, bits, scale, zero)
-            c, q, _ = quantize(W[:, j], scale[:, gcol[j]], zero[:, gcol[j]], bits)
+            c, q, _ = quantize(W[:, j], scale[:, gcol[j]], zero[:, gcol[j]], bits, maxq)
             rho = W[:, j] - q
             eta = rho / R[j, j]
             loss[j] = float(np.sum(rho ** 2)) / (2.0 * R[j, j] ** 2)
@@ -324,7 +353,7 @@ def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int, dynamic: int = 0)
 
 
 def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: float = 1e-3,
-                    dynamic: int = 0, other_zero=None):
+                    dynamic: int = 0, other_zero=None, maxq=None):
     """Check another implementation's codes against this recursion, decision by decision.
 
     Runs the unblocked Cholesky-form recursion ([T] eq.(42)) in fp64 on the same inputs, but at
@@ -351,7 +380,7 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
     R = np.asarray(R, np.float64)
     other = np.asarray(other_codes, np.int64)
     m, d = W.shape
-    maxq = 2 ** bits - 1
+    maxq = _code_max(bits, maxq)
     identical = in_band = violations = 0
     max_excess = 0.0
     Qr = np.zeros((m, d), np.float64)
@@ -378,7 +407,7 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
             zero[:, k] = z_g
         delta = np.asarray(scale[:, gcol[j]], np.float32)
         z = np.asarray(zero[:, gcol[j]], np.int64)
-        c_o, _, u = quantize(W[:, j], delta, z, bits)
+        c_o, _, u = quantize(W[:, j], delta, z, bits, maxq)
         c_g = other[:, j]
         same = c_o == c_g
         identical += int(np.sum(same))
@@ -411,7 +440,8 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
 # --------------------------------------------------------------------------------------------
 def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 0.01,
                act_order: bool = False, method: str = "explicit", grid=None,
-               eps: float = FP32_EPS, perm=None, dynamic: bool = False):
+               eps: float = FP32_EPS, perm=None, dynamic: bool = False,
+               grid_kind: str = "minmax"):
     """The layer-wise hot path of [T] §10, end to end on one layer.
 
     1. grid: fitted on the original W before anything else (static groups), unless given;
@@ -425,17 +455,27 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     returned scale / zero are indexed by processing group; group_id[π_j] = j // g maps each
     original column to its group ([T] §8.3, §8.4 table).
 
+    grid_kind (static groups): "minmax" (`fit_grid`), "symmetric" (`fit_grid_symmetric` with
+    maxq = 2^b - 1) or "ternary" (bits = 2, `fit_grid_symmetric` with maxq = 2, codes 0..2).
+
     Returns a dict with codes [m,d] int64, W_hat [m,d], scale, zero, col_loss [d], perm, dead,
-    lam, G, R, H_lambda, Wp (the permuted working copy fed to the recursion), gcol, group_id.
+    lam, G, R, H_lambda, Wp (the permuted working copy fed to the recursion), gcol, group_id,
+    maxq.
     """
     W = np.asarray(W, np.float64)
     m, d = W.shape
     if dynamic and group <= 0:
         raise ValueError("dynamic groups need group > 0")
+    if grid_kind not in ("minmax", "symmetric", "ternary") or (grid_kind == "ternary" and
+                                                                 bits != 2):
+        raise ValueError(f"grid_kind {grid_kind!r} with bits={bits}")
+    maxq = 2 if grid_kind == "ternary" else 2 ** bits - 1
     prep = prepare_with_retry(H, percdamp, act_order, eps, perm=perm)
     perm, dead = prep["perm"], prep["dead"]
     if dynamic:
         scale, zero = dynamic_grid_arrays(m, d, group)
+    elif grid is None and grid_kind != "minmax":
+        scale, zero = fit_grid_symmetric(W, maxq, group)
     elif grid is None:
         scale, zero = fit_grid(W, bits, group)
     else:
@@ -446,9 +486,11 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     dyn = int(group) if dynamic else 0
     gcol = np.arange(d) // dyn if dynamic else _group_of_column(perm, d, group)
     if method == "explicit":
-        codes_p, Q_p, loss_p, _ = gptq_explicit(Wp, prep["G"], scale, zero, gcol, bits, dyn)
+        codes_p, Q_p, loss_p, _ = gptq_explicit(Wp, prep["G"], scale, zero, gcol, bits, dyn,
+                                                maxq)
     elif method == "lazy":
-        codes_p, Q_p, loss_p = gptq_lazy(Wp, prep["R"], scale, zero, gcol, bits, block, dyn)
+        codes_p, Q_p, loss_p = gptq_lazy(Wp, prep["R"], scale, zero, gcol, bits, block, dyn,
+                                         maxq)
     else:
         raise ValueError(method)
     codes = np.empty_like(codes_p)
@@ -462,7 +504,7 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     return dict(codes=codes, W_hat=W_hat, scale=scale, zero=zero, col_loss=col_loss,
                 perm=perm, dead=dead, lam=prep["lam"], G=prep["G"], R=prep["R"],
                 H_lambda=prep["H_lambda"], retries=prep["retries"], Wp=Wp, gcol=gcol,
-                group_id=group_id)
+                group_id=group_id, maxq=maxq)
 
 
 def is_valid_act_order(perm, H, rtol: float = 1e-5) -> bool:

@@ -160,7 +160,8 @@ def gptq_prepare_hinv(ctx: Context, S, n_total: int, percdamp: float, act_order:
 def gptq_quantize_layer(ctx: Context, W, R, perm, dead, bits: int, group: int, block: int,
                         grid_given, scales, zeros, codes, W_hat, col_loss):
     """perm / dead may be None (identity order / no dead features).  grid_given: False / 0 fit a
-    static grid, True / 1 use the given one, 2 dynamic groups (see include/gptq.h)."""
+    static min-max grid, True / 1 use the given one, 2 dynamic groups, 3 fit a static symmetric
+    grid, 4 fit the static ternary grid (bits = 2); see include/gptq.h."""
     m, d = W.shape
     _dev(W, name="W")
     for t, dt, nm in ((R, torch.float32, "R"), (scales, torch.float32, "scales"),

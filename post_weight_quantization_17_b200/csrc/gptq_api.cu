@@ -195,7 +195,7 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   if (!W || !R || !scales || !zeros || !codes || !W_hat || !col_loss || !valid_dtype(w_dtype) ||
       m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || (long long)m * d > (1LL << 40) ||
       bits < 1 || bits > 8 || !(group == -1 || group > 0) || block < 1 || grid_given < 0 ||
-      grid_given > 2)
+      grid_given > 4 || (grid_given == 4 && bits != 2))
     GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "quantize_layer: bad argument (m=%lld d=%lld bits=%d group=%d block=%d)",
                  (long long)m, (long long)d, bits, group, block);
   // dynamic groups: a group is one 32-column sub-block or one 128-column block of the column
@@ -232,7 +232,10 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   const bool pair_ws = cv.ok();
   if (!pair_ws) Ehi = Elo = Rhi = Rlo = nullptr;
   int rc;
-  if (grid_given == 0 && (rc = gptq::grid_fit(c, W, w_dtype, mi, di, bits, group, scales, zeros)))
+  // largest code: 2^b - 1, or 2 for the ternary grid
+  const int maxq = (grid_given == 4) ? 2 : (1 << bits) - 1;
+  if ((grid_given == 0 || grid_given >= 3) &&
+      (rc = gptq::grid_fit(c, W, w_dtype, mi, di, maxq, grid_given >= 3, group, scales, zeros)))
     return rc;
   if ((rc = gptq::make_gcol(c, perm, di, group, dyn != 0, gcol, general ? inv : nullptr))) return rc;
   if ((rc = gptq::init_work(c, W, w_dtype, mi, di, perm, dead, !general, Wk))) return rc;
@@ -249,7 +252,7 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
       const bool uniform = dyn || (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
       float* Et = E + (i - s0);
       if ((rc = gptq::column_block(c, Wk, mi, di, i, nb, R, scales, zeros, ng, gcol, uniform,
-                                   dyn, bits, Et, Ehi ? Ehi + (i - s0) : nullptr,
+                                   dyn, maxq, Et, Ehi ? Ehi + (i - s0) : nullptr,
                                    Elo ? Elo + (i - s0) : nullptr, gptq::kSuperCols, codes_p,
                                    loss_part)))
         return rc;

@@ -15,15 +15,24 @@
 namespace gptq {
 
 // ------------------------------------------------------------------------------------------
-// a4: static min-max grid per (row, group of original columns), [T] §1.1 and §8.3.
-// One warp per (row, group); the range is extended to contain 0; fp32 arithmetic.
+// a4: static grid per (row, group of original columns), [T] §1.1 and §8.3: the min-max fit
+// (range extended to contain 0), or the symmetric fit around 0 (Δ = 2 max|w| / maxq,
+// z = (maxq + 1) / 2; maxq = 2 is the ternary grid).  fp32 arithmetic.
 template <class T>
-__device__ __forceinline__ void gridfit_finish(float mn, float mx, bool bad, int bits, int r,
-                                               float* scale, int32_t* zero, DeviceStatus* st) {
+__device__ __forceinline__ void gridfit_finish(float mn, float mx, bool bad, int maxq_i,
+                                               bool symmetric, int r, float* scale,
+                                               int32_t* zero, DeviceStatus* st) {
   if (bad) raise_error(st, GPTQ_ERR_NONFINITE, r);
-  const float maxq = (float)((1 << bits) - 1);
-  float delta = (mx == mn) ? 1.f : __fdiv_rn(__fsub_rn(mx, mn), maxq);
-  float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, delta)), 0.f), maxq);
+  const float maxq = (float)maxq_i;
+  float delta, z;
+  if (symmetric) {
+    const float M = fmaxf(-mn, mx);  // mn <= 0 <= mx
+    delta = (M == 0.f) ? 1.f : __fdiv_rn(2.f * M, maxq);
+    z = (float)((maxq_i + 1) / 2);
+  } else {
+    delta = (mx == mn) ? 1.f : __fdiv_rn(__fsub_rn(mx, mn), maxq);
+    z = fminf(fmaxf(rintf(__fdiv_rn(-mn, delta)), 0.f), maxq);
+  }
   *scale = delta;
   *zero = (int32_t)z;
 }
@@ -32,8 +41,8 @@ __device__ __forceinline__ void gridfit_finish(float mn, float mx, bool bad, int
 // loads its 4 elements of all 4 groups up front (8 bytes each) and the four reductions run
 // side by side.  Otherwise one warp per (row, group).
 template <class T>
-__global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, int bits,
-                          float* __restrict__ scales, int32_t* __restrict__ zeros,
+__global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, int maxq,
+                          bool symmetric, float* __restrict__ scales, int32_t* __restrict__ zeros,
                           DeviceStatus* st) {
   pdl_wait();
   pdl_release();
@@ -81,7 +90,7 @@ __global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, 
           b = mx[u];
         }
       const long long o = (long long)r * ng + k0 + lane;
-      gridfit_finish<T>(a, b, bad && lane == 0, bits, r, scales + o, zeros + o, st);
+      gridfit_finish<T>(a, b, bad && lane == 0, maxq, symmetric, r, scales + o, zeros + o, st);
     }
     return;
   }
@@ -103,12 +112,12 @@ __global__ void k_gridfit(const T* __restrict__ W, int m, int d, int g, int ng, 
   }
   bad = __any_sync(0xffffffffu, bad);
   if (lane == 0)
-    gridfit_finish<T>(mn, mx, bad, bits, r, scales + (long long)r * ng + k,
+    gridfit_finish<T>(mn, mx, bad, maxq, symmetric, r, scales + (long long)r * ng + k,
                       zeros + (long long)r * ng + k, st);
 }
 
-int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int group,
-             float* scales, int32_t* zeros) {
+int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int maxq, bool symmetric,
+             int group, float* scales, int32_t* zeros) {
   const int g = (group == -1) ? d : group;
   const int ng = (d + g - 1) / g;
   const bool quad = (g == 128) && (d % 512 == 0) && (w_dtype != GPTQ_F32) &&
@@ -116,13 +125,13 @@ int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int gro
   const long long warps = (long long)m * (quad ? ng / 4 : ng);
   const int blocks = (int)((warps * 32 + 255) / 256);
   if (w_dtype == GPTQ_F16)
-    GPTQ_LAUNCH(c, k_gridfit<__half>, blocks, 256, 0, (const __half*)W, m, d, g, ng, bits, scales,
+    GPTQ_LAUNCH(c, k_gridfit<__half>, blocks, 256, 0, (const __half*)W, m, d, g, ng, maxq, symmetric, scales,
                 zeros, c->status);
   else if (w_dtype == GPTQ_BF16)
     GPTQ_LAUNCH(c, k_gridfit<__nv_bfloat16>, blocks, 256, 0, (const __nv_bfloat16*)W, m, d, g, ng,
-                bits, scales, zeros, c->status);
+                maxq, symmetric, scales, zeros, c->status);
   else
-    GPTQ_LAUNCH(c, k_gridfit<float>, blocks, 256, 0, (const float*)W, m, d, g, ng, bits, scales,
+    GPTQ_LAUNCH(c, k_gridfit<float>, blocks, 256, 0, (const float*)W, m, d, g, ng, maxq, symmetric, scales,
                 zeros, c->status);
   return GPTQ_OK;
 }
@@ -426,7 +435,7 @@ template <bool UNIFORM>
 __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     float* __restrict__ Wk, int m, int d, int i, int nb, const float* __restrict__ R,
     float* __restrict__ scales, int32_t* __restrict__ zeros, int ng,
-    const int32_t* __restrict__ gcol, int dyn, int bits, float* __restrict__ E,
+    const int32_t* __restrict__ gcol, int dyn, int maxq, float* __restrict__ E,
     float* __restrict__ Ehi,
     float* __restrict__ Elo, int ldE, uint8_t* __restrict__ codes,
     float* __restrict__ loss_part) {
@@ -498,7 +507,7 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
   args.srow = (long long)(active ? row : 0) * ng;
   args.q = q; args.src0 = lane & ~(unsigned)(kColLanes - 1);
   args.active = active;
-  args.maxq = (float)((1 << bits) - 1);
+  args.maxq = (float)maxq;
   args.D0 = 1.f; args.Z0 = 0.f; args.Y0 = 1.f;
   bool fast = true;
   if (UNIFORM && dyn == 128) {
@@ -552,7 +561,7 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
 }
 
 int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R, float* scales,
-                 int32_t* zeros, int ng, const int32_t* gcol, bool uniform_grid, int dyn, int bits,
+                 int32_t* zeros, int ng, const int32_t* gcol, bool uniform_grid, int dyn, int maxq,
                  float* E, float* Ehi, float* Elo, int ldE, uint8_t* codes, float* loss_part) {
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_colblock<true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kColSmem));
@@ -561,10 +570,10 @@ int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
   const int blocks = (m + kColCtaRows - 1) / kColCtaRows;
   if (uniform_grid || dyn)
     GPTQ_LAUNCH(c, k_colblock<true>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales,
-                zeros, ng, gcol, dyn, bits, E, Ehi, Elo, ldE, codes, loss_part);
+                zeros, ng, gcol, dyn, maxq, E, Ehi, Elo, ldE, codes, loss_part);
   else
     GPTQ_LAUNCH(c, k_colblock<false>, blocks, 32 * kColWarps, kColSmem, Wk, m, d, i, nb, R, scales,
-                zeros, ng, gcol, 0, bits, E, Ehi, Elo, ldE, codes, loss_part);
+                zeros, ng, gcol, 0, maxq, E, Ehi, Elo, ldE, codes, loss_part);
   return GPTQ_OK;
 }
 

@@ -22,8 +22,8 @@ size_t factor_tmp_floats(int d);
 int factor_inverse(Ctx* c, float* M, int d, float* tmp);
 
 // ---- a4-a7 quantization
-int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int bits, int group,
-             float* scales, int32_t* zeros);
+int grid_fit(Ctx* c, const void* W, int w_dtype, int m, int d, int maxq, bool symmetric,
+             int group, float* scales, int32_t* zeros);
 // grid index of each processing position: static groups floor(π_j / g), dynamic groups j / g
 int make_gcol(Ctx* c, const int32_t* perm, int d, int group, bool dynamic, int32_t* gcol,
               int32_t* inv);
@@ -34,7 +34,7 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 // fits and writes to scales/zeros; 0: the grid is read from scales/zeros.
 int column_block(Ctx* c, float* Wk, int m, int d, int i, int nb, const float* R,
                  float* scales, int32_t* zeros, int ng, const int32_t* gcol,
-                 bool uniform_grid, int dyn, int bits, float* E, float* Ehi, float* Elo, int ldE,
+                 bool uniform_grid, int dyn, int maxq, float* E, float* Ehi, float* Elo, int ldE,
                  uint8_t* codes, float* loss_part);
 // Tail update on CTA pairs with operands split into tf32 halves (k_gemm_pair.cu):
 // C = alpha A B + beta C, A [M, K] (lda), B [K, N] (ldb), both row-major.

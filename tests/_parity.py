@@ -95,7 +95,8 @@ def check_hessian(gpu, Xt):
 TOL_DYN_SCALE = 1e-4
 
 
-def check_layer(gpu, Wn, H, spec, block=None, method="explicit", dynamic=False, grid=None):
+def check_layer(gpu, Wn, H, spec, block=None, method="explicit", dynamic=False, grid=None,
+                grid_kind="minmax"):
     """Oracle on the same H and W; returns a dict of the measured discrepancies after
     asserting the contract's tolerances.
 
@@ -112,7 +113,8 @@ def check_layer(gpu, Wn, H, spec, block=None, method="explicit", dynamic=False, 
     else:
         assert np.array_equal(perm_g, np.arange(H.shape[0]))
     o = O.gptq_layer(Wn, H, spec.bits, spec.group, block or spec.block, spec.percdamp,
-                     spec.act_order, method=method, perm=perm, dynamic=dynamic, grid=grid)
+                     spec.act_order, method=method, perm=perm, dynamic=dynamic, grid=grid,
+                     grid_kind=grid_kind)
     res = {}
     if not dynamic:
         # grid: bit-exact (both sides decide in fp32 on the same fp16 values)
@@ -138,7 +140,7 @@ def check_layer(gpu, Wn, H, spec, block=None, method="explicit", dynamic=False, 
         assert res["grid_scale_rel"] <= TOL_DYN_SCALE, res
     else:
         rep = O.decision_replay(o["Wp"], o["R"], o["scale"], o["zero"], o["gcol"], spec.bits,
-                                codes_p, band=BAND)
+                                codes_p, band=BAND, maxq=o["maxq"])
     res["identical"] = rep["identical"] / rep["n"]
     res["in_band"] = rep["in_band"]
     res["violations"] = rep["violations"]

@@ -93,6 +93,36 @@ def test_given_symmetric_grid_parity(ctx, act_order):
     print("given_grid", act_order, res)
 
 
+GRID_VARIANTS = [
+    # symmetric 4-bit g128 under act-order (grid_given = 3)
+    ("symmetric_4bit_g128", dataclasses.replace(
+        CONFIGS[2][0].scaled(160, 384, 3000, chunk=1024), act_order=True), 15, 3, "symmetric"),
+    # symmetric 3-bit per row, ragged
+    ("symmetric_3bit_row_ragged", LayerSpec("sym3", 77, 333, 1001, bits=3, group=-1, block=128,
+                                            act_order=False, x_kind="lowrank_t3", x_rank=40,
+                                            chunk=333), 16, 3, "symmetric"),
+    # the ternary grid at g = 8 (grid_given = 4), the extreme case of the results
+    ("ternary_g8", dataclasses.replace(
+        CONFIGS[5][1].scaled(130, 256, 2048, chunk=512), group=8), 17, 4, "ternary"),
+    ("ternary_g8_actorder_ragged", dataclasses.replace(
+        CONFIGS[3][0].scaled(61, 203, 1500, chunk=500), group=8, bits=2), 18, 4, "ternary"),
+]
+
+
+@pytest.mark.parametrize("name,spec,seed,mode,kind", GRID_VARIANTS,
+                         ids=[c[0] for c in GRID_VARIANTS])
+def test_grid_variants_parity(ctx, name, spec, seed, mode, kind):
+    """Symmetric and ternary static grids fitted on the GPU, then the same recursion."""
+    W, chunks = P.make_inputs(spec, seed)
+    gpu = P.gpu_run(ctx, spec, W, chunks, grid_given=mode)
+    if kind == "ternary":
+        assert gpu["codes"].max() <= 2 and np.all(gpu["zeros"] == 1)
+    Xt = torch.cat(chunks).cpu().double().numpy()
+    H, herr = P.check_hessian(gpu, Xt)
+    res = P.check_layer(gpu, P.to_np64(W), H, spec, grid_kind=kind)
+    print(name, f"H={herr:.2e}", {k: (f"{v:.2e}" if isinstance(v, float) else v) for k, v in res.items()})
+
+
 DYNAMIC = [
     # g = 128: one grid per kernel block, fitted from the staged block; ragged last group
     ("dyn128_qproj_shape", CONFIGS[2][0].scaled(160, 600, 3000, chunk=1024), 1, 128),
@@ -121,18 +151,21 @@ def test_dynamic_groups_parity(ctx, name, spec, seed, block):
     print(name, f"H={herr:.2e}", {k: (f"{v:.2e}" if isinstance(v, float) else v) for k, v in res.items()})
 
 
-def test_dynamic_groups_rejects_unsupported(ctx):
-    """Dynamic groups other than 32 / 128, or a group that a column block would split, are
-    argument errors reported by the library, not silently static."""
+def test_grid_modes_reject_unsupported(ctx):
+    """Dynamic groups other than 32 / 128, or a group that a column block would split, the
+    ternary grid with other than 2 bits, and unknown grid modes are argument errors reported by
+    the library, not silently another grid."""
     import post_weight_quantization_17_b200 as G
     spec = CONFIGS[2][0].scaled(64, 256, 512, chunk=512)
     W, chunks = P.make_inputs(spec, 3)
-    for group, block in ((64, 128), (128, 64), (32, 48)):
-        bufs = G.LayerBuffers(64, 256, 4, group, W.device)
+    for group, block, mode, bits in ((64, 128, 2, 4), (128, 64, 2, 4), (32, 48, 2, 4),
+                                     (8, 128, 4, 3), (8, 128, 4, 4), (128, 128, 5, 4),
+                                     (128, 128, -1, 4)):
+        bufs = G.LayerBuffers(64, 256, bits, group, W.device)
         bufs.R.copy_(torch.eye(256))
         with pytest.raises(RuntimeError):
-            G.gptq_quantize_layer(ctx, W, bufs.R, None, bufs.dead, 4, group, block, 2, bufs.scales,
-                                  bufs.zeros, bufs.codes, bufs.W_hat, bufs.col_loss)
+            G.gptq_quantize_layer(ctx, W, bufs.R, None, bufs.dead, bits, group, block, mode,
+                                  bufs.scales, bufs.zeros, bufs.codes, bufs.W_hat, bufs.col_loss)
 
 
 @pytest.mark.parametrize("d", [700, 257, 1000])

@@ -490,3 +490,82 @@ def test_dynamic_replay_zero_point_decisions():
     bad[1, 0] += 1 if bad[1, 0] < 15 else -1
     rep = replay(bad)
     assert rep["grid_violations"] == 1
+
+
+# ------------------------------------------------ grid variants ([T] §1.1, [W] extreme section)
+def test_symmetric_grid_worked_values():
+    """By hand: a group with max |w| = 0.3 under 4 bits has Δ = 0.6 / 15 = 0.04 and z = 8, so the
+    grid is 0.04·{-8..7}; 0.25 / 0.04 = 6.25 rounds to 6 (code 14, value 0.24), and -0.3 / 0.04
+    (just below -7.5 in fp32) rounds to -8 (code 0).  An all-zero group gets Δ = 1."""
+    W = np.array([[-0.3, 0.1, 0.25, 0.0], [0.0, 0.0, 0.0, 0.0]])
+    sc, ze = O.fit_grid_symmetric(W, 15, -1)
+    assert sc[0, 0] == np.float32(0.6) / np.float32(15) and ze[0, 0] == 8
+    assert sc[1, 0] == 1.0 and ze[1, 0] == 8
+    c, q, _ = O.quantize(W[0], sc[0, 0], ze[0, 0], 4)
+    assert list(c) == [0, 10, 14, 8]
+    assert np.allclose(q, [-0.32, 0.08, 0.24, 0.0], atol=1e-7)
+
+
+def test_ternary_grid_worked_values():
+    """The ternary grid of the extreme-quantization results: Δ = max |w|, z = 1, codes 0..2 in
+    2-bit storage, values {-Δ, 0, +Δ}.  w / Δ = 0.52 rounds to 1 (code 2); nothing reaches the
+    fourth 2-bit code."""
+    w = np.array([[0.5, -0.2, 0.1, -0.05, 0.0, 0.26, -0.5, 0.2]])
+    sc, ze = O.fit_grid_symmetric(w, 2, 8)
+    assert sc[0, 0] == np.float32(0.5) and ze[0, 0] == 1
+    c, q = O.quantize_rtn(w, sc, ze, 2, 8, maxq=2)
+    assert list(c[0]) == [2, 1, 1, 1, 1, 2, 0, 1]
+    assert set(np.unique(q)) <= {-0.5, 0.0, 0.5}
+    # without the level cap a 2-bit code could reach 3 = +2Δ
+    c3, _, _ = O.quantize(np.array([1.2]), np.float32(0.5), 1, 2)
+    c2, _, _ = O.quantize(np.array([1.2]), np.float32(0.5), 1, 2, maxq=2)
+    assert c3[0] == 3 and c2[0] == 2
+
+
+@pytest.mark.parametrize("kind,bits", [("symmetric", 4), ("symmetric", 3), ("ternary", 2)])
+def test_grid_variants_gptq_identities(kind, bits):
+    """The recursion's identities hold for the other grids: a diagonal H gives round-to-nearest
+    on the grid; lazy blocks give the unblocked result; codes stay within 0..maxq; Ŵ lies on
+    the grid."""
+    W, X = _layer(10, 32, 128, 27)
+    H = O.hessian(X)
+    g = 8
+    ref = O.gptq_layer(W, H, bits, g, method="explicit", act_order=True, grid_kind=kind)
+    maxq = ref["maxq"]
+    assert maxq == (2 if kind == "ternary" else 2 ** bits - 1)
+    sc, ze = O.fit_grid_symmetric(W, maxq, g)
+    assert np.array_equal(ref["scale"], sc) and np.array_equal(ref["zero"], ze)
+    assert ref["codes"].min() >= 0 and ref["codes"].max() <= maxq
+    gid = np.arange(32) // g
+    assert np.allclose(ref["W_hat"], sc[:, gid] * (ref["codes"] - ze[:, gid]), rtol=1e-6)
+    for block in (1, 5, 8, 32):
+        out = O.gptq_layer(W, H, bits, g, block=block, method="lazy", act_order=True,
+                           grid_kind=kind)
+        assert np.array_equal(out["codes"], ref["codes"]), block
+    dg = np.diag(np.linspace(2.0, 1.0, 32))
+    diag = O.gptq_layer(W, dg, bits, g, method="explicit", grid_kind=kind)
+    c, _ = O.quantize_rtn(W, sc, ze, bits, g, maxq=maxq)
+    assert np.array_equal(diag["codes"], c)
+    with pytest.raises(ValueError):
+        O.gptq_layer(W, H, 3, g, grid_kind="ternary")
+
+
+def test_ternary_brute_force_tiny():
+    """On a 1 x 4 layer the exhaustive search over the 3^4 ternary code vectors bounds the
+    GPTQ layer error from below, and at d = 1 GPTQ attains it (one column is plain rounding,
+    which is optimal for a single weight)."""
+    rng = np.random.default_rng(28)
+    W = rng.normal(0, 0.02, (1, 4))
+    X = rng.normal(0, 1, (4, 40))
+    H = O.hessian(X)
+    out = O.gptq_layer(W, H, 2, -1, method="explicit", grid_kind="ternary")
+    sc, ze = out["scale"][0, 0], out["zero"][0, 0]
+    best = min(O.layer_error(W, sc * (np.array(cs)[None, :] - ze), H)
+               for cs in np.ndindex(3, 3, 3, 3))
+    assert O.layer_error(W, out["W_hat"], H) >= best - 1e-15
+    W1 = W[:, :1]
+    H1 = H[:1, :1]
+    one = O.gptq_layer(W1, H1, 2, -1, method="explicit", grid_kind="ternary")
+    best1 = min(O.layer_error(W1, one["scale"][0, 0] * (np.array([[c]]) - 1), H1)
+                for c in range(3))
+    assert np.isclose(O.layer_error(W1, one["W_hat"], H1), best1, rtol=1e-12)
