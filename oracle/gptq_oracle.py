@@ -90,9 +90,9 @@ def fit_grid(W, bits: int, group: int):
 
 def fit_grid_symmetric(W, maxq: int, group: int):
     """Static symmetric grid per row or per (row, group of original columns): the grid is
-    centred on 0, the choice [T] §1.1 names beside the min-max fit ("real quantizers also
-    handle symmetric grids").  With maxq = 2 it is the ternary grid {-Δ, 0, +Δ} of [W]'s
-    section "extreme quantization: 2-bit and ternary".
+    centred on 0, which [T] §1.1 mentions beside the min-max fit as a choice real quantizers
+    make.  With maxq = 2 it is the ternary grid {-Δ, 0, +Δ} of [W]'s section on extreme
+    quantization (2-bit and ternary).
 
     Readings: M = max |w| over the group; Δ = 2M / maxq (so the codes span [-M, M]); M = 0 gives
     Δ = 1; z = (maxq + 1) // 2 (= 2^(b-1) for maxq = 2^b - 1, 1 for the ternary grid).  fp32
