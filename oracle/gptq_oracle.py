@@ -15,6 +15,9 @@ Sources, cited by page title and section / equation:
   [W]  "GPTQ 完全拆解：二阶信息驱动的权重量化，如何把 175B 模型塞进一张 A100"
        (pinghaoyang.com.cn walkthrough): OBS update and greedy criterion, toy example,
        Algorithm 1.
+  [A]  "什么是GPTQ（GPTQ）？一种面向生成式预训练 Transformer 的一次性权重量化方法"
+       (aiboss88.com wiki), section "工作机制" (how it works): at inference the 4-bit weights
+       are dequantized on the fly inside a fused kernel.
 
 Precision: fp64 everywhere, except where floating point decides an integer.  The grid fit
 (Δ, z) and each code decision c = clip(rint(w/Δ)+z) are taken in fp32 (IEEE division,
@@ -569,3 +572,30 @@ def unpack(packed, d: int, bits: int):
             bit = (packed[:, pos // 32] >> np.uint64(pos % 32)) & np.uint64(1)
             codes[:, k] |= (bit.astype(np.int64) << t)
     return codes
+
+
+# --------------------------------------------------------------------------------------------
+# Consumer of the packed format: the W4A16 product
+# --------------------------------------------------------------------------------------------
+def dequant_matmul(X, packed, d: int, bits: int, scale, zero, group: int, group_id=None):
+    """Y = X Ŵᵀ for 16-bit activations and the packed codes, the product a W4A16 layer computes
+    at inference ([T] §1.2: weights stored as codes, activations kept in FP16/BF16; [A] "how it
+    works": the codes are dequantized inside the fused kernel).
+
+    X [T, d] (token-major), packed [m, words] in the layout of `pack`, scale [m, n_g] fp32,
+    zero [m, n_g].  The weight is the quantizer's output Ŵ[r, k] = Δ[r, g(k)] (c[r, k] -
+    z[r, g(k)]) in fp32 ([T] eq.(36), §8.4), with g(k) = group_id[k] when given (dynamic groups
+    under act-order, [T] §8.4 table) else k // group (static groups; 0 for group = -1).
+    Returns Y [T, m] in fp64 (X and Ŵ taken exactly, products and sums in fp64).
+    """
+    codes = unpack(packed, d, bits)
+    if group_id is not None:
+        gid = np.asarray(group_id, np.int64)
+    elif group == -1:
+        gid = np.zeros(d, np.int64)
+    else:
+        gid = np.arange(d) // int(group)
+    sc = np.asarray(scale, np.float32)[:, gid]
+    ze = np.asarray(zero, np.int64)[:, gid]
+    W_hat = (sc * (codes - ze).astype(np.float32)).astype(np.float32)
+    return np.asarray(X, np.float64) @ W_hat.astype(np.float64).T

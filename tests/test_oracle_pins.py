@@ -569,3 +569,36 @@ def test_ternary_brute_force_tiny():
     best1 = min(O.layer_error(W1, one["scale"][0, 0] * (np.array([[c]]) - 1), H1)
                 for c in range(3))
     assert np.isclose(O.layer_error(W1, one["W_hat"], H1), best1, rtol=1e-12)
+
+
+# ------------------------------------------------------------- W4A16 consumer ([T] §1.2, [A])
+def test_dequant_matmul_worked_values():
+    """By hand: one row of 8 codes 0..7 packed at 4 bits is the word 0x76543210; with Δ = 0.5
+    and z = 3 the weights are 0.5·(c - 3) = -1.5, -1, ..., 2; against x = 1..8 the product is
+    Σ 0.5 (c - 3)(c + 1) = 0.5 (Σ c² - 2 Σ c - 3·8) = 0.5 (140 - 56 - 24) = 30."""
+    packed = np.array([[0x76543210]], np.uint64)
+    y = O.dequant_matmul(np.arange(1, 9, dtype=np.float64)[None, :], packed, 8, 4,
+                         np.array([[0.5]], np.float32), np.array([[3]]), -1)
+    assert y.shape == (1, 1) and y[0, 0] == 30.0
+
+
+@pytest.mark.parametrize("act_order,dynamic", [(False, False), (True, False), (True, True)])
+def test_dequant_matmul_reproduces_layer_output(act_order, dynamic):
+    """The packed codes with the layer's grid give back exactly X Ŵᵀ for the Ŵ that the
+    quantization returned (static groups indexed by original column; dynamic groups through
+    group_id), and at 16 bits of exact weights it is a plain matrix product."""
+    W, X = _layer(12, 64, 200, 29)
+    H = O.hessian(X)
+    g = 16
+    out = O.gptq_layer(W, H, 4, g, act_order=act_order, dynamic=dynamic, method="lazy",
+                       block=16)
+    packed = O.pack(out["codes"], 4)
+    Xa = np.random.default_rng(30).normal(size=(5, 64)).astype(np.float32).astype(np.float64)
+    y = O.dequant_matmul(Xa, packed, 64, 4, out["scale"], out["zero"], g,
+                         group_id=out["group_id"] if dynamic else None)
+    assert np.allclose(y, Xa @ out["W_hat"].T, rtol=0, atol=1e-12)
+    # an exact identity: Δ = 1, z = 0 and 8-bit codes are the integer matrix itself
+    C = np.random.default_rng(31).integers(0, 256, size=(7, 40))
+    y8 = O.dequant_matmul(Xa[:, :40], O.pack(C, 8), 40, 8, np.ones((7, 1), np.float32),
+                          np.zeros((7, 1), np.int64), -1)
+    assert np.array_equal(y8, Xa[:, :40] @ C.T.astype(np.float64))
