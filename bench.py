@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--grid", choices=sorted(GRID_MODES), default="static",
                     help="static groups (the default line) or dynamic groups (grid refitted per "
                          "processing group on the GPU)")
+    ap.add_argument("--w4a16", choices=["q_proj", "fc2"], default=None,
+                    help="instead of the quantization step, time the W4A16 product X Ŵᵀ over "
+                         "packed 4-bit g128 codes of this layer shape (one call = one step)")
+    ap.add_argument("--w4a16-tokens", type=int, default=1)
     ap.add_argument("--n-tokens", type=int, default=0,
                     help="calibration tokens (profiling captures only; the bench line uses all)")
     return ap.parse_args()
@@ -466,8 +470,75 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_w4a16(args):
+    """The consumer of the packed format on one GPU: Y [T, m] = X [T, d] Ŵᵀ with X bf16 and
+    random valid 4-bit codes (g = 128).  Small T is bound by reading the codes from HBM, large T
+    by the tensor cores; the line reports the bound that applies."""
+    import torch
+    import post_weight_quantization_17_b200 as G
+    m, d = {"q_proj": (4096, 4096), "fc2": (12288, 49152)}[args.w4a16]
+    T, g = args.w4a16_tokens, 128
+    torch.cuda.set_device(0)
+    gen = torch.Generator(device="cuda").manual_seed(1)
+    packed = torch.randint(-2 ** 31, 2 ** 31 - 1, (m, d // 8), dtype=torch.int32, device="cuda",
+                           generator=gen)
+    scales = torch.rand(m, d // g, device="cuda", generator=gen) * 0.02 + 1e-3
+    zeros = torch.randint(0, 16, (m, d // g), dtype=torch.int32, device="cuda", generator=gen)
+    X = torch.randn(T, d, device="cuda", generator=gen).to(torch.bfloat16)
+    Y = torch.empty(T, m, device="cuda")
+    ctx = G.Context(m_max=4096, d_max=4096, act_order=True)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        G.gptq_dequant_matmul(ctx, X, packed, d, 4, g, scales, zeros, Y)
+    G.gptq_sync_status(ctx)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    times = []
+    launches0 = G.gptq_kernel_launches(ctx)
+    for _ in range(args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        G.gptq_dequant_matmul(ctx, X, packed, d, 4, g, scales, zeros, Y)
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b) * 1e-3)
+    clk = clocks.stop()
+    launches = G.gptq_kernel_launches(ctx) - launches0
+    G.gptq_sync_status(ctx)
+    t = sum(times) / len(times)
+    tflops_peak, hbm_peak, src = measured_peaks()
+    nbytes = m * d // 2 + m * (d // g) * 8 + T * d * 2 + T * m * 4
+    flops = 2.0 * T * m * d
+    hbm_bound = nbytes / (hbm_peak * 1e9) >= flops / (tflops_peak * 1e12)
+    if hbm_bound:
+        ach = nbytes / t / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                "frac": ach / hbm_peak, "traffic": None, "peak_source": src}
+    else:
+        ach = flops / t / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": tflops_peak, "unit": "TFLOP/s",
+                "frac": ach / tflops_peak, "traffic": None, "peak_source": src}
+    line = {"metric": "W4A16 product X W_hat^T from packed 4-bit g128 codes, weights per second",
+            "value": m * d / t, "unit": "weights/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 X, exact (c - z), f32 accumulate",
+            "data": "synthetic (random valid codes, seeded)",
+            "config": {"workload": f"{args.w4a16} {m}x{d}, T={T} tokens", "m": m, "d": d, "T": T,
+                       "group": g, "l2": "flushed between timed calls (256 MiB write)"},
+            "roofline": roof, "clocks": clk, "gpu_launches": launches}
+    print(json.dumps(line), flush=True)
+    ctx.close()
+
+
 def main():
     args = parse()
+    if args.w4a16:
+        run_w4a16(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -183,6 +183,31 @@ int gptq_pack(gptq_ctx* ctx, const uint8_t* codes, int64_t m, int64_t d, int bit
 int gptq_unpack(gptq_ctx* ctx, const uint32_t* packed, int64_t m, int64_t d, int bits,
                 uint8_t* codes);
 
+/* The consumer of the packed format: Y = X Ŵᵀ, the product of a W4A16 linear layer at inference
+ * ([T] §1.2: codes stored, activations kept in FP16/BF16; [A] "how it works": the codes are
+ * dequantized on the fly inside the fused kernel), with Ŵ[r, k] = Δ[r, g(k)] (c[r, k] - z[r, g(k)])
+ * exactly as gptq_quantize_layer defines W_hat.
+ *   X        [T, d] of type x_dtype (GPTQ_BF16 / GPTQ_F16 / GPTQ_F32), token-major, device.
+ *   packed   [m, ceil(d bits / 32)] uint32 in gptq_pack's layout, device; bits 1..8.
+ *   group    -1 or > 0; group_id [d] int32 device or NULL.  NULL: column k uses grid column
+ *            k / group (0 for group -1), as static groups do; otherwise group_id[k] (dynamic
+ *            groups under act-order: group_id[π_j] = j / g).
+ *   n_g      grid columns per row (the row stride of scales / zeros); with group_id NULL it
+ *            must be at least ceil(d / group) (1 for group -1).
+ *   scales   [m, n_g] fp32, zeros [m, n_g] int32, device; on the tensor path the zeros
+ *            must lie in 0..15 (any 4-bit grid does), else ARG via gptq_sync_status.
+ *   Y        [T, m] fp32 out (token-major), device.  T <= 524280.
+ * 4-bit codes with 16-bit X (d % 32 == 0, X and packed 16-byte aligned, group -1 or a multiple
+ * of 128, group_id NULL) run on the tensor cores: (c - z) is exact in X's 16-bit type and each
+ * 128-column partial sum is scaled by its Δ in fp32.  Every other case runs on CUDA cores.
+ * Split-K partials use the context workspace (T m per split, fp32); with too little workspace
+ * the product runs unsplit.  Asynchronous.  Errors: ARG (also a group_id entry outside
+ * [0, n_g), reported via gptq_sync_status), CUDA, TIMEOUT via gptq_sync_status. */
+int gptq_dequant_matmul(gptq_ctx* ctx, const void* X, int x_dtype, int64_t T, int64_t d,
+                        const uint32_t* packed, int64_t m, int bits, int group,
+                        const int32_t* group_id, int64_t n_g, const float* scales,
+                        const int32_t* zeros, float* Y);
+
 #ifdef __cplusplus
 }
 #endif

@@ -56,6 +56,8 @@ _SIGS = {
                                            _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "gptq_pack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
     "gptq_unpack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
+    "gptq_dequant_matmul": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _i64, _i32, _i32, _vp, _i64,
+                                   _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)  # AttributeError here means the library lacks a declared symbol
@@ -203,6 +205,24 @@ def gptq_unpack(ctx: Context, packed, d: int, bits: int, codes):
     _dev(packed, torch.int32, "packed")
     rc = _lib.gptq_unpack(ctx.handle, _ptr(packed), m, d, bits, _ptr(codes))
     ctx.check(rc, "gptq_unpack")
+
+
+def gptq_dequant_matmul(ctx: Context, X, packed, d: int, bits: int, group: int, scales, zeros,
+                        Y, group_id=None):
+    """Y [T, m] = X [T, d] Ŵᵀ from the packed codes (the W4A16 product; see include/gptq.h).
+    group_id: per-column grid index [d] int32 (dynamic groups under act-order) or None."""
+    T = X.shape[0]
+    m = packed.shape[0]
+    _dev(X, name="X")
+    for t, dt, nm in ((packed, torch.int32, "packed"), (scales, torch.float32, "scales"),
+                      (zeros, torch.int32, "zeros"), (Y, torch.float32, "Y")):
+        _dev(t, dt, nm)
+    if group_id is not None:
+        _dev(group_id, torch.int32, "group_id")
+    rc = _lib.gptq_dequant_matmul(ctx.handle, _ptr(X), _DTYPE_CODE[X.dtype], T, d, _ptr(packed),
+                                  m, bits, group, _ptr(group_id), scales.shape[1], _ptr(scales),
+                                  _ptr(zeros), _ptr(Y))
+    ctx.check(rc, "gptq_dequant_matmul")
 
 
 def words_per_row(d: int, bits: int) -> int:

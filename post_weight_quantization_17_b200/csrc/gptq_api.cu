@@ -297,4 +297,25 @@ int gptq_unpack(gptq_ctx* h, const uint32_t* packed, int64_t m, int64_t d, int b
   return gptq::unpack_codes(c, packed, (int)m, (int)d, bits, codes);
 }
 
+int gptq_dequant_matmul(gptq_ctx* h, const void* X, int x_dtype, int64_t T, int64_t d,
+                        const uint32_t* packed, int64_t m, int bits, int group,
+                        const int32_t* group_id, int64_t n_g, const float* scales,
+                        const int32_t* zeros, float* Y) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!X || !packed || !scales || !zeros || !Y || !valid_dtype(x_dtype) || T < 1 || d < 1 ||
+      m < 1 || T > 65535LL * 8 || d > INT32_MAX || m > INT32_MAX || bits < 1 || bits > 8 ||
+      !(group == -1 || group > 0) || n_g < 1 || n_g > INT32_MAX ||
+      (!group_id && n_g < (group == -1 ? 1 : (d + group - 1) / group)))
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "dequant_matmul: bad argument (T=%lld d=%lld m=%lld bits=%d group=%d n_g=%lld)",
+                 (long long)T, (long long)d, (long long)m, bits, group, (long long)n_g);
+  Carver cv(c);
+  const size_t avail = (c->ws_bytes > gptq::kStatusBytes + 256)
+                            ? (c->ws_bytes - gptq::kStatusBytes - 256) / 4
+                            : 0;
+  float* part = cv.take<float>(0);
+  return gptq::dequant_matmul(c, X, x_dtype, (int)T, (int)d, packed, (int)m, bits, group,
+                              group_id, (int)n_g, scales, zeros, Y, part, avail);
+}
+
 }  // extern "C"

@@ -56,6 +56,14 @@ int unpermute(Ctx* c, int m, int d, const int32_t* inv, const uint8_t* codes_p,
 int pack_codes(Ctx* c, const uint8_t* codes, int m, int d, int bits, uint32_t* packed);
 int unpack_codes(Ctx* c, const uint32_t* packed, int m, int d, int bits, uint8_t* codes);
 
+// ---- the W4A16 consumer of the packed codes (k_dqmm.cu): Y [T, m] = X [T, d] Ŵᵀ
+bool dequant_matmul_tc_applies(const void* X, int x_dtype, int d, const uint32_t* packed,
+                               int bits, int group, const int32_t* group_id);
+int dequant_matmul(Ctx* c, const void* X, int x_dtype, int T, int d, const uint32_t* packed,
+                   int m, int bits, int group, const int32_t* group_id, int ng,
+                   const float* scales, const int32_t* zeros, float* Y, float* part_ws,
+                   size_t part_floats);
+
 constexpr int kColRows = 32;      // rows per column-block CTA (8 warps, 8 lanes per row)
 constexpr int kColMax = 128;      // columns per kernel block
 constexpr int kSuperCols = 512;   // columns per super-block of the two-level lazy update
