@@ -106,6 +106,30 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// As mbar_wait, but each try suspends the thread in hardware (up to `hint_ns`) until the phase
+// completes, instead of returning at once: waiting warps then take no issue slots from the
+// warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(tc::smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, long long budget) {
+  if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_hint(bar, parity, 20000u)) {
+    if (clock64() - t0 > budget) return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -202,7 +226,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
       for (int j = 0; j < nst && !*abort_flag; ++j) {
         const int s = j % Cfg::CST;
         const uint32_t ph = (uint32_t)(j / Cfg::CST) & 1u;
-        if (!tc::mbar_wait_sleep(&empty_c[s], ph ^ 1u, budget)) {
+        if (!mbar_wait_sleep(&empty_c[s], ph ^ 1u, budget)) {
           raise_error(st, GPTQ_ERR_TIMEOUT, 41);
           *abort_flag = 1;
           break;
@@ -216,7 +240,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
         issued = j + 1;
       }
       for (int j = max(0, issued - Cfg::CST); j < issued; ++j)
-        if (!tc::mbar_wait_sleep(&full_c[j % Cfg::CST], (uint32_t)(j / Cfg::CST) & 1u, budget))
+        if (!mbar_wait_sleep(&full_c[j % Cfg::CST], (uint32_t)(j / Cfg::CST) & 1u, budget))
           raise_error(st, GPTQ_ERR_TIMEOUT, 42);
     }
   } else if (warp == 2) {
@@ -226,7 +250,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
       for (int i = 0; i < n && !*abort_flag; ++i) {
         const int s = i % Cfg::XST;
         const uint32_t ph = (uint32_t)(i / Cfg::XST) & 1u;
-        if (!tc::mbar_wait_sleep(&empty_x[s], ph ^ 1u, budget)) {
+        if (!mbar_wait_sleep(&empty_x[s], ph ^ 1u, budget)) {
           raise_error(st, GPTQ_ERR_TIMEOUT, 47);
           *abort_flag = 1;
           break;
@@ -239,7 +263,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
         issued = i + 1;
       }
       for (int i = max(0, issued - Cfg::XST); i < issued; ++i)
-        if (!tc::mbar_wait_sleep(&full_x[i % Cfg::XST], (uint32_t)(i / Cfg::XST) & 1u, budget))
+        if (!mbar_wait_sleep(&full_x[i % Cfg::XST], (uint32_t)(i / Cfg::XST) & 1u, budget))
           raise_error(st, GPTQ_ERR_TIMEOUT, 48);
     }
   } else if (warp == 1) {
@@ -249,8 +273,8 @@ __global__ void __launch_bounds__(DQ_THREADS)
         const int s = i % Cfg::XST, a = i % DQ_NA, b = i % Cfg::ND;
         const uint32_t ph = (uint32_t)(i / Cfg::XST) & 1u;
         const uint32_t aph = (uint32_t)(i / DQ_NA) & 1u, dph = (uint32_t)(i / Cfg::ND) & 1u;
-        if (!tc::mbar_wait_sleep(&d_empty[b], dph ^ 1u, budget) ||
-            !tc::mbar_wait_sleep(&a_full[a], aph, budget) || !tc::mbar_wait_sleep(&full_x[s], ph, budget)) {
+        if (!mbar_wait_sleep(&d_empty[b], dph ^ 1u, budget) ||
+            !mbar_wait_sleep(&a_full[a], aph, budget) || !mbar_wait_sleep(&full_x[s], ph, budget)) {
           raise_error(st, GPTQ_ERR_TIMEOUT, 43);
           *abort_flag = 1;
           break;
@@ -299,7 +323,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
         const uint16_t u = *reinterpret_cast<const uint16_t*>(&hz);
         zz = (uint32_t)u | ((uint32_t)u << 16);
       }
-      if (within == 0 && !tc::mbar_wait_sleep(&full_c[cs], cph, budget)) {
+      if (within == 0 && !mbar_wait_sleep(&full_c[cs], cph, budget)) {
         raise_error(st, GPTQ_ERR_TIMEOUT, 44);
         *abort_flag = 1;
         break;
@@ -317,7 +341,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
         if (lane == 0) tc::mbar_arrive(&empty_c[cs]);
       }
       // A buffer a was last read by the MMAs of step i - 4
-      if (i >= DQ_NA && !tc::mbar_wait_sleep(&a_free[a], aph ^ 1u, budget)) {
+      if (i >= DQ_NA && !mbar_wait_sleep(&a_free[a], aph ^ 1u, budget)) {
         raise_error(st, GPTQ_ERR_TIMEOUT, 45);
         *abort_flag = 1;
         break;
@@ -358,7 +382,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
       const float delta = delta_next;
       if (active && i + 1 < n)
         delta_next = srow[p.group_steps ? (k_begin + i + 1) / p.group_steps : 0];
-      if (!tc::mbar_wait_sleep(&d_full[b], dph, budget)) {
+      if (!mbar_wait_sleep(&d_full[b], dph, budget)) {
         raise_error(st, GPTQ_ERR_TIMEOUT, 46);
         *abort_flag = 1;
         ok = false;
