@@ -178,6 +178,36 @@ def gptq2d_lazy(X, GA, GB, w: int):
     return Z, eta
 
 
+def gptq2d_replay(X, GA, GB, other_Z, band: float = 1e-3):
+    """Check another implementation's rounding against the buffered recursion, cell by cell in
+    anti-diagonal order, following the other's decisions.  A differing integer is accepted iff it
+    is adjacent to this recursion's and the pre-round value lies within `band` of the rounding
+    boundary between the two (the decision is taken in another precision); anything else is a
+    violation.  Returns dict(n, identical, in_band, violations, eta) with the scaled residuals
+    of the followed decisions."""
+    Y = np.array(X, np.float64, copy=True)
+    m, n = Y.shape
+    other = np.asarray(other_Z, np.float64)
+    RA, RB = factor_upper_inverse(GA), factor_upper_inverse(GB)
+    eta = np.zeros((m, n))
+    C = np.zeros((m, n))
+    identical = in_band = violations = 0
+    for i, j in antidiagonal_order(m, n):
+        z_o = np.rint(Y[i, j])
+        z_g = other[i, j]
+        if z_o == z_g:
+            identical += 1
+        elif abs(z_o - z_g) == 1 and abs(Y[i, j] - (min(z_o, z_g) + 0.5)) <= band:
+            in_band += 1
+        else:
+            violations += 1
+        eta[i, j] = (Y[i, j] - z_g) / (RA[i, i] * RB[j, j])
+        C[i:, j] += eta[i, j] * RA[i, i:]
+        Y[i + 1:, j] -= eta[i, j] * RA[i, i + 1:] * RB[j, j]
+        Y[i, j + 1:] -= C[i, j] * RB[j, j + 1:]
+    return dict(n=m * n, identical=identical, in_band=in_band, violations=violations, eta=eta)
+
+
 def to_skewed(X, fill=0.0):
     """The skewed layout of [D] "存储也要讲究": S[s, j] = X[s - j, j], one row per anti-diagonal
     s = i + j (shape [m + n - 1, n]); a column of X is a vertical run, a row of X a diagonal of

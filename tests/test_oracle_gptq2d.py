@@ -167,3 +167,21 @@ def test_skewed_layout():
         cells = [(i, s - i) for i in range(m) if 0 <= s - i < n]
         assert sorted(S[s][S[s] != 0]) == sorted(X[i, j] for i, j in cells)
     assert np.array_equal(D.from_skewed(S, m, n), X)
+
+
+def test_replay_accepts_self_and_catches_a_planted_mistake():
+    """The replay follows the given decisions: the recursion's own result is all identical; an
+    integer moved by one away from any boundary is a violation; a value exactly on a rounding
+    boundary (x = 0.5 in a 1 x 1 problem) accepts both neighbours."""
+    X, GA, GB = _problem(5, 4, 16)
+    Z, eta, _ = D.gptq2d_buffered(X, GA, GB)
+    rep = D.gptq2d_replay(X, GA, GB, Z)
+    assert rep["identical"] == 20 and rep["violations"] == 0
+    assert np.allclose(rep["eta"], eta, atol=1e-12)
+    Y0 = X[0, 0]  # the first cell's pre-round value is X itself
+    bad = Z.copy()
+    bad[0, 0] += 1 if Y0 - np.rint(Y0) < 0.4 else -1
+    assert abs(abs(Y0 - np.rint(Y0)) - 0.5) > 0.05  # the planted move is far from a tie
+    assert D.gptq2d_replay(X, GA, GB, bad)["violations"] >= 1
+    one = D.gptq2d_replay(np.array([[0.5]]), np.eye(1), np.eye(1), np.array([[1.0]]))
+    assert one["in_band"] == 1 and one["violations"] == 0
