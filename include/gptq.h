@@ -208,6 +208,28 @@ int gptq_dequant_matmul(gptq_ctx* ctx, const void* X, int x_dtype, int64_t T, in
                         const int32_t* group_id, int64_t n_g, const float* scales,
                         const int32_t* zeros, float* Y);
 
+/* Two-sided rounding (GPTQ-2D, [D] "GPTQ-2D：把一个"四次方"难题压回"三次方"的故事"): X [m, n] is
+ * rounded to an integer matrix Z for the metric ||A (Z - X) B||^2, given the metric factors
+ * G_A = A^T A (m x m) and G_B = B B^T (n x n).  First each factor is turned in place into the
+ * upper-triangular R with R^T R = G^{-1} (the reverse Cholesky and triangular inverse of
+ * gptq_prepare_hinv, without damping):
+ *   G        [k, k] fp32 symmetric positive definite, device; on return its upper triangle is R
+ *            and its strict lower triangle is zero.
+ * Synchronizes the stream.  Errors: ARG, NOMEM (workspace), NOT_PD, CUDA. */
+int gptq_twosided_factor(gptq_ctx* ctx, float* G, int64_t k);
+
+/* Then the rounding: the buffered row / column push of [D] (its Algorithm 3) over anti-diagonal
+ * wavefronts (its Theorem 1), equal in exact arithmetic to one-dimensional GPTQ on the
+ * vectorized problem with the Kronecker metric G_A ⊗ G_B:
+ *   X        [m, n] fp32 row-major, device, not modified.
+ *   RA       [m, m] and RB [n, n] from gptq_twosided_factor (row-major), device.
+ *   Z        [m, n] fp32 out: the integers (round half to even of the compensated value).
+ *   eta      [m, n] fp32 out: the scaled residuals η = (y - z) / (RA_ii RB_jj), whose squares
+ *            sum to ||A (Z - X) B||^2.
+ * Workspace: 2 m n fp32.  Asynchronous.  Errors: ARG, NOMEM, CUDA. */
+int gptq_twosided_round(gptq_ctx* ctx, const float* X, int64_t m, int64_t n, const float* RA,
+                        const float* RB, float* Z, float* eta);
+
 #ifdef __cplusplus
 }
 #endif

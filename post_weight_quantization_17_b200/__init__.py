@@ -58,6 +58,8 @@ _SIGS = {
     "gptq_unpack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
     "gptq_dequant_matmul": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _i64, _i32, _i32, _vp, _i64,
                                    _vp, _vp, _vp]),
+    "gptq_twosided_factor": (_i32, [_vp, _vp, _i64]),
+    "gptq_twosided_round": (_i32, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)  # AttributeError here means the library lacks a declared symbol
@@ -223,6 +225,22 @@ def gptq_dequant_matmul(ctx: Context, X, packed, d: int, bits: int, group: int, 
                                   m, bits, group, _ptr(group_id), scales.shape[1], _ptr(scales),
                                   _ptr(zeros), _ptr(Y))
     ctx.check(rc, "gptq_dequant_matmul")
+
+
+def gptq_twosided_factor(ctx: Context, G):
+    """In place: G [k, k] fp32 (symmetric positive definite) -> R upper with R^T R = G^-1."""
+    _dev(G, torch.float32, "G")
+    ctx.check(_lib.gptq_twosided_factor(ctx.handle, _ptr(G), G.shape[0]), "gptq_twosided_factor")
+
+
+def gptq_twosided_round(ctx: Context, X, RA, RB, Z, eta):
+    """Two-sided GPTQ rounding of X [m, n] with the factors from gptq_twosided_factor; writes the
+    integers Z and the scaled residuals eta (see include/gptq.h)."""
+    m, n = X.shape
+    for t, nm in ((X, "X"), (RA, "RA"), (RB, "RB"), (Z, "Z"), (eta, "eta")):
+        _dev(t, torch.float32, nm)
+    ctx.check(_lib.gptq_twosided_round(ctx.handle, _ptr(X), m, n, _ptr(RA), _ptr(RB), _ptr(Z),
+                                       _ptr(eta)), "gptq_twosided_round")
 
 
 def words_per_row(d: int, bits: int) -> int:

@@ -318,4 +318,40 @@ int gptq_dequant_matmul(gptq_ctx* h, const void* X, int x_dtype, int64_t T, int6
                               group_id, (int)n_g, scales, zeros, Y, part, avail);
 }
 
+int gptq_twosided_factor(gptq_ctx* h, float* G, int64_t k) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!G || k < 1 || k > 65535)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "twosided_factor: bad argument (k=%lld)", (long long)k);
+  Carver cv(c);
+  float* tmp = cv.take<float>(gptq::factor_tmp_floats((int)k));
+  if (!cv.ok())
+    GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "twosided_factor: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
+  int rc;
+  if ((rc = gptq::factor_inverse(c, G, (int)k, tmp))) return rc;
+  gptq::DeviceStatus st{};
+  if ((rc = read_status(c, &st))) return rc;
+  if (st.code == 0) return GPTQ_OK;
+  if ((rc = clear_status(c))) return rc;
+  if (st.code == GPTQ_ERR_NOT_PD)
+    GPTQ_SET_ERR(c, GPTQ_ERR_NOT_PD, "twosided_factor: G not positive definite");
+  c->last_error = "twosided_factor: device status " + std::to_string(st.code);
+  return st.code;
+}
+
+int gptq_twosided_round(gptq_ctx* h, const float* X, int64_t m, int64_t n, const float* RA,
+                        const float* RB, float* Z, float* eta) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  if (!X || !RA || !RB || !Z || !eta || m < 1 || n < 1 || m > 65535 || n > 65535)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "twosided_round: bad argument (m=%lld n=%lld)", (long long)m,
+                 (long long)n);
+  Carver cv(c);
+  float* Y = cv.take<float>((size_t)m * n);
+  float* C = cv.take<float>((size_t)m * n);
+  if (!cv.ok())
+    GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "twosided_round: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
+  return gptq::twosided_round(c, X, (int)m, (int)n, RA, RB, Z, eta, Y, C);
+}
+
 }  // extern "C"
