@@ -226,7 +226,9 @@ int gptq_twosided_factor(gptq_ctx* ctx, float* G, int64_t k);
  *   Z        [m, n] fp32 out: the integers (round half to even of the compensated value).
  *   eta      [m, n] fp32 out: the scaled residuals η = (y - z) / (RA_ii RB_jj), whose squares
  *            sum to ||A (Z - X) B||^2.
- * Workspace: 2 m n fp32.  Asynchronous.  Errors: ARG, NOMEM, CUDA. */
+ * Runs as a wavefront of 64 x 64 tiles: the cells of a tile in shared memory, the effects
+ * between tiles as GEMMs.  Workspace: 3 m n + m^2 fp32.  Asynchronous.  Errors: ARG, NOMEM,
+ * CUDA. */
 int gptq_twosided_round(gptq_ctx* ctx, const float* X, int64_t m, int64_t n, const float* RA,
                         const float* RB, float* Z, float* eta);
 

@@ -349,9 +349,11 @@ int gptq_twosided_round(gptq_ctx* h, const float* X, int64_t m, int64_t n, const
   Carver cv(c);
   float* Y = cv.take<float>((size_t)m * n);
   float* C = cv.take<float>((size_t)m * n);
+  float* etas = cv.take<float>((size_t)m * n);
+  float* RAT = cv.take<float>((size_t)m * m);
   if (!cv.ok())
     GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "twosided_round: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
-  return gptq::twosided_round(c, X, (int)m, (int)n, RA, RB, Z, eta, Y, C);
+  return gptq::twosided_round(c, X, (int)m, (int)n, RA, RB, Z, eta, Y, C, etas, RAT);
 }
 
 }  // extern "C"

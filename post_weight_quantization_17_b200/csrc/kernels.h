@@ -64,9 +64,10 @@ int dequant_matmul(Ctx* c, const void* X, int x_dtype, int T, int d, const uint3
                    const float* scales, const int32_t* zeros, float* Y, float* part_ws,
                    size_t part_floats);
 
-// ---- two-sided rounding (GPTQ-2D, k_twosided.cu); Y and C: m n floats of workspace each
+// ---- two-sided rounding (GPTQ-2D, k_twosided.cu); workspace: Y, C, etas (m n floats each) and
+// RAT (m m floats)
 int twosided_round(Ctx* c, const float* X, int m, int n, const float* RA, const float* RB,
-                   float* Z, float* eta, float* Y, float* C);
+                   float* Z, float* eta, float* Y, float* C, float* etas, float* RAT);
 
 constexpr int kColRows = 32;      // rows per column-block CTA (8 warps, 8 lanes per row)
 constexpr int kColMax = 128;      // columns per kernel block
