@@ -602,3 +602,20 @@ def test_dequant_matmul_reproduces_layer_output(act_order, dynamic):
     y8 = O.dequant_matmul(Xa[:, :40], O.pack(C, 8), 40, 8, np.ones((7, 1), np.float32),
                           np.zeros((7, 1), np.int64), -1)
     assert np.array_equal(y8, Xa[:, :40] @ C.T.astype(np.float64))
+
+
+@pytest.mark.parametrize("bits,group", [(3, 16), (2, 8), (4, -1), (5, 12)])
+def test_dequant_matmul_other_widths(bits, group):
+    """Codes that straddle 32-bit words (3 and 5 bits) and narrow groups: the product over the
+    packed words equals the product over the unpacked code matrix formed directly."""
+    rng = np.random.default_rng(32 + bits)
+    m, d, T = 9, 70, 4
+    codes = rng.integers(0, 2 ** bits, size=(m, d))
+    ng = 1 if group == -1 else -(-d // group)
+    sc = rng.uniform(0.01, 0.1, (m, ng)).astype(np.float32)
+    ze = rng.integers(0, 2 ** bits, (m, ng))
+    X = rng.normal(size=(T, d))
+    gid = np.zeros(d, np.int64) if group == -1 else np.arange(d) // group
+    W_hat = (sc[:, gid] * (codes - ze[:, gid]).astype(np.float32)).astype(np.float32)
+    y = O.dequant_matmul(X, O.pack(codes, bits), d, bits, sc, ze, group)
+    assert np.allclose(y, X @ W_hat.astype(np.float64).T, rtol=0, atol=1e-12)
