@@ -53,6 +53,9 @@ def parse():
                     help="instead of the quantization step, time the W4A16 product X Ŵᵀ over "
                          "packed 4-bit g128 codes of this layer shape (one call = one step)")
     ap.add_argument("--w4a16-tokens", type=int, default=1)
+    ap.add_argument("--w4a16-layout", choices=["rows", "tiles"], default="rows",
+                    help="codes in gptq_pack's row layout, or re-laid into 16 KB tiles first "
+                         "(gptq_retile_codes, outside the timed region)")
     ap.add_argument("--n-tokens", type=int, default=0,
                     help="calibration tokens (profiling captures only; the bench line uses all)")
     return ap.parse_args()
@@ -489,8 +492,17 @@ def run_w4a16(args):
     ctx = G.Context(m_max=4096, d_max=4096, act_order=True)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
+    if args.w4a16_layout == "tiles":
+        tiled = torch.empty(G.gptq_tiled_words(m, d), dtype=torch.int32, device="cuda")
+        G.gptq_retile_codes(ctx, packed, d, tiled)
+
+        def product():
+            G.gptq_dequant_matmul_tiled(ctx, X, tiled, m, g, scales, zeros, Y)
+    else:
+        def product():
+            G.gptq_dequant_matmul(ctx, X, packed, d, 4, g, scales, zeros, Y)
     for _ in range(max(3, args.warmup)):
-        G.gptq_dequant_matmul(ctx, X, packed, d, 4, g, scales, zeros, Y)
+        product()
     G.gptq_sync_status(ctx)
     torch.cuda.synchronize()
     clocks = ClockSampler(0)
@@ -502,7 +514,7 @@ def run_w4a16(args):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        G.gptq_dequant_matmul(ctx, X, packed, d, 4, g, scales, zeros, Y)
+        product()
         b.record(stream)
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b) * 1e-3)
@@ -527,7 +539,8 @@ def run_w4a16(args):
             "warmup": max(3, args.warmup), "ms_per_step": t * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 X, exact (c - z), f32 accumulate",
             "data": "synthetic (random valid codes, seeded)",
-            "config": {"workload": f"{args.w4a16} {m}x{d}, T={T} tokens", "m": m, "d": d, "T": T,
+            "config": {"workload": f"{args.w4a16} {m}x{d}, T={T} tokens, {args.w4a16_layout} "
+                                   "layout", "m": m, "d": d, "T": T, "layout": args.w4a16_layout,
                        "group": g, "l2": "flushed between timed calls (256 MiB write)"},
             "roofline": roof, "clocks": clk, "gpu_launches": launches}
     print(json.dumps(line), flush=True)

@@ -208,6 +208,28 @@ int gptq_dequant_matmul(gptq_ctx* ctx, const void* X, int x_dtype, int64_t T, in
                         const int32_t* group_id, int64_t n_g, const float* scales,
                         const int32_t* zeros, float* Y);
 
+/* A tile-contiguous copy of 4-bit packed codes for gptq_dequant_matmul_tiled: the codes of
+ * 128 rows x 256 columns form one 16 KB tile (row blocks of 128, then column blocks of 256, in
+ * row-major order of tiles); inside a tile row r takes 128 bytes, and its 16-byte chunk c (32
+ * codes) is stored at position c XOR (r mod 8) of the row.  Rows and columns past the matrix are
+ * zero.  The pages fix no layout for the deployed codes; this one lets the product read each
+ * tile with one contiguous copy.
+ *   packed   [m, d / 8] uint32 in gptq_pack's layout for 4-bit codes, d % 32 == 0, 16-byte
+ *            aligned, device.
+ *   tiled    gptq_tiled_words(m, d) uint32 out, 16-byte aligned, device.
+ * Asynchronous.  Errors: ARG. */
+long long gptq_tiled_words(int64_t m, int64_t d);
+int gptq_retile_codes(gptq_ctx* ctx, const uint32_t* packed, int64_t m, int64_t d,
+                      uint32_t* tiled);
+
+/* gptq_dequant_matmul over the tile-contiguous codes, on the tensor path only: 4-bit codes, X
+ * bf16 / f16 with d % 32 == 0 and 16-byte aligned, group -1 or a multiple of 128; the other
+ * arguments as for gptq_dequant_matmul.  Asynchronous.  Errors: ARG, CUDA; ARG or TIMEOUT via
+ * gptq_sync_status. */
+int gptq_dequant_matmul_tiled(gptq_ctx* ctx, const void* X, int x_dtype, int64_t T, int64_t d,
+                              const uint32_t* tiled, int64_t m, int group, int64_t n_g,
+                              const float* scales, const int32_t* zeros, float* Y);
+
 /* Two-sided rounding (GPTQ-2D, [D] "GPTQ-2D：把一个"四次方"难题压回"三次方"的故事"): X [m, n] is
  * rounded to an integer matrix Z for the metric ||A (Z - X) B||^2, given the metric factors
  * G_A = A^T A (m x m) and G_B = B B^T (n x n).  First each factor is turned in place into the

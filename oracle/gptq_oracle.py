@@ -599,3 +599,33 @@ def dequant_matmul(X, packed, d: int, bits: int, scale, zero, group: int, group_
     ze = np.asarray(zero, np.int64)[:, gid]
     W_hat = (sc * (codes - ze).astype(np.float32)).astype(np.float32)
     return np.asarray(X, np.float64) @ W_hat.astype(np.float64).T
+
+
+def tile_codes4(packed, m: int, d: int):
+    """The tile-contiguous layout of 4-bit packed codes that the library's product can read with
+    whole-tile copies (a layout of this library; the pages fix none for deployed codes): 16 KB
+    tiles of 128 rows x 256 codes, tiles in row-major order of (row block, column block); inside a
+    tile row r takes 128 bytes and its 16-byte chunk c (32 codes, words 4c .. 4c + 3 of the
+    block) sits at position c XOR (r mod 8).  Rows and columns past the matrix are zero.
+    Returns a flat uint32 array."""
+    packed = np.asarray(packed, np.uint32)
+    wpr = d // 8
+    RT, KT = -(-m // 128), -(-d // 256)
+    full = np.zeros((RT * 128, KT * 32), np.uint32)
+    full[:m, :wpr] = packed[:, :wpr]
+    t = full.reshape(RT, 128, KT, 8, 4).transpose(0, 2, 1, 3, 4)    # [RT, KT, r, c, word]
+    r = np.arange(128)[:, None]
+    logical = np.arange(8)[None, :] ^ (r & 7)                      # chunk stored at pc
+    out = np.take_along_axis(t, logical[None, None, :, :, None], axis=3)
+    return out.reshape(-1)
+
+
+def untile_codes4(tiled, m: int, d: int):
+    """Inverse of `tile_codes4` (the [m, d / 8] packed words)."""
+    RT, KT = -(-m // 128), -(-d // 256)
+    t = np.asarray(tiled, np.uint32).reshape(RT, KT, 128, 8, 4)
+    r = np.arange(128)[:, None]
+    stored_at = np.arange(8)[None, :] ^ (r & 7)                    # where logical chunk c sits
+    logical = np.take_along_axis(t, stored_at[None, None, :, :, None], axis=3)
+    full = logical.transpose(0, 2, 1, 3, 4).reshape(RT * 128, KT * 32)
+    return full[:m, :d // 8]

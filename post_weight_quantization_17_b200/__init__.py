@@ -58,6 +58,10 @@ _SIGS = {
     "gptq_unpack": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
     "gptq_dequant_matmul": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _i64, _i32, _i32, _vp, _i64,
                                    _vp, _vp, _vp]),
+    "gptq_tiled_words": (ctypes.c_longlong, [_i64, _i64]),
+    "gptq_retile_codes": (_i32, [_vp, _vp, _i64, _i64, _vp]),
+    "gptq_dequant_matmul_tiled": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _i64, _i32, _i64, _vp,
+                                         _vp, _vp]),
     "gptq_twosided_factor": (_i32, [_vp, _vp, _i64]),
     "gptq_twosided_round": (_i32, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]),
 }
@@ -225,6 +229,31 @@ def gptq_dequant_matmul(ctx: Context, X, packed, d: int, bits: int, group: int, 
                                   m, bits, group, _ptr(group_id), scales.shape[1], _ptr(scales),
                                   _ptr(zeros), _ptr(Y))
     ctx.check(rc, "gptq_dequant_matmul")
+
+
+def gptq_tiled_words(m: int, d: int) -> int:
+    return int(_lib.gptq_tiled_words(m, d))
+
+
+def gptq_retile_codes(ctx: Context, packed, d: int, tiled):
+    """4-bit packed codes [m, d / 8] -> the tile-contiguous copy (see include/gptq.h)."""
+    _dev(packed, torch.int32, "packed")
+    _dev(tiled, torch.int32, "tiled")
+    ctx.check(_lib.gptq_retile_codes(ctx.handle, _ptr(packed), packed.shape[0], d, _ptr(tiled)),
+              "gptq_retile_codes")
+
+
+def gptq_dequant_matmul_tiled(ctx: Context, X, tiled, m: int, group: int, scales, zeros, Y):
+    """Y [T, m] = X [T, d] Ŵᵀ over the tile-contiguous 4-bit codes."""
+    T, d = X.shape
+    _dev(X, name="X")
+    for t, dt, nm in ((tiled, torch.int32, "tiled"), (scales, torch.float32, "scales"),
+                      (zeros, torch.int32, "zeros"), (Y, torch.float32, "Y")):
+        _dev(t, dt, nm)
+    ctx.check(_lib.gptq_dequant_matmul_tiled(ctx.handle, _ptr(X), _DTYPE_CODE[X.dtype], T, d,
+                                             _ptr(tiled), m, group, scales.shape[1],
+                                             _ptr(scales), _ptr(zeros), _ptr(Y)),
+              "gptq_dequant_matmul_tiled")
 
 
 def gptq_twosided_factor(ctx: Context, G):

@@ -318,6 +318,44 @@ int gptq_dequant_matmul(gptq_ctx* h, const void* X, int x_dtype, int64_t T, int6
                               group_id, (int)n_g, scales, zeros, Y, part, avail);
 }
 
+long long gptq_tiled_words(int64_t m, int64_t d) {
+  if (m < 1 || d < 1) return 0;
+  return gptq::retile_words(m, d);
+}
+
+int gptq_retile_codes(gptq_ctx* h, const uint32_t* packed, int64_t m, int64_t d,
+                      uint32_t* tiled) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  if (!packed || !tiled || m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || d % 32 != 0 ||
+      !al(packed) || !al(tiled))
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "retile_codes: bad argument (m=%lld d=%lld)", (long long)m,
+                 (long long)d);
+  return gptq::retile_codes(c, packed, (int)m, (int)d, tiled);
+}
+
+int gptq_dequant_matmul_tiled(gptq_ctx* h, const void* X, int x_dtype, int64_t T, int64_t d,
+                              const uint32_t* tiled, int64_t m, int group, int64_t n_g,
+                              const float* scales, const int32_t* zeros, float* Y) {
+  if (!h) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  if (!X || !tiled || !scales || !zeros || !Y || !(x_dtype == GPTQ_BF16 || x_dtype == GPTQ_F16) ||
+      T < 1 || d < 1 || m < 1 || T > 65535LL * 8 || d > INT32_MAX || m > INT32_MAX ||
+      d % 32 != 0 || !al(X) || !al(tiled) || !(group == -1 || (group > 0 && group % 128 == 0)) ||
+      n_g < (group == -1 ? 1 : (d + group - 1) / group) || n_g > INT32_MAX)
+    GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "dequant_matmul_tiled: bad argument (T=%lld d=%lld m=%lld group=%d)",
+                 (long long)T, (long long)d, (long long)m, group);
+  Carver cv(c);
+  const size_t avail = (c->ws_bytes > gptq::kStatusBytes + 256)
+                            ? (c->ws_bytes - gptq::kStatusBytes - 256) / 4
+                            : 0;
+  float* part = cv.take<float>(0);
+  return gptq::dequant_matmul_tiled(c, X, x_dtype, (int)T, (int)d, tiled, (int)m, group,
+                                    (int)n_g, scales, zeros, Y, part, avail);
+}
+
 int gptq_twosided_factor(gptq_ctx* h, float* G, int64_t k) {
   if (!h) return GPTQ_ERR_ARG;
   Ctx* c = &h->c;

@@ -31,6 +31,7 @@
 #include "tc_util.cuh"
 
 #include <algorithm>
+#include <cstring>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -72,6 +73,8 @@ struct DqParams {
   const float* scales;
   const int32_t* zeros;
   float* out;              // Y [T, m], or the split-K partials [splits, T, m]
+  const uint32_t* tiled;   // codes in the tile-contiguous layout (gptq_retile_codes), or null
+  int ktiles;              // 256-code tiles per row block in that layout
   long long split_stride;  // T * m when partials are written, else 0
   uint32_t idesc;
 };
@@ -130,6 +133,17 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, 
   return true;
 }
 
+// One contiguous global -> shared copy of `bytes` (16-byte aligned, a multiple of 16) whose
+// completion is counted on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(tc::smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -160,7 +174,7 @@ __device__ __forceinline__ void dequant_word(uint32_t word, uint32_t zz, uint32_
   }
 }
 
-template <int BN, bool BF16>
+template <int BN, bool BF16, bool TILED>
 __global__ void __launch_bounds__(DQ_THREADS)
     k_dqmm_tc(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
               DqParams p, DeviceStatus* st, long long budget) {
@@ -207,7 +221,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
     tc::mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
-    tc::prefetch_tmap(&tmC);
+    if (!TILED) tc::prefetch_tmap(&tmC);
     tc::prefetch_tmap(&tmX);
   }
   if (warp == 1) tc::tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -231,12 +245,28 @@ __global__ void __launch_bounds__(DQ_THREADS)
           *abort_flag = 1;
           break;
         }
-        tc::mbar_expect_tx(&full_c[s], Cfg::C_BYTES);
-        const int x0 = (k_begin + j * Cfg::SPS) * 16;  // in 32-bit words
+        if (TILED) {
+          // whole 16 KB tiles, already in the swizzled order the reads below expect; a tile past
+          // the row's end is not loaded (its steps are never processed)
+          const int kt0 = (k_begin + j * Cfg::SPS) / 2;
+          int nbox = 0;
 #pragma unroll
-        for (int bx = 0; bx < Cfg::NB; ++bx)
-          tc::tma_load_2d(cbuf + s * Cfg::C_BYTES + bx * DQ_BOX, &tmC, &full_c[s], x0 + 32 * bx,
-                          row0);
+          for (int bx = 0; bx < Cfg::NB; ++bx) nbox += (kt0 + bx < p.ktiles) ? 1 : 0;
+          tc::mbar_expect_tx(&full_c[s], nbox * DQ_BOX);
+#pragma unroll
+          for (int bx = 0; bx < Cfg::NB; ++bx)
+            if (kt0 + bx < p.ktiles)
+              bulk_load_1d(cbuf + s * Cfg::C_BYTES + bx * DQ_BOX,
+                           p.tiled + ((size_t)blockIdx.x * p.ktiles + kt0 + bx) * (DQ_BOX / 4),
+                           DQ_BOX, &full_c[s]);
+        } else {
+          tc::mbar_expect_tx(&full_c[s], Cfg::C_BYTES);
+          const int x0 = (k_begin + j * Cfg::SPS) * 16;  // in 32-bit words
+#pragma unroll
+          for (int bx = 0; bx < Cfg::NB; ++bx)
+            tc::tma_load_2d(cbuf + s * Cfg::C_BYTES + bx * DQ_BOX, &tmC, &full_c[s], x0 + 32 * bx,
+                            row0);
+        }
         issued = j + 1;
       }
       for (int j = max(0, issued - Cfg::CST); j < issued; ++j)
@@ -533,15 +563,16 @@ bool dequant_matmul_tc_applies(const void* X, int x_dtype, int d, const uint32_t
          al(packed) && (group == -1 || group % DQ_KS == 0) && group_id == nullptr;
 }
 
-template <int BN, bool BF16>
+template <int BN, bool BF16, bool TILED>
 static int launch_dqmm_tc(Ctx* c, const void* X, int T, int d, const uint32_t* packed, int m,
                           int group, int ng, const float* scales, const int32_t* zeros, float* Y,
                           float* part_ws, size_t part_floats) {
   using Cfg = DqCfg<BN>;
   const int wpr = d / 8;
   CUtensorMap mc, mx;
-  if (!dq_map(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, wpr, m, wpr, 32, DQ_BM,
-              CU_TENSOR_MAP_SWIZZLE_128B))
+  memset(&mc, 0, sizeof(mc));
+  if (!TILED && !dq_map(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, wpr, m, wpr, 32, DQ_BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
     GPTQ_SET_ERR(c, GPTQ_ERR_CUDA, "dequant_matmul: tensor map for the codes failed");
   if (!dq_map(&mx, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
               X, d, T, d, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -555,6 +586,7 @@ static int launch_dqmm_tc(Ctx* c, const void* X, int T, int d, const uint32_t* p
   if (BN <= 64) {
     long long best = -1;
     for (int cand = ks; cand >= 1; --cand) {
+      if (TILED && cand != ks && cand % 2) continue;  // splits start on whole 256-code tiles
       const long long sp = (ks + cand - 1) / cand;
       if (sp > 1 && (size_t)sp * T * m > part_floats) break;
       const long long waves = (rt * tt * sp + slots - 1) / slots;
@@ -575,11 +607,13 @@ static int launch_dqmm_tc(Ctx* c, const void* X, int T, int d, const uint32_t* p
   p.zeros = zeros;
   p.out = (splits > 1) ? part_ws : Y;
   p.split_stride = (splits > 1) ? (long long)T * m : 0;
+  p.tiled = TILED ? packed : nullptr;
+  p.ktiles = (d + 255) / 256;
   p.idesc = tc::idesc_f32acc(BF16 ? 1u : 0u, false, false, DQ_BM, BN);
-  GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_dqmm_tc<BN, BF16>,
+  GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_dqmm_tc<BN, BF16, TILED>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
-  GPTQ_LAUNCH(c, k_dqmm_tc<BN, BF16>, dim3(rt, tt, splits), DQ_THREADS, Cfg::SMEM, mc, mx, p,
-              c->status, c->timeout_cycles);
+  GPTQ_LAUNCH(c, k_dqmm_tc<BN, BF16, TILED>, dim3(rt, tt, splits), DQ_THREADS, Cfg::SMEM, mc, mx,
+              p, c->status, c->timeout_cycles);
   if (splits > 1) {
     const long long nel = (long long)T * m;
     GPTQ_LAUNCH(c, k_dqmm_reduce, (int)((nel + 255) / 256), 256, 0, (const float*)part_ws, splits,
@@ -588,27 +622,70 @@ static int launch_dqmm_tc(Ctx* c, const void* X, int T, int d, const uint32_t* p
   return GPTQ_OK;
 }
 
+template <bool TILED>
+static int dispatch_dqmm_tc(Ctx* c, const void* X, int x_dtype, int T, int d,
+                            const uint32_t* codes, int m, int group, int ng, const float* scales,
+                            const int32_t* zeros, float* Y, float* part_ws, size_t part_floats) {
+  const bool bf = (x_dtype == GPTQ_BF16);
+  if (T <= 16)
+    return bf ? launch_dqmm_tc<16, true, TILED>(c, X, T, d, codes, m, group, ng, scales, zeros,
+                                                Y, part_ws, part_floats)
+              : launch_dqmm_tc<16, false, TILED>(c, X, T, d, codes, m, group, ng, scales, zeros,
+                                                 Y, part_ws, part_floats);
+  if (T <= 64)
+    return bf ? launch_dqmm_tc<64, true, TILED>(c, X, T, d, codes, m, group, ng, scales, zeros,
+                                                Y, part_ws, part_floats)
+              : launch_dqmm_tc<64, false, TILED>(c, X, T, d, codes, m, group, ng, scales, zeros,
+                                                 Y, part_ws, part_floats);
+  return bf ? launch_dqmm_tc<128, true, TILED>(c, X, T, d, codes, m, group, ng, scales, zeros, Y,
+                                               part_ws, part_floats)
+            : launch_dqmm_tc<128, false, TILED>(c, X, T, d, codes, m, group, ng, scales, zeros, Y,
+                                                part_ws, part_floats);
+}
+
+int dequant_matmul_tiled(Ctx* c, const void* X, int x_dtype, int T, int d,
+                         const uint32_t* tiled, int m, int group, int ng, const float* scales,
+                         const int32_t* zeros, float* Y, float* part_ws, size_t part_floats) {
+  return dispatch_dqmm_tc<true>(c, X, x_dtype, T, d, tiled, m, group, ng, scales, zeros, Y,
+                                part_ws, part_floats);
+}
+
+// 16-byte chunk o of the tile-contiguous layout: tile o / 1024 (row block rt, 256-code column
+// block kt), row r = (o % 1024) / 8 of the tile, stored chunk pc = o % 8 holding the row's
+// logical chunk pc ^ (r & 7) (the 128-byte swizzle); rows and columns past the matrix are zero.
+__global__ void k_retile_w4(const uint32_t* __restrict__ packed, int m, int wpr, int ktiles,
+                            long long nchunks, uint32_t* __restrict__ tiled) {
+  pdl_wait();
+  pdl_release();
+  const long long o = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= nchunks) return;
+  const long long tile = o / 1024;
+  const int q = (int)(o % 1024), r = q / 8, pc = q % 8, cidx = pc ^ (r & 7);
+  const long long rt = tile / ktiles, kt = tile % ktiles;
+  const long long row = rt * DQ_BM + r, word = kt * 32 + cidx * 4;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (row < m && word + 4 <= wpr) v = *reinterpret_cast<const uint4*>(packed + row * wpr + word);
+  reinterpret_cast<uint4*>(tiled)[o] = v;
+}
+
+long long retile_words(long long m, long long d) {
+  return ((m + DQ_BM - 1) / DQ_BM) * ((d + 255) / 256) * (DQ_BOX / 4);
+}
+
+int retile_codes(Ctx* c, const uint32_t* packed, int m, int d, uint32_t* tiled) {
+  const long long nchunks = retile_words(m, d) / 4;
+  GPTQ_LAUNCH(c, k_retile_w4, (int)((nchunks + 255) / 256), 256, 0, packed, m, d / 8,
+              (d + 255) / 256, nchunks, tiled);
+  return GPTQ_OK;
+}
+
 int dequant_matmul(Ctx* c, const void* X, int x_dtype, int T, int d, const uint32_t* packed,
                    int m, int bits, int group, const int32_t* group_id, int ng,
                    const float* scales, const int32_t* zeros, float* Y, float* part_ws,
                    size_t part_floats) {
-  if (dequant_matmul_tc_applies(X, x_dtype, d, packed, bits, group, group_id)) {
-    const bool bf = (x_dtype == GPTQ_BF16);
-    if (T <= 16)
-      return bf ? launch_dqmm_tc<16, true>(c, X, T, d, packed, m, group, ng, scales, zeros, Y,
-                                           part_ws, part_floats)
-                : launch_dqmm_tc<16, false>(c, X, T, d, packed, m, group, ng, scales, zeros, Y,
-                                            part_ws, part_floats);
-    if (T <= 64)
-      return bf ? launch_dqmm_tc<64, true>(c, X, T, d, packed, m, group, ng, scales, zeros, Y,
-                                           part_ws, part_floats)
-                : launch_dqmm_tc<64, false>(c, X, T, d, packed, m, group, ng, scales, zeros, Y,
-                                            part_ws, part_floats);
-    return bf ? launch_dqmm_tc<128, true>(c, X, T, d, packed, m, group, ng, scales, zeros, Y,
-                                          part_ws, part_floats)
-              : launch_dqmm_tc<128, false>(c, X, T, d, packed, m, group, ng, scales, zeros, Y,
-                                           part_ws, part_floats);
-  }
+  if (dequant_matmul_tc_applies(X, x_dtype, d, packed, bits, group, group_id))
+    return dispatch_dqmm_tc<false>(c, X, x_dtype, T, d, packed, m, group, ng, scales, zeros, Y,
+                                   part_ws, part_floats);
   const int wpr = (int)(((long long)d * bits + 31) / 32);
   const dim3 grid((m + 127) / 128, (T + 7) / 8);
   if (x_dtype == GPTQ_BF16)

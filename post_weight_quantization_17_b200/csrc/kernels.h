@@ -63,6 +63,13 @@ int dequant_matmul(Ctx* c, const void* X, int x_dtype, int T, int d, const uint3
                    int m, int bits, int group, const int32_t* group_id, int ng,
                    const float* scales, const int32_t* zeros, float* Y, float* part_ws,
                    size_t part_floats);
+// the tile-contiguous layout of 4-bit codes (16 KB tiles of 128 rows x 256 codes, swizzled as the
+// tensor kernel reads them) and the product over it
+long long retile_words(long long m, long long d);
+int retile_codes(Ctx* c, const uint32_t* packed, int m, int d, uint32_t* tiled);
+int dequant_matmul_tiled(Ctx* c, const void* X, int x_dtype, int T, int d,
+                         const uint32_t* tiled, int m, int group, int ng, const float* scales,
+                         const int32_t* zeros, float* Y, float* part_ws, size_t part_floats);
 
 // ---- two-sided rounding (GPTQ-2D, k_twosided.cu); workspace: Y, C, etas (m n floats each) and
 // RAT (m m floats)

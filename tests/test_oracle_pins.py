@@ -619,3 +619,19 @@ def test_dequant_matmul_other_widths(bits, group):
     W_hat = (sc[:, gid] * (codes - ze[:, gid]).astype(np.float32)).astype(np.float32)
     y = O.dequant_matmul(X, O.pack(codes, bits), d, bits, sc, ze, group)
     assert np.allclose(y, X @ W_hat.astype(np.float64).T, rtol=0, atol=1e-12)
+
+
+def test_tile_codes4_layout():
+    """Worked positions of the tile-contiguous layout, its inverse, and its zero padding."""
+    rng = np.random.default_rng(40)
+    m, d = 130, 288                      # 2 row blocks (the second ragged), 2 column blocks
+    packed = rng.integers(1, 2 ** 32, size=(m, d // 8), dtype=np.uint64).astype(np.uint32)
+    t = O.tile_codes4(packed, m, d)
+    assert t.size == 2 * 2 * 4096
+    assert np.array_equal(t[0:32], packed[0, 0:32])            # row 0: no swizzle
+    assert np.array_equal(t[32 + 4:32 + 8], packed[1, 0:4])    # row 1, chunk 0 -> position 1
+    assert np.array_equal(t[32 * 5 + 4 * 2:32 * 5 + 4 * 3], packed[5, 4 * 7:4 * 8])  # 7 ^ 5 = 2
+    assert np.array_equal(t[4096:4096 + 4], packed[0, 32:36])  # column block 1 of row block 0
+    # row block 1 holds rows 128, 129 and 126 zero rows; column block 1 holds 4 words per row
+    assert np.count_nonzero(t) == np.count_nonzero(packed)
+    assert np.array_equal(O.untile_codes4(t, m, d), packed)
