@@ -30,6 +30,13 @@ def test_null_context_is_an_argument_error():
                                  None, None, None) == G.GPTQ_ERR_ARG
     assert L.gptq_pack(None, None, 1, 1, 4, None) == G.GPTQ_ERR_ARG
     assert L.gptq_unpack(None, None, 1, 1, 4, None) == G.GPTQ_ERR_ARG
+    assert L.gptq_dequant_matmul(None, None, 0, 1, 32, None, 1, 4, 128, None, 1, None, None,
+                                 None) == G.GPTQ_ERR_ARG
+    assert L.gptq_dequant_matmul_tiled(None, None, 0, 1, 32, None, 1, 128, 1, None, None,
+                                       None) == G.GPTQ_ERR_ARG
+    assert L.gptq_retile_codes(None, None, 1, 32, None) == G.GPTQ_ERR_ARG
+    assert L.gptq_twosided_factor(None, None, 4) == G.GPTQ_ERR_ARG
+    assert L.gptq_twosided_round(None, None, 2, 2, None, None, None, None) == G.GPTQ_ERR_ARG
     assert L.gptq_sync_status(None) == G.GPTQ_ERR_ARG
     assert L.gptq_destroy(None) == G.GPTQ_ERR_ARG
     assert L.gptq_last_error(None) == b""
@@ -50,6 +57,15 @@ def test_workspace_bytes_cover_the_buffers(m, d):
     assert ws0 >= 4 * (d // 2 + 64) ** 2
     # act-order adds the permuted working copy (fp32) and permuted codes
     assert ws1 >= m * d * 5
+
+
+def test_tiled_words():
+    """16 KB (4096 words) per 128-row x 256-code tile, ragged blocks rounded up; 0 for empty."""
+    assert G.gptq_tiled_words(128, 256) == 4096
+    assert G.gptq_tiled_words(129, 256) == 2 * 4096
+    assert G.gptq_tiled_words(12288, 49152) == 96 * 192 * 4096
+    assert G.gptq_tiled_words(300, 1056) == 3 * 5 * 4096
+    assert G.gptq_tiled_words(0, 256) == 0
 
 
 def test_words_per_row():
