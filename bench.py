@@ -473,6 +473,24 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def oracle_w4a16_sample(m: int, d: int, T: int, rows: int, g: int = 128):
+    """The CPU oracle's W4A16 product (unpack, dequantize, multiply in fp64) on `rows` of the m
+    rows; returns (seconds for the sample, seconds extrapolated to all m rows, description)."""
+    import numpy as np
+    from oracle import gptq_oracle as O
+    rng = np.random.default_rng(1)
+    packed = rng.integers(0, 2 ** 32, size=(rows, d // 8), dtype=np.uint64).astype(np.uint32)
+    scales = rng.uniform(1e-3, 2.1e-2, (rows, d // g)).astype(np.float32)
+    zeros = rng.integers(0, 16, (rows, d // g))
+    X = rng.normal(size=(T, d)).astype(np.float32).astype(np.float64)
+    t0 = time.perf_counter()
+    O.dequant_matmul(X, packed, d, 4, scales, zeros, g)
+    dt = time.perf_counter() - t0
+    desc = (f"the oracle's product on {rows} of {m} rows (time x{m / rows:g}), T={T}; "
+            "extrapolated to the whole layer")
+    return dt, dt * m / rows, desc
+
+
 def run_w4a16(args):
     """The consumer of the packed format on one GPU: Y [T, m] = X [T, d] Ŵᵀ with X bf16 and
     random valid 4-bit codes (g = 128).  Small T is bound by reading the codes from HBM, large T
@@ -543,6 +561,11 @@ def run_w4a16(args):
                                    "layout", "m": m, "d": d, "T": T, "layout": args.w4a16_layout,
                        "group": g, "l2": "flushed between timed calls (256 MiB write)"},
             "roofline": roof, "clocks": clk, "gpu_launches": launches}
+    if not args.no_cpu_baseline:
+        sample_s, full_s, desc = oracle_w4a16_sample(m, d, T, 512 if d > 8192 else m)
+        line["cpu_baseline"] = {"value": m * d / full_s, "unit": "weights/s",
+                                "cores": cores_used(), "kind": "oracle", "sample": desc,
+                                "sample_seconds": sample_s}
     print(json.dumps(line), flush=True)
     ctx.close()
 
