@@ -516,6 +516,17 @@ def run_w4a16(args):
 
         def product():
             G.gptq_dequant_matmul_tiled(ctx, X, tiled, m, g, scales, zeros, Y)
+
+        # the tiled product must equal the row-layout product (same definition; the split of K
+        # may differ, so the sums agree to rounding) before it is timed
+        Y_rows = torch.empty_like(Y)
+        G.gptq_dequant_matmul(ctx, X, packed, d, 4, g, scales, zeros, Y_rows)
+        product()
+        G.gptq_sync_status(ctx)
+        rel = float((Y - Y_rows).norm() / Y_rows.norm())
+        if not rel <= 1e-5:
+            raise RuntimeError(f"tiled W4A16 product differs from the row-layout one: rel {rel:.2e}")
+        del Y_rows
     else:
         def product():
             G.gptq_dequant_matmul(ctx, X, packed, d, 4, g, scales, zeros, Y)

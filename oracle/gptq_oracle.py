@@ -53,13 +53,6 @@ def hessian_tokens(Xt) -> np.ndarray:
     return (2.0 / Xt.shape[0]) * (Xt.T @ Xt)
 
 
-def token_sum(Xt) -> np.ndarray:
-    """S = sum_t x_t x_t^T, the unnormalised statistic (so that H = 2 S / N).  [T] §9.4 table:
-    X X^T can be accumulated in batches."""
-    Xt = np.asarray(Xt, dtype=np.float64)
-    return Xt.T @ Xt
-
-
 # --------------------------------------------------------------------------------------------
 # Quantization grid and quantizer
 # --------------------------------------------------------------------------------------------

@@ -303,6 +303,66 @@ def test_retry_raises_damping():
         O.prepare_with_retry(np.array([[1.0, 0.0], [0.0, -100.0]]), percdamp=0.01)
 
 
+def test_damping_lambda_hand_values():
+    """[T] §10 order (dead features, then the permutation, then damping) and eq.(12): λ is
+    percdamp times the mean of diag(H') taken AFTER the dead diagonal entries became 1, with the
+    fp32 eps as its floor.  Hand values: diag(H) = (4, 2, 0) -> dead fix-up (4, 2, 1), mean 7/3,
+    percdamp 0.03 -> λ = 0.07 (a mean taken before the fix-up would give 0.06)."""
+    H = np.array([[4.0, 1.0, 0.0], [1.0, 2.0, 0.0], [0.0, 0.0, 0.0]])
+    Hl, perm, dead, lam, Hp = O.prepare(H, 0.03, act_order=True)
+    assert abs(lam - 0.07) < 1e-15
+    assert dead.tolist() == [False, False, True]
+    assert perm.tolist() == [0, 1, 2]               # 4 > 2 > 1 (the dead entry counts as 1)
+    assert np.allclose(np.diag(Hl), [4.07, 2.07, 1.07], rtol=0, atol=1e-15)
+    assert Hl[0, 1] == 1.0 and Hl[1, 0] == 1.0 and np.all(Hl[2, :2] == 0.0)
+    assert np.allclose(Hl - Hp, 0.07 * np.eye(3), rtol=0, atol=1e-15)
+    # act-order moves the dead column: diag (1, 5, 0) -> (1, 5, 1), order 1, 0, 2 (stable tie)
+    H2 = np.diag([1.0, 5.0, 0.0])
+    _, perm2, _, lam2, Hp2 = O.prepare(H2, 0.3, act_order=True)
+    assert perm2.tolist() == [1, 0, 2] and np.array_equal(np.diag(Hp2), [5.0, 1.0, 1.0])
+    assert abs(lam2 - 0.3 * 7.0 / 3.0) < 1e-15
+    # the floor: percdamp 0 (and a percdamp whose λ falls below it) gives exactly 2^-23
+    for pd in (0.0, 1e-12):
+        assert O.prepare(np.diag([1.0, 1.0]), pd)[3] == 2.0 ** -23
+    assert O.FP32_EPS == float(np.finfo(np.float32).eps)
+
+
+def test_damping_retry_hand_values():
+    """The retry reading of [T] §10's remark: percdamp x10 per failed factorization, at most 3
+    times.  H = [[1, 1.5], [1.5, 1]] has eigenvalues 2.5 and -0.5 and mean diagonal 1, so
+    λ = 0.01 and 0.1 fail and λ = 1 succeeds: two retries, λ = 1.  [[1, 3], [3, 1]] (eigenvalue
+    -2) needs λ = 10: three retries.  [[1, 30], [30, 1]] still fails at λ = 10 and raises."""
+    out = O.prepare_with_retry(np.array([[1.0, 1.5], [1.5, 1.0]]), percdamp=0.01)
+    assert out["retries"] == 2 and abs(out["lam"] - 1.0) < 1e-12
+    assert np.allclose(out["H_lambda"], [[2.0, 1.5], [1.5, 2.0]], atol=1e-12)
+    out3 = O.prepare_with_retry(np.array([[1.0, 3.0], [3.0, 1.0]]), percdamp=0.01)
+    assert out3["retries"] == 3 and abs(out3["lam"] - 10.0) < 1e-9
+    with pytest.raises(np.linalg.LinAlgError):
+        O.prepare_with_retry(np.array([[1.0, 30.0], [30.0, 1.0]]), percdamp=0.01)
+
+
+def test_is_valid_act_order_accepts_and_rejects():
+    """The parity checker for another implementation's act-order permutation: a descending order
+    of diag(H) (dead entries counted as 1), near-ties within rtol in either order, and nothing
+    else."""
+    H = np.diag([3.0, 0.0, 0.5, 2.0, 2.0 * (1 + 4e-6)])   # dead feature 1 counts as 1
+    assert O.is_valid_act_order([0, 4, 3, 1, 2], H)        # exact descending order
+    assert O.is_valid_act_order([0, 3, 4, 1, 2], H)        # near-tie (4e-6 < 1e-5) swapped
+    assert not O.is_valid_act_order([0, 3, 4, 1, 2], H, rtol=1e-6)  # same swap beyond rtol
+    assert not O.is_valid_act_order([0, 4, 3, 2, 1], H)    # 0.5 before the dead entry's 1
+    assert not O.is_valid_act_order([4, 0, 3, 1, 2], H)    # 2 before 3: far beyond rtol
+    assert not O.is_valid_act_order([0, 4, 4, 1, 2], H)    # repeated index
+    assert not O.is_valid_act_order([0, 4, 3, 1], H)       # short list
+    assert not O.is_valid_act_order([0, 4, 3, 1, 5], H)    # index out of range
+    # it agrees with the oracle's own stable argsort on a random Hessian
+    rng = np.random.default_rng(3)
+    A = rng.normal(size=(9, 30))
+    Hr = A @ A.T
+    assert O.is_valid_act_order(O.prepare(Hr, 0.01, True)[1], Hr)
+    assert not O.is_valid_act_order(np.arange(9)[::-1].copy(), Hr) or \
+        np.all(np.diff(np.diag(Hr)) >= 0)
+
+
 # ---------------------------------------------------------------- block formula ≡ lazy update
 def test_eq32_block_formula_equals_lazy_tail():
     """eq.(32)/(49): D Γ^{-1} G_BT equals E R_BT for a block of already-chosen grid values."""
