@@ -1,25 +1,31 @@
 #!/usr/bin/env python
 """GPTQ layer-quantization throughput on B200: weights quantized per second.
 
-Workload (one "step" = the whole hot path on one layer): a Llama-7B-shaped q_proj,
-W 4096 x 4096 fp16 (1% outlier columns x10), X = 262,144 calibration tokens (bf16, low rank
-256 + noise with Student-t(3) feature scales), 4-bit asymmetric grids per 128 columns, lazy
-blocks of 128.  A step runs the four C-ABI calls: Hessian accumulation over all tokens,
-preparation of R (dead features, damping, factorization), column-wise quantization with lazy
-trailing updates, and packing.  Inputs are synthetic and seeded (workloads/synth.py).
+One "step" is the whole hot path on the configuration's layers: Hessian accumulation over all
+calibration tokens, preparation of R (dead features, damping, factorization), column-wise
+quantization with lazy trailing updates, and packing, through the four C-ABI calls.  Inputs
+are synthetic and seeded (workloads/synth.py).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Default workload (the largest single-GPU configuration): a 175B-shaped fc2, W 12288 x 49152
+fp16 with 0.5 % outlier columns, X = 65,536 calibration tokens (bf16, ReLU of a rank-1024
+mixture plus noise) accumulated in 8192-token chunks, 4-bit asymmetric grids per 128 columns,
+lazy blocks of 128 (--bits 2 for its 2-bit line).  --config 2 / 3 / 4 time the q_proj, the
+act-order down_proj and the 7B decoder block (seven matrices over four shared inputs).
 
-With N > 1 (torchrun, one process per GPU) every rank quantizes its own independent layer
-(weak scaling, no data-path collective); value = all ranks' weights / max-over-ranks time.
-Rank 0 prints one JSON line.
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+
+With N > 1 every rank quantizes its own independent layer (weak scaling, no data-path
+collective); value = all ranks' weights / max-over-ranks time.  Without a launcher's
+environment, --gpus N > 1 starts the N ranks itself.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
+import socket
 import subprocess
 import sys
 import tempfile
@@ -31,21 +37,25 @@ sys.path.insert(0, ROOT)
 METRIC = "GPTQ weights quantized/sec per layer (4-bit g128) on 1 B200; % of roofline"
 UNIT = "weights/s"
 
-
 GRID_MODES = {"static": 0, "dynamic": 2}  # the library's grid_given argument
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--chunk", type=int, default=262144, help="tokens per accumulate call")
+    ap.add_argument("--config", type=int, choices=[2, 3, 4, 5], default=5,
+                    help="5: 175B fc2 (default); 2: q_proj; 3: act-order down_proj; 4: 7B block")
+    ap.add_argument("--bits", type=int, choices=[2, 3, 4], default=0,
+                    help="override the configuration's bit width (the fc2's 2-bit line: 2)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stage-profile", action="store_true",
+                    help="skip the extra, untimed step that times every kernel by stage")
     ap.add_argument("--scale", type=float, default=1.0,
-                    help="shrink the layer (tests only); the bench line is for 1.0")
+                    help="shrink the layers (tests only); the bench line is for 1.0")
     ap.add_argument("--grid", choices=sorted(GRID_MODES), default="static",
                     help="static groups (the default line) or dynamic groups (grid refitted per "
                          "processing group on the GPU)")
@@ -58,31 +68,70 @@ def parse():
                          "(gptq_retile_codes, outside the timed region)")
     ap.add_argument("--n-tokens", type=int, default=0,
                     help="calibration tokens (profiling captures only; the bench line uses all)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
-def workload(scale: float, n_tokens: int = 0):
-    import dataclasses
-    from workloads.synth import CONFIGS
-    spec = CONFIGS[2][0]
-    if scale != 1.0:
-        spec = spec.scaled(max(32, int(spec.m * scale)), max(128, int(spec.d * scale)),
-                           max(512, int(spec.n_tokens * scale)))
-    if n_tokens:
-        spec = dataclasses.replace(spec, n_tokens=n_tokens)
-    return spec
+@dataclasses.dataclass
+class Group:
+    """One calibration input (one Hessian, one factorization) and the matrices that share it."""
+    name: str
+    x_spec: object                  # LayerSpec whose d, N and X recipe define the input
+    mats: list                      # LayerSpecs quantized with this input's R
+    seed: int
 
 
-def workload_config(spec, chunk, grid="static"):
-    return {"workload": f"q_proj {spec.m}x{spec.d} fp16 W, N={spec.n_tokens} bf16 tokens, "
-                        f"{spec.bits}-bit g{spec.group}" +
-                        (" (dynamic groups)" if grid == "dynamic" else "") +
-                        f", block {spec.block}",
-            "grid": grid,
-            "m": spec.m, "d": spec.d, "n_tokens": spec.n_tokens, "bits": spec.bits,
-            "group": spec.group, "block": spec.block, "act_order": spec.act_order,
-            "chunk_tokens": min(chunk, spec.n_tokens),
-            "l2": "flushed between timed steps (256 MiB write)"}
+def workload(config: int, scale: float = 1.0, n_tokens: int = 0, bits: int = 0, seed: int = 1):
+    """The configuration's layer groups (config 4: seven matrices over four inputs)."""
+    from workloads.synth import BLOCK7B_SHARED_INPUT, CONFIGS
+
+    def adjust(spec):
+        if config != 5:
+            # only the fc2 configuration streams its tokens in chunks; the others are one
+            # accumulation over all calibration tokens
+            spec = dataclasses.replace(spec, chunk=spec.n_tokens)
+        if bits:
+            spec = dataclasses.replace(spec, bits=bits)
+        if scale != 1.0:
+            spec = spec.scaled(max(32, int(spec.m * scale)), max(128, int(spec.d * scale)),
+                               max(512, int(spec.n_tokens * scale)))
+        if n_tokens:
+            spec = dataclasses.replace(spec, n_tokens=n_tokens, chunk=min(spec.chunk, n_tokens))
+        return spec
+
+    if config == 4:
+        specs = {s.name.split("_")[0]: adjust(s) for s in CONFIGS[4]}
+        return [Group(g, specs[members[0]], [specs[n] for n in members], 100 * seed + k)
+                for k, (g, members) in enumerate(BLOCK7B_SHARED_INPUT.items())]
+    spec = adjust(CONFIGS[config][0])
+    return [Group(spec.name, spec, [spec], seed)]
+
+
+def workload_name(config: int, groups) -> str:
+    s = groups[0].mats[0]
+    if config == 4:
+        return (f"7B decoder block: 7 fp16 matrices (q,k,v,o 4096x4096; gate,up 11008x4096; down "
+                f"4096x11008) over 4 shared inputs, N={s.n_tokens} bf16 tokens each, "
+                f"{s.bits}-bit g{s.group}, block {s.block}")
+    kind = {2: "q_proj", 3: "down_proj", 5: "175B fc2"}[config]
+    ao = ", act-order" if s.act_order else ""
+    return (f"{kind} {s.m}x{s.d} fp16 W, N={s.n_tokens} bf16 tokens in {s.chunk}-token chunks, "
+            f"{s.bits}-bit g{s.group}{ao}, block {s.block}")
+
+
+def workload_config(config, groups, grid="static"):
+    s = groups[0].mats[0]
+    return {"workload": workload_name(config, groups) +
+                        (" (dynamic groups)" if grid == "dynamic" else ""),
+            "config": config, "grid": grid,
+            "matrices": [[t.m, t.d] for g in groups for t in g.mats],
+            "n_tokens": s.n_tokens, "chunk_tokens": s.chunk, "bits": s.bits,
+            "group": s.group, "block": s.block, "act_order": s.act_order,
+            "weights_per_step": weights_per_step(groups),
+            "l2": "flushed between timed steps (256 MiB write); X is larger than L2"}
+
+
+def weights_per_step(groups) -> int:
+    return sum(t.m * t.d for g in groups for t in g.mats)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -140,12 +189,46 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- helpers
 def measured_peaks():
+    """Roofline denominators from MEASURED_PEAKS.json (measured on this machine's B200s):
+    bf16 TFLOP/s burst and sustained, HBM GB/s; else the recipe's fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             j = json.load(f)
-        return j.get("bf16_tflops", 1590.0), j.get("hbm_gbs", 6650.0), "measured"
-    return 1590.0, 6650.0, "fallback"
+        return {"bf16": j.get("bf16_tflops", 1590.0),
+                "bf16_sustained": j.get("bf16_tflops_sustained", 1400.0),
+                "hbm": j.get("hbm_gbs", 6650.0), "source": "measured"}
+    return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def measure_tf32_peak(device) -> float:
+    """Dense TF32 tensor throughput of this GPU, measured the way the bf16 peak was: one cuBLAS
+    matmul of 8192^3 in fp32 with TF32 allowed, best of 10, CUDA events (TFLOP/s)."""
+    import torch
+    n = 8192
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = True
+    try:
+        g = torch.Generator(device=device).manual_seed(0)
+        a = torch.randn(n, n, device=device, generator=g)
+        b = torch.randn(n, n, device=device, generator=g)
+        c = torch.empty(n, n, device=device)
+        for _ in range(3):
+            torch.matmul(a, b, out=c)
+        best = float("inf")
+        for _ in range(10):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b, out=c)
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    del a, b, c
+    torch.cuda.empty_cache()
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
 def kernel_source_digest(files):
@@ -185,7 +268,7 @@ def dist_setup(args):
         import torch.distributed as dist
         import datetime
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     else:
         torch.cuda.set_device(0)
     return world, rank, local
@@ -214,77 +297,123 @@ def rank_seed(rank: int) -> int:
     return 1 + rank
 
 
-def weak_scaling_value(world: int, m: int, d: int, per_step_s: float) -> float:
-    """Whole-job weights per second: every rank quantizes m x d weights per step, and the job
-    takes as long as its slowest rank."""
-    return world * m * d / per_step_s
+def weak_scaling_value(world: int, weights: int, per_step_s: float) -> float:
+    """Whole-job weights per second: every rank quantizes `weights` weights per step, and the
+    job takes as long as its slowest rank."""
+    return world * weights / per_step_s
 
 
-# ----------------------------------------------------------------------------- oracle leg
-def oracle_sample(spec, seed: int, n_tok: int, rows: int, grid: str = "static"):
-    """The CPU oracle on a bounded sample of the layer: H from `n_tok` tokens at full d,
-    preparation at full d, lazy-block quantization of `rows` rows.  Returns (seconds for the
-    sample, seconds extrapolated to the whole layer, description)."""
-    import numpy as np
-    import torch
-    from oracle import gptq_oracle as O
-    from workloads.synth import XSource, make_weight
-
-    W = make_weight(spec, seed, "cpu")[:rows].float().double().numpy()
-    xs = XSource(spec.scaled(spec.m, spec.d, n_tok, chunk=n_tok), seed, "cpu")
-    Xt = xs.chunk(0).float().double().numpy()
-    t0 = time.perf_counter()
-    H = O.hessian_tokens(Xt)
-    t1 = time.perf_counter()
-    prep = O.prepare_with_retry(H, spec.percdamp, spec.act_order)
-    t2 = time.perf_counter()
-    Wp = W[:, prep["perm"]]
-    if grid == "dynamic":
-        sc, ze = O.dynamic_grid_arrays(rows, spec.d, spec.group)
-        O.gptq_lazy(Wp, prep["R"], sc, ze, np.arange(spec.d) // spec.group, spec.bits,
-                    spec.block, dynamic=spec.group)
-    else:
-        sc, ze = O.fit_grid(W, spec.bits, spec.group)
-        gcol = (prep["perm"] // spec.group) if spec.group != -1 else np.zeros(spec.d, int)
-        O.gptq_lazy(Wp, prep["R"], sc, ze, gcol, spec.bits, spec.block)
-    t3 = time.perf_counter()
-    full = (t1 - t0) * (spec.n_tokens / n_tok) + (t2 - t1) + (t3 - t2) * (spec.m / rows)
-    desc = (f"H from {n_tok} of {spec.n_tokens} tokens (time x{spec.n_tokens / n_tok:g}), "
-            f"prepare at full d={spec.d}, quantize {rows} of {spec.m} rows "
-            f"(time x{spec.m / rows:g}); extrapolated to the whole layer")
-    return t3 - t0, full, desc
+def self_launch(args, argv) -> int:
+    """--gpus N > 1 without a launcher: start N ranks of this script with torch.distributed.run
+    on this node (rendezvous on 127.0.0.1) and return its exit status."""
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd, cwd=ROOT)
 
 
 def cores_used():
+    """Threads the oracle's numpy BLAS runs with (its parallel part), else the CPUs this process
+    may run on."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and max(n) > 0:
+            return int(max(n))
+    except Exception:
+        pass
     try:
         return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count()
 
 
+# ----------------------------------------------------------------------------- oracle leg
+def oracle_instance(W, x_chunks, spec, cols: int, grid: str = "static"):
+    """The CPU oracle, timed, on a leading block of one layer: the first `cols` input features
+    (columns of W and the matching rows of X) with every row of W and every token given.  W is
+    a torch tensor [m, d], x_chunks an iterable of token-major torch chunks [C, d] (any device).
+    Returns (seconds, weights quantized, description)."""
+    import numpy as np
+    from oracle import gptq_oracle as O
+    Wn = W[:, :cols].float().cpu().double().numpy()
+    m = Wn.shape[0]
+    t0 = time.perf_counter()
+    S = np.zeros((cols, cols))
+    n = 0
+    for c in x_chunks:
+        xc = c[:, :cols].float().cpu().double().numpy()
+        S += xc.T @ xc                           # the statistic, chunk by chunk ([T] §9.4)
+        n += xc.shape[0]
+    H = (2.0 / n) * S
+    prep = O.prepare_with_retry(H, spec.percdamp, spec.act_order)
+    Wp = Wn.copy()
+    Wp[:, prep["dead"]] = 0.0
+    Wp = Wp[:, prep["perm"]]
+    if grid == "dynamic":
+        sc, ze = O.dynamic_grid_arrays(m, cols, spec.group)
+        O.gptq_lazy(Wp, prep["R"], sc, ze, np.arange(cols) // spec.group, spec.bits,
+                    spec.block, dynamic=spec.group)
+    else:
+        sc, ze = O.fit_grid(Wn, spec.bits, spec.group)
+        gcol = (prep["perm"] // spec.group) if spec.group != -1 else np.zeros(cols, int)
+        codes, _, _ = O.gptq_lazy(Wp, prep["R"], sc, ze, gcol, spec.bits, spec.block)
+        O.pack(codes, spec.bits)
+    dt = time.perf_counter() - t0
+    desc = (f"the whole hot path (H over {n} tokens, prepare, lazy-block quantization, pack) on "
+            f"the layer's first {cols} of {spec.d} input features: {m}x{cols} weights, timed "
+            "in full, not extrapolated")
+    return dt, m * cols, desc
+
+
+def baseline_cols(d: int, n_tokens: int) -> int:
+    """Leading input features of the CPU baseline's instance: the largest power of two (at most
+    d) with n_tokens * cols^2 <= 2.75e11, which keeps the oracle's fp64 Hessian near 5e11 flop
+    and the whole instance at about 10-30 s on a 16-core host (2048 columns at 65536 tokens)."""
+    if n_tokens * d * d <= 2.75e11:
+        return d
+    cols = 1
+    while cols * 2 <= d and n_tokens * (cols * 2) ** 2 <= 2.75e11:
+        cols *= 2
+    return min(cols, d)
+
+
 def run_reference(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    """The oracle as it stands on the host cores, one bounded sample of the workload per step:
+    the first 512 input features of the configuration's first matrix (all its rows) over its
+    first 8192 tokens.  value = the weights of the sample / its measured time."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    spec = workload(args.scale, args.n_tokens)
-    n_tok, rows = min(2048, spec.n_tokens), min(16, spec.m)
+    from workloads.synth import XSource, make_weight
+    groups = workload(args.config, args.scale, args.n_tokens, args.bits)
+    spec = groups[0].mats[0]
+    cols, ntok = min(512, spec.d), min(8192, spec.n_tokens)
+    sub = spec.scaled(spec.m, cols, ntok, chunk=ntok)
+    W = make_weight(sub, 1, "cpu")
+    X = XSource(sub, 1, "cpu").chunk(0)
     for _ in range(args.warmup):
-        oracle_sample(spec, 1, n_tok, rows, args.grid)
-    fulls = []
-    desc = ""
+        oracle_instance(W, [X], sub, cols, args.grid)
+    times = []
+    desc, n_w = "", 0
     t_start = time.perf_counter()
     for _ in range(args.steps):
-        _, full, desc = oracle_sample(spec, 1, n_tok, rows, args.grid)
-        fulls.append(full)
+        dt, n_w, desc = oracle_instance(W, [X], sub, cols, args.grid)
+        times.append(dt)
     wall = time.perf_counter() - t_start
-    per_layer = sum(fulls) / len(fulls)
-    value = spec.m * spec.d / per_layer
+    per = sum(times) / len(times)
+    value = n_w / per
+    desc = ("a sample of the same recipe per step: " + desc +
+            f"; the per-weight cost grows with d and N, so this rate is above the full layer's")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": per_layer * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(spec, args.chunk, args.grid),
+            "config": workload_config(args.config, groups, args.grid),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores_used(),
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -294,53 +423,132 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- our path
+STAGE_KERNEL_FILES = {
+    "a1_hessian": ["post_weight_quantization_17_b200/csrc/k_syrk.cu",
+                   "post_weight_quantization_17_b200/csrc/tc_util.cuh"],
+    "a3_factor_gemm": ["post_weight_quantization_17_b200/csrc/k_gemm_tc.cu",
+                       "post_weight_quantization_17_b200/csrc/tc_util.cuh"],
+    "a6_update": ["post_weight_quantization_17_b200/csrc/k_gemm_pair.cu",
+                  "post_weight_quantization_17_b200/csrc/k_gemm_tc.cu",
+                  "post_weight_quantization_17_b200/csrc/tc_util.cuh"],
+}
+
+
+def stage_rooflines(groups, stage_ms, kern, peaks, tf32):
+    """Per-stage roofline entries: algorithmic work of the stage (flop or bytes, per step) over
+    its time per step, against the peak of the unit that bounds it.  stage_ms: event times of the
+    ABI calls in the timed steps; kern: per-stage kernel times of the profiled step (or None).
+    3xTF32 stages count fp32-accurate flops against a third of the TF32 peak (three tf32 products
+    per fp32-accurate product)."""
+    mats = [t for g in groups for t in g.mats]
+    f_syrk = sum(float(g.x_spec.n_tokens) * g.x_spec.d * (g.x_spec.d + 1) for g in groups)
+    f_fact = sum(2.0 / 3.0 * float(g.x_spec.d) ** 3 for g in groups)
+    f_upd = sum(float(t.m) * t.d * t.d for t in mats)
+    b_col = sum(19.0 * t.m * t.d for t in mats)       # W fp16 in, working copy, q, E, codes
+    b_grid = sum(2.0 * t.m * t.d + 8.0 * t.m * t.n_groups for t in mats)
+    b_pack = sum(t.m * t.d * (1.0 + t.bits / 8.0) for t in mats)
+    fp32_peak = tf32 / 3.0
+    out = {}
+
+    def tensor(name, flops, ms, peak, src, time_src):
+        if not ms:
+            return
+        ach = flops / (ms * 1e-3) / 1e12
+        out[name] = {"bound": "tensor", "work": flops, "work_unit": "flop", "ms_per_step": ms,
+                     "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                     "peak_source": src, "time": time_src}
+
+    def hbm(name, nbytes, ms):
+        if not ms:
+            return
+        ach = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"bound": "hbm", "work": nbytes, "work_unit": "byte", "ms_per_step": ms,
+                     "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm"], "peak_source": f"{peaks['source']} copy",
+                     "time": "kernel events (profiled step)"}
+
+    bf16_src = f"{peaks['source']} bf16 burst"
+    tf_src = "TF32 peak measured live (cuBLAS 8192^3, best of 10) / 3 for 3xTF32"
+    tensor("a1_hessian", f_syrk, stage_ms.get("hessian"), peaks["bf16"], bf16_src,
+           "ABI-call events (timed steps)")
+    tensor("a3_factor", f_fact, stage_ms.get("prepare"), fp32_peak, tf_src,
+           "ABI-call events of gptq_prepare_hinv (timed steps; includes a2)")
+    if kern:
+        k = lambda n: kern.get(n, (0.0, 0))[0]
+        tensor("a3_factor_gemm", f_fact, k("factor_gemm"), fp32_peak, tf_src,
+               "kernel events (profiled step); the second stream's GEMMs overlap the first's")
+        tensor("a6_update", f_upd, k("update"), fp32_peak, tf_src, "kernel events (profiled step)")
+        hbm("a4_grid", b_grid, k("grid"))
+        hbm("a5_column", b_col, k("column"))
+        hbm("a8_pack", b_pack, k("pack"))
+    return out
+
+
 def run_ours(args):
     import torch
     import post_weight_quantization_17_b200 as G
     from workloads.synth import XSource, make_weight
 
     world, rank, local = dist_setup(args)
-    spec = workload(args.scale, args.n_tokens)
     seed = rank_seed(rank)
+    groups = workload(args.config, args.scale, args.n_tokens, args.bits, seed)
     dev = torch.device("cuda", torch.cuda.current_device())
-    W = make_weight(spec, seed, dev)
-    # the data do not depend on --chunk: 8192-token chunks are generated and regrouped
-    xs = XSource(spec, seed, dev)
-    per = max(1, args.chunk // spec.chunk)
-    chunks = []
-    group = []
-    for c in xs.chunks():
-        group.append(c)
-        if len(group) == per:
-            chunks.append(torch.cat(group) if per > 1 else group[0])
-            group = []
-    if group:
-        chunks.append(torch.cat(group))
-    del group
+    peaks = measured_peaks()
+    tf32 = measure_tf32_peak(dev)
     stream = torch.cuda.Stream(dev)
-    ctx = G.Context(m_max=spec.m, d_max=spec.d, act_order=spec.act_order, stream=stream)
-    bufs = G.LayerBuffers(spec.m, spec.d, spec.bits, spec.group, dev)
+    m_max = max(t.m for g in groups for t in g.mats)
+    d_max = max(g.x_spec.d for g in groups)
+    ao = any(t.act_order for g in groups for t in g.mats)
+    ctx = G.Context(m_max=m_max, d_max=d_max, act_order=ao, stream=stream)
+    data = []
+    for g in groups:
+        chunks = list(XSource(g.x_spec, g.seed, dev).chunks())
+        Ws = [make_weight(t, g.seed * 10 + k, dev) for k, t in enumerate(g.mats)]
+        d = g.x_spec.d
+        S = torch.empty(d, d, device=dev)
+        R = torch.empty(d, d, device=dev)
+        perm = torch.empty(d, dtype=torch.int32, device=dev)
+        dead = torch.empty(d, dtype=torch.uint8, device=dev)
+        outs = [G.LayerBuffers(t.m, d, t.bits, t.group, dev, with_factor=False)
+                for t in g.mats]
+        data.append((g, chunks, Ws, S, R, perm, dead, outs))
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    syrk_ev = []
+    W_total = weights_per_step(groups)
+    STAGE_CALLS = ("hessian", "prepare", "quantize", "pack")
 
-    def step(record=False):
-        n = 0
-        for xc in chunks:
-            if record:
-                a = torch.cuda.Event(enable_timing=True)
+    def step(ev=None):
+        """One pass of the hot path over every group; ev: per-call event pairs to fill."""
+        def mark(name):
+            if ev is None:
+                return None
+            a = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            return (name, a)
+
+        def done(m):
+            if m is not None:
                 b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-            n = G.gptq_hessian_accumulate(ctx, xc, bufs.S, n)
-            if record:
                 b.record(stream)
-                syrk_ev.append((a, b))
-        G.gptq_prepare_hinv(ctx, bufs.S, n, spec.percdamp, spec.act_order, bufs.R, bufs.perm,
-                            bufs.dead)
-        G.gptq_quantize_layer(ctx, W, bufs.R, bufs.perm if spec.act_order else None, bufs.dead,
-                              spec.bits, spec.group, spec.block, GRID_MODES[args.grid],
-                              bufs.scales, bufs.zeros,
-                              bufs.codes, bufs.W_hat, bufs.col_loss)
-        G.gptq_pack(ctx, bufs.codes, spec.bits, bufs.packed)
+                ev.append((m[0], m[1], b))
+
+        for g, chunks, Ws, S, R, perm, dead, outs in data:
+            mk = mark("hessian")
+            n = 0
+            for xc in chunks:
+                n = G.gptq_hessian_accumulate(ctx, xc, S, n)
+            done(mk)
+            mk = mark("prepare")
+            G.gptq_prepare_hinv(ctx, S, n, g.x_spec.percdamp, g.x_spec.act_order, R, perm, dead)
+            done(mk)
+            for t, W, o in zip(g.mats, Ws, outs):
+                mk = mark("quantize")
+                G.gptq_quantize_layer(ctx, W, R, perm if t.act_order else None, dead, t.bits,
+                                      t.group, t.block, GRID_MODES[args.grid], o.scales, o.zeros,
+                                      o.codes, o.W_hat, o.col_loss)
+                done(mk)
+                mk = mark("pack")
+                G.gptq_pack(ctx, o.codes, t.bits, o.packed)
+                done(mk)
 
     clocks = ClockSampler(local)
     clocks.start()  # sampling covers the warm-up and the timed steps (nvidia-smi needs ~0.2 s)
@@ -352,13 +560,13 @@ def run_ours(args):
         barrier(world)
         torch.cuda.synchronize()
         launches0 = G.gptq_kernel_launches(ctx)
-        step_ev = []
+        step_ev, call_ev = [], []
         for _ in range(args.steps):
             flush.zero_()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            step(record=True)
+            step(call_ev)
             b.record(stream)
             step_ev.append((a, b))
         torch.cuda.synchronize()
@@ -367,94 +575,59 @@ def run_ours(args):
         clk = clocks.stop()
         launches = G.gptq_kernel_launches(ctx) - launches0
         G.gptq_sync_status(ctx)
+        # one more step, untimed, with every kernel bracketed by events, for the per-stage
+        # kernel times (the events serialize the launches, so this step is not a bench value)
+        kern = None
+        if not args.no_stage_profile:
+            flush.zero_()
+            G.gptq_timing_enable(ctx, True)
+            step()
+            kern = G.gptq_timing_read(ctx)
+            G.gptq_timing_enable(ctx, False)
+            G.gptq_sync_status(ctx)
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    syrk_ms = sum(a.elapsed_time(b) for a, b in syrk_ev) / args.steps
+    stage_ms = {k: 0.0 for k in STAGE_CALLS}
+    for name, a, b in call_ev:
+        stage_ms[name] += a.elapsed_time(b) / args.steps
     total_s = max_over_ranks(sum(step_ms) / 1e3, world)
     per_step_s = total_s / args.steps
-    value = weak_scaling_value(world, spec.m, spec.d, per_step_s)
+    value = weak_scaling_value(world, W_total, per_step_s)
 
-    # roofline of the dominant kernel (Hessian accumulation): algorithmic flops per launch
-    bf16_peak, hbm_peak, peak_src = measured_peaks()
-    syrk_flops = float(spec.n_tokens) * spec.d * (spec.d + 1)   # lower triangle incl. diagonal
-    n_launch = len(chunks)
-    achieved = syrk_flops / (syrk_ms / 1e3) / 1e12
-    digest = kernel_source_digest(["post_weight_quantization_17_b200/csrc/k_syrk.cu",
-                                   "post_weight_quantization_17_b200/csrc/gemm_simt.cuh",
-                                   "post_weight_quantization_17_b200/csrc/tc_util.cuh"])
-    roofline = {"kernel": "hessian_accumulate (S += X^T X)", "bound": "tensor",
-                "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
-                "frac": achieved / bf16_peak, "peak_source": f"{peak_src} bf16 burst",
-                "traffic": ncu_traffic("hessian_accumulate", digest, 1.0 / n_launch),
-                "algorithmic_flops_per_step": syrk_flops, "launches_per_step": n_launch,
-                "kernel_ms_per_step": syrk_ms, "source_digest": digest}
+    stages = stage_rooflines(groups, stage_ms, kern, peaks, tf32)
+    # the headline roofline: the stage that takes the longest
+    main_name = max((n for n in ("a1_hessian", "a3_factor_gemm", "a6_update") if n in stages),
+                    key=lambda n: stages[n]["ms_per_step"], default="a1_hessian")
+    roofline = dict(stages.get(main_name, {}))
+    if roofline:
+        roofline["stage"] = main_name
+        roofline["kernel"] = {"a1_hessian": "k_syrk_tc2 (S += X^T X)",
+                              "a3_factor_gemm": "k_gemm_tc (factorization recursion GEMMs)",
+                              "a6_update": "k_gemm_pair + k_gemm_tc (lazy trailing updates)"}[
+            main_name]
+        digest = kernel_source_digest(STAGE_KERNEL_FILES[main_name])
+        roofline["source_digest"] = digest
+        launches_main = (kern or {}).get({"a1_hessian": "hessian", "a3_factor_gemm": "factor_gemm",
+                                          "a6_update": "update"}[main_name], (0, 0))[1]
+        roofline["launches_per_step"] = launches_main
+        tr = ncu_traffic(main_name, digest)
+        roofline["traffic"] = tr
+        roofline["traffic_per"] = "step" if tr is not None else None
 
     # end to end through the public API with host buffers (pinned), copies inside the region:
-    # X goes up in 16384-token slabs on a copy stream, double-buffered, and each slab's Hessian
-    # update runs while the next slab is in flight; then prepare, quantize, pack, and the packed
-    # codes with their grid come back to the host
+    # X goes up in slabs on a copy stream, double-buffered, each slab's Hessian update running
+    # while the next slab is in flight; W goes up beside it; then prepare, quantize, pack, and the
+    # packed codes with their grid come back to the host
     e2e = None
     if not args.no_e2e:
-        import post_weight_quantization_17_b200 as G
-        X_host = torch.cat([c.cpu() for c in chunks]).pin_memory()
-        W_host = W.cpu().pin_memory()
-        out_host = [torch.empty_like(t, device="cpu").pin_memory() for t in
-                    (bufs.packed, bufs.scales, bufs.zeros)]
-        h2d = X_host.numel() * X_host.element_size() + W_host.numel() * W_host.element_size()
-        d2h = sum(t.numel() * t.element_size() for t in out_host)
-        slab = 16384
-        n_tok = X_host.shape[0]
-        slabs = [(a0, min(n_tok, a0 + slab)) for a0 in range(0, n_tok, slab)]
-        dbuf = [torch.empty(slab, spec.d, dtype=X_host.dtype, device=dev) for _ in range(2)]
-        copy_stream = torch.cuda.Stream()
-        e2e_steps = max(3, min(args.steps, 10))
-        with torch.cuda.stream(stream):
-            torch.cuda.synchronize()
-            barrier(world)
-            t_ev = []
-            for _ in range(e2e_steps):
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                landed = [torch.cuda.Event(), torch.cuda.Event()]
-                free = [torch.cuda.Event(), torch.cuda.Event()]
-                a.record(stream)
-                W.copy_(W_host, non_blocking=True)
-                copy_stream.wait_event(a)
-                n_total = 0
-                for k, (a0, a1) in enumerate(slabs):
-                    u = k % 2
-                    with torch.cuda.stream(copy_stream):
-                        if k >= 2:
-                            copy_stream.wait_event(free[u])
-                        dbuf[u][:a1 - a0].copy_(X_host[a0:a1], non_blocking=True)
-                        landed[u].record(copy_stream)
-                    stream.wait_event(landed[u])
-                    n_total = G.gptq_hessian_accumulate(ctx, dbuf[u][:a1 - a0], bufs.S, n_total)
-                    free[u].record(stream)
-                G.gptq_prepare_hinv(ctx, bufs.S, n_total, spec.percdamp, spec.act_order, bufs.R,
-                                    bufs.perm, bufs.dead)
-                G.gptq_quantize_layer(ctx, W, bufs.R, bufs.perm if spec.act_order else None,
-                                      bufs.dead, spec.bits, spec.group, spec.block,
-                                      GRID_MODES[args.grid],
-                                      bufs.scales, bufs.zeros, bufs.codes, bufs.W_hat,
-                                      bufs.col_loss)
-                G.gptq_pack(ctx, bufs.codes, spec.bits, bufs.packed)
-                for hd, dv in zip(out_host, (bufs.packed, bufs.scales, bufs.zeros)):
-                    hd.copy_(dv, non_blocking=True)
-                b.record(stream)
-                b.synchronize()
-                t_ev.append((a, b))
-            barrier(world)
-        e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in t_ev) / 1e3 / e2e_steps, world)
-        e2e = {"value": weak_scaling_value(world, spec.m, spec.d, e2e_s), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_s * 1e3, "h2d_slab_tokens": slab}
+        e2e = run_e2e(args, G, ctx, stream, data, world, W_total)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_tok, rows = min(131072, spec.n_tokens), min(3072, spec.m)
-        sample_s, full_s, desc = oracle_sample(spec, seed, n_tok, rows, args.grid)
-        cpu = {"value": spec.m * spec.d / full_s, "unit": UNIT, "cores": cores_used(),
-               "kind": "oracle", "sample": desc, "sample_seconds": sample_s}
+        g0, chunks0, Ws0 = data[0][0], data[0][1], data[0][2]
+        cols = baseline_cols(g0.x_spec.d, g0.x_spec.n_tokens)
+        dt, nw, desc = oracle_instance(Ws0[0], chunks0, g0.mats[0], cols, args.grid)
+        cpu = {"value": nw / dt, "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+               "sample": desc, "sample_seconds": dt}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -462,8 +635,13 @@ def run_ours(args):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16 products, f32 accumulate/factor/quantize",
                 "data": "synthetic (seeded; workloads/synth.py)",
-                "config": workload_config(spec, args.chunk, args.grid),
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+                "config": workload_config(args.config, groups, args.grid),
+                "roofline": roofline, "stages": stages,
+                "stage_ms_per_step": stage_ms,
+                "kernel_ms_profiled_step": {k: v[0] for k, v in (kern or {}).items()},
+                "kernel_launches_profiled_step": {k: v[1] for k, v in (kern or {}).items()},
+                "tf32_tflops_measured": tf32,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
                 "gpu_launches": launches, "gpu_launches_per_step": launches / args.steps,
                 "step_ms_min": min(step_ms), "step_ms_max": max(step_ms)}
         print(json.dumps(line), flush=True)
@@ -471,6 +649,80 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_e2e(args, G, ctx, stream, data, world, W_total):
+    import torch
+    host = []
+    h2d = d2h = 0
+    for g, chunks, Ws, S, R, perm, dead, outs in data:
+        X_host = [c.cpu().pin_memory() for c in chunks]
+        W_host = [W.cpu().pin_memory() for W in Ws]
+        o_host = [[torch.empty_like(t, device="cpu").pin_memory()
+                   for t in (o.packed, o.scales, o.zeros)] for o in outs]
+        h2d += sum(x.numel() * x.element_size() for x in X_host)
+        h2d += sum(w.numel() * w.element_size() for w in W_host)
+        d2h += sum(t.numel() * t.element_size() for oh in o_host for t in oh)
+        host.append((X_host, W_host, o_host))
+    dev = stream.device
+    slab = max(c.shape[0] for d in data for c in d[1])
+    d_max = max(d[0].x_spec.d for d in data)
+    xdt = data[0][1][0].dtype
+    dbuf = [torch.empty(slab * d_max, dtype=xdt, device=dev) for _ in range(2)]
+    copy_stream = torch.cuda.Stream(dev)
+    e2e_steps = max(3, min(args.steps, 5))
+    with torch.cuda.stream(stream):
+        torch.cuda.synchronize()
+        barrier(world)
+        t_ev = []
+        for _ in range(e2e_steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            copy_stream.wait_event(a)
+            landed = [torch.cuda.Event(), torch.cuda.Event()]
+            free = [torch.cuda.Event(), torch.cuda.Event()]
+            k = 0
+            for (g, chunks, Ws, S, R, perm, dead, outs), (X_host, W_host, o_host) in zip(data, host):
+                d = g.x_spec.d
+                for W, Wh in zip(Ws, W_host):
+                    with torch.cuda.stream(copy_stream):
+                        W.copy_(Wh, non_blocking=True)
+                w_landed = torch.cuda.Event()
+                w_landed.record(copy_stream)
+                n_total = 0
+                for xh in X_host:
+                    u = k % 2
+                    rows = xh.shape[0]
+                    buf = dbuf[u][:rows * d].view(rows, d)
+                    with torch.cuda.stream(copy_stream):
+                        if k >= 2:
+                            copy_stream.wait_event(free[u])
+                        buf.copy_(xh, non_blocking=True)
+                        landed[u].record(copy_stream)
+                    stream.wait_event(landed[u])
+                    n_total = G.gptq_hessian_accumulate(ctx, buf, S, n_total)
+                    free[u].record(stream)
+                    k += 1
+                G.gptq_prepare_hinv(ctx, S, n_total, g.x_spec.percdamp, g.x_spec.act_order, R,
+                                    perm, dead)
+                stream.wait_event(w_landed)
+                for t, W, o, oh in zip(g.mats, Ws, outs, o_host):
+                    G.gptq_quantize_layer(ctx, W, R, perm if t.act_order else None, dead, t.bits,
+                                          t.group, t.block, GRID_MODES[args.grid], o.scales,
+                                          o.zeros, o.codes, o.W_hat, o.col_loss)
+                    G.gptq_pack(ctx, o.codes, t.bits, o.packed)
+                    for hd, dv in zip(oh, (o.packed, o.scales, o.zeros)):
+                        hd.copy_(dv, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            t_ev.append((a, b))
+        barrier(world)
+    G.gptq_sync_status(ctx)
+    e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in t_ev) / 1e3 / e2e_steps, world)
+    return {"value": weak_scaling_value(world, W_total, e2e_s), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": e2e_s * 1e3, "h2d_slab_tokens": slab, "steps": e2e_steps}
 
 
 def oracle_w4a16_sample(m: int, d: int, T: int, rows: int, g: int = 128):
@@ -551,7 +803,8 @@ def run_w4a16(args):
     launches = G.gptq_kernel_launches(ctx) - launches0
     G.gptq_sync_status(ctx)
     t = sum(times) / len(times)
-    tflops_peak, hbm_peak, src = measured_peaks()
+    pk = measured_peaks()
+    tflops_peak, hbm_peak, src = pk["bf16"], pk["hbm"], pk["source"]
     nbytes = m * d // 2 + m * (d // g) * 8 + T * d * 2 + T * m * 4
     flops = 2.0 * T * m * d
     hbm_bound = nbytes / (hbm_peak * 1e9) >= flops / (tflops_peak * 1e12)
@@ -582,10 +835,13 @@ def run_w4a16(args):
 
 
 def main():
-    args = parse()
+    argv = sys.argv[1:]
+    args = parse(argv)
     if args.w4a16:
         run_w4a16(args)
         return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(self_launch(args, argv))
     if args.impl == "reference":
         run_reference(args)
     else:

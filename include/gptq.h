@@ -71,6 +71,42 @@ const char* gptq_last_error(const gptq_ctx* ctx);
 /* Number of kernels this context has launched so far (a host-side counter; no sync). */
 uint64_t gptq_kernel_launches(const gptq_ctx* ctx);
 
+/* Sets how long a pipelined kernel launched through this context waits for its next stage,
+ * buffer or partial before it gives up (GPU clock cycles; 0 restores the default, 4e9 cycles,
+ * about 2 s at the B200's clock).  A wait that runs out records GPTQ_ERR_TIMEOUT in the device
+ * status word, and its CTA waits for the copies and tensor-core operations it has already issued
+ * (a separate, fixed budget), frees its tensor memory and exits; the context stays usable.
+ * Kernels that run on CTA pairs keep the default budget.  The pages have no counterpart: this is
+ * the failure path of the library's own bounded waits, for callers that need a hang turned into an
+ * error quickly and for testing that path.  Errors: ARG (cycles < 0). */
+int gptq_set_wait_budget(gptq_ctx* ctx, int64_t cycles);
+
+/* Stages that gptq_timing_read reports; every kernel launch counts under one of them.  The
+ * a-numbers are the steps of the hot path: a1 Hessian, a2 preconditioning, a3 factorization
+ * (base blocks, recursion GEMMs, copies), a4 grid fit, a5 column loop (working copy, column
+ * blocks), a6 lazy trailing updates, a7 outputs in original order, a8 packing; then the W4A16
+ * product and two-sided rounding. */
+enum {
+  GPTQ_STAGE_HESSIAN = 0, GPTQ_STAGE_PREPARE = 1, GPTQ_STAGE_FACTOR_BASE = 2,
+  GPTQ_STAGE_FACTOR_GEMM = 3, GPTQ_STAGE_FACTOR_COPY = 4, GPTQ_STAGE_GRID = 5,
+  GPTQ_STAGE_COLUMN = 6, GPTQ_STAGE_UPDATE = 7, GPTQ_STAGE_OUTPUT = 8, GPTQ_STAGE_PACK = 9,
+  GPTQ_STAGE_DEQUANT = 10, GPTQ_STAGE_TWOSIDED = 11, GPTQ_STAGE_OTHER = 12,
+  GPTQ_NUM_STAGES = 13
+};
+
+/* Per-stage kernel timing, for measurement.  on != 0: from now on every kernel this context
+ * launches is bracketed by two CUDA events on its stream (which serializes it with its
+ * neighbours: programmatic dependent launch no longer overlaps their set-up), and the records
+ * kept so far are dropped; on == 0: launches are no longer timed.  Errors: ARG. */
+int gptq_timing_enable(gptq_ctx* ctx, int on);
+
+/* Synchronizes on the last timed launch and adds up, per stage, the time between each timed
+ * launch's two events (ms, host double[GPTQ_NUM_STAGES]) and the number of timed launches (host
+ * int64_t[GPTQ_NUM_STAGES]); then drops the records.  Launches on the factorization's second
+ * stream overlap those on the first, so the sum of a stage can exceed its elapsed time.
+ * Errors: ARG, CUDA. */
+int gptq_timing_read(gptq_ctx* ctx, double* ms, int64_t* launches);
+
 /* Synchronizes the context stream, returns and clears the device status word
  * (GPTQ_OK, GPTQ_ERR_NONFINITE, GPTQ_ERR_NOT_PD or GPTQ_ERR_TIMEOUT), or GPTQ_ERR_CUDA. */
 int gptq_sync_status(gptq_ctx* ctx);
@@ -159,10 +195,18 @@ int gptq_quantize_layer(gptq_ctx* ctx, const void* W, int w_dtype, int64_t m, in
  *   other arguments exactly as for gptq_quantize_layer.
  * The scratch must hold about 4 m (512 + d / 32) + 12 d bytes, plus 5 m d bytes when perm is
  * not NULL; a layer that needs more returns GPTQ_ERR_ARG (the only work enqueued then clears
- * the scratch's status word).  The
- * first call on a device looks up the array's device address (cudaGetSymbolAddress) and should
- * come before any stream capture.  The call synchronizes `cuda_stream` and returns the device
- * status (GPTQ_OK or GPTQ_ERR_NONFINITE) like gptq_sync_status.  Every call shares the one
+ * the scratch's status word).
+ * Device memory: under CUDA's lazy module loading the array is reserved on a device when the
+ * library's module is first loaded there, i.e. at the first call of this entry point on that
+ * device (or at any earlier library call there).  A caller with a fixed device budget should make
+ * that first call before committing the rest of the device's memory; if the module cannot be
+ * loaded the call returns GPTQ_ERR_CUDA.  Every call looks up the array's device address on the
+ * current device (cudaGetSymbolAddress, which allocates nothing); the first call on a device
+ * should come before any stream capture.
+ * `cuda_stream` must belong to the current device, else GPTQ_ERR_ARG.
+ * The call synchronizes `cuda_stream` and returns the device status (GPTQ_OK or
+ * GPTQ_ERR_NONFINITE) like gptq_sync_status.  If a launch fails after earlier kernels were
+ * enqueued it synchronizes the stream too and returns GPTQ_ERR_CUDA.  Every call shares the one
  * array and it keeps the last call's contents: calls whose work overlaps on the GPU (other
  * streams or host threads) race and must be serialized by the caller. */
 int gptq_quantize_layer_noalloc(void* cuda_stream, const void* W, int w_dtype, int64_t m,

@@ -27,6 +27,10 @@ STATUS_NAMES = {0: "OK", 1: "ERR_ARG", 2: "ERR_CUDA", 3: "ERR_NOT_PD", 4: "ERR_N
 
 _DTYPE_CODE = {torch.bfloat16: GPTQ_BF16, torch.float16: GPTQ_F16, torch.float32: GPTQ_F32}
 
+# stages of gptq_timing_read, in the order of the GPTQ_STAGE_* constants
+STAGES = ("hessian", "prepare", "factor_base", "factor_gemm", "factor_copy", "grid", "column",
+          "update", "output", "pack", "dequant", "twosided", "other")
+
 
 class GPTQError(RuntimeError):
     def __init__(self, code: int, msg: str):
@@ -47,6 +51,9 @@ _SIGS = {
     "gptq_last_error": (ctypes.c_char_p, [_vp]),
     "gptq_kernel_launches": (ctypes.c_uint64, [_vp]),
     "gptq_sync_status": (_i32, [_vp]),
+    "gptq_set_wait_budget": (_i32, [_vp, _i64]),
+    "gptq_timing_enable": (_i32, [_vp, _i32]),
+    "gptq_timing_read": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]),
     "gptq_hessian_accumulate": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, ctypes.POINTER(_i64)]),
     "gptq_prepare_hinv": (_i32, [_vp, _vp, _i64, _i64, ctypes.c_float, _i32, _vp, _vp, _vp,
                                  ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_i32)]),
@@ -132,6 +139,24 @@ def gptq_kernel_launches(ctx: Context) -> int:
     return int(_lib.gptq_kernel_launches(ctx.handle))
 
 
+def gptq_set_wait_budget(ctx: Context, cycles: int):
+    """Wait budget of this context's pipelined kernels in GPU cycles (0 = the default)."""
+    ctx.check(_lib.gptq_set_wait_budget(ctx.handle, int(cycles)), "gptq_set_wait_budget")
+
+
+def gptq_timing_enable(ctx: Context, on: bool = True):
+    """Time every launch of this context with CUDA events (serializes neighbouring launches)."""
+    ctx.check(_lib.gptq_timing_enable(ctx.handle, 1 if on else 0), "gptq_timing_enable")
+
+
+def gptq_timing_read(ctx: Context) -> dict:
+    """{stage: (milliseconds summed over its timed launches, launches)} since the last read."""
+    ms = (ctypes.c_double * len(STAGES))()
+    n = (_i64 * len(STAGES))()
+    ctx.check(_lib.gptq_timing_read(ctx.handle, ms, n), "gptq_timing_read")
+    return {name: (ms[k], int(n[k])) for k, name in enumerate(STAGES) if n[k]}
+
+
 def gptq_sync_status(ctx: Context) -> int:
     rc = _lib.gptq_sync_status(ctx.handle)
     ctx.check(rc, "gptq_sync_status")
@@ -191,10 +216,11 @@ def gptq_quantize_layer_noalloc(W, R, perm, dead, bits: int, group: int, block: 
     m, d = W.shape
     _dev(W, name="W")
     s = stream if stream is not None else torch.cuda.current_stream(W.device)
-    return int(_lib.gptq_quantize_layer_noalloc(
-        ctypes.c_void_p(s.cuda_stream), _ptr(W), _DTYPE_CODE[W.dtype], m, d, _ptr(R), _ptr(perm),
-        _ptr(dead), bits, group, block, int(grid_given), _ptr(scales), _ptr(zeros),
-        _ptr(codes), _ptr(W_hat), _ptr(col_loss)))
+    with torch.cuda.device(W.device):   # the library resolves its scratch on the current device
+        return int(_lib.gptq_quantize_layer_noalloc(
+            ctypes.c_void_p(s.cuda_stream), _ptr(W), _DTYPE_CODE[W.dtype], m, d, _ptr(R),
+            _ptr(perm), _ptr(dead), bits, group, block, int(grid_given), _ptr(scales),
+            _ptr(zeros), _ptr(codes), _ptr(W_hat), _ptr(col_loss)))
 
 
 def gptq_pack(ctx: Context, codes, bits: int, packed):
@@ -277,15 +303,18 @@ def words_per_row(d: int, bits: int) -> int:
 
 
 class LayerBuffers:
-    """Device buffers of one layer's outputs (allocated once, reused across calls)."""
+    """Device buffers of one layer's outputs (allocated once, reused across calls).  With
+    with_factor=False only the quantization outputs are allocated (for matrices that share
+    another layer's S, R, perm and dead)."""
 
-    def __init__(self, m: int, d: int, bits: int, group: int, device):
+    def __init__(self, m: int, d: int, bits: int, group: int, device, with_factor: bool = True):
         ng = 1 if group == -1 else -(-d // group)
         f32 = torch.float32
-        self.S = torch.empty(d, d, dtype=f32, device=device)
-        self.R = torch.empty(d, d, dtype=f32, device=device)
-        self.perm = torch.empty(d, dtype=torch.int32, device=device)
-        self.dead = torch.empty(d, dtype=torch.uint8, device=device)
+        if with_factor:
+            self.S = torch.empty(d, d, dtype=f32, device=device)
+            self.R = torch.empty(d, d, dtype=f32, device=device)
+            self.perm = torch.empty(d, dtype=torch.int32, device=device)
+            self.dead = torch.empty(d, dtype=torch.uint8, device=device)
         self.scales = torch.empty(m, ng, dtype=f32, device=device)
         self.zeros = torch.empty(m, ng, dtype=torch.int32, device=device)
         self.codes = torch.empty(m, d, dtype=torch.uint8, device=device)

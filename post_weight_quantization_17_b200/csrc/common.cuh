@@ -7,6 +7,7 @@
 #include <stdio.h>
 #include <string>
 #include <utility>
+#include <vector>
 
 #include "../../include/gptq.h"
 
@@ -21,6 +22,19 @@ struct DeviceStatus {
   float pad;
 };
 
+// Bounded waits.  A pipeline wait (for the next stage, buffer or partial) gives up after the
+// context's budget, records GPTQ_ERR_TIMEOUT and makes its CTA unwind.  While unwinding, a CTA
+// waits for the copies and tensor-core operations it issued itself, with the fixed drain
+// budget: those complete on their own, and no CTA may free TMEM or exit before they have.
+constexpr long long kDefaultWaitCycles = 4000000000LL;
+constexpr long long kDrainCycles = 4000000000LL;
+
+// One timed launch: CUDA events recorded on the launching stream around the kernel.
+struct TimedLaunch {
+  int stage;
+  cudaEvent_t start, stop;
+};
+
 struct Ctx {
   cudaStream_t stream = nullptr;
   int device = 0;
@@ -30,11 +44,37 @@ struct Ctx {
   bool owns_ws = false;
   DeviceStatus* status = nullptr;  // lives at the start of ws
   std::string last_error;
-  long long timeout_cycles = 4000000000LL;  // bounded waits in the pipelined kernels
+  long long timeout_cycles = kDefaultWaitCycles;  // pipeline waits (gptq_set_wait_budget)
   unsigned long long launches = 0;          // kernels this context has launched
   cudaStream_t side = nullptr;              // second stream of the factorization recursion
   cudaEvent_t ev[2 * 64] = {};              // its per-level events
+  // per-stage timing (gptq_timing_enable): the stage every launch is counted under, the launches
+  // recorded since the last read, and a pool of reusable events
+  int stage = GPTQ_STAGE_OTHER;
+  bool timing = false;
+  std::vector<TimedLaunch> timed;
+  std::vector<cudaEvent_t> event_pool;
+  size_t pool_used = 0;
 };
+
+// Sets the stage that launches are counted under for the lifetime of the scope.
+struct StageScope {
+  Ctx* c;
+  int saved;
+  StageScope(Ctx* ctx, int stage) : c(ctx), saved(ctx->stage) { c->stage = stage; }
+  ~StageScope() { c->stage = saved; }
+};
+
+inline cudaError_t pooled_event(Ctx* c, cudaEvent_t* e) {
+  if (c->pool_used == c->event_pool.size()) {
+    cudaEvent_t n;
+    cudaError_t r = cudaEventCreate(&n);
+    if (r != cudaSuccess) return r;
+    c->event_pool.push_back(n);
+  }
+  *e = c->event_pool[c->pool_used++];
+  return cudaSuccess;
+}
 
 constexpr size_t kStatusBytes = 256;
 
@@ -85,7 +125,16 @@ inline cudaError_t launch_pdl(Ctx* c, void (*kernel)(KArgs...), dim3 grid, dim3 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   ++c->launches;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (!c->timing) return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  // timed launch: the events serialize this kernel with its neighbours on the stream
+  TimedLaunch t{c->stage, nullptr, nullptr};
+  cudaError_t r = pooled_event(c, &t.start);
+  if (r == cudaSuccess) r = pooled_event(c, &t.stop);
+  if (r == cudaSuccess) r = cudaEventRecord(t.start, c->stream);
+  if (r == cudaSuccess) r = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (r == cudaSuccess) r = cudaEventRecord(t.stop, c->stream);
+  if (r == cudaSuccess) c->timed.push_back(t);
+  return r;
 }
 
 template <class T> __device__ __forceinline__ float to_f32(T v);

@@ -98,6 +98,7 @@ int gptq_create(gptq_ctx** out, void* stream, void* workspace, size_t workspace_
 
 int gptq_destroy(gptq_ctx* h) {
   if (!h) return GPTQ_ERR_ARG;
+  for (cudaEvent_t e : h->c.event_pool) cudaEventDestroy(e);
   if (h->c.side) {
     cudaStreamSynchronize(h->c.side);
     for (int k = 0; k < 2 * 64; ++k)
@@ -112,6 +113,45 @@ int gptq_destroy(gptq_ctx* h) {
 const char* gptq_last_error(const gptq_ctx* h) { return h ? h->c.last_error.c_str() : ""; }
 
 uint64_t gptq_kernel_launches(const gptq_ctx* h) { return h ? h->c.launches : 0; }
+
+int gptq_set_wait_budget(gptq_ctx* h, int64_t cycles) {
+  if (!h) return GPTQ_ERR_ARG;
+  if (cycles < 0) GPTQ_SET_ERR(&h->c, GPTQ_ERR_ARG, "set_wait_budget: cycles < 0");
+  h->c.timeout_cycles = cycles == 0 ? gptq::kDefaultWaitCycles : (long long)cycles;
+  return GPTQ_OK;
+}
+
+int gptq_timing_enable(gptq_ctx* h, int on) {
+  if (!h) return GPTQ_ERR_ARG;
+  h->c.timing = on != 0;
+  if (on) {
+    h->c.timed.clear();
+    h->c.pool_used = 0;
+  }
+  return GPTQ_OK;
+}
+
+int gptq_timing_read(gptq_ctx* h, double* ms, int64_t* launches) {
+  if (!h || !ms || !launches) return GPTQ_ERR_ARG;
+  Ctx* c = &h->c;
+  for (int k = 0; k < GPTQ_NUM_STAGES; ++k) {
+    ms[k] = 0.0;
+    launches[k] = 0;
+  }
+  if (!c->timed.empty()) GPTQ_CUDA_CHECK(c, cudaEventSynchronize(c->timed.back().stop));
+  for (const gptq::TimedLaunch& t : c->timed) {
+    // a launch on the factorization's second stream may finish after the last one recorded
+    GPTQ_CUDA_CHECK(c, cudaEventSynchronize(t.stop));
+    float e = 0.f;
+    GPTQ_CUDA_CHECK(c, cudaEventElapsedTime(&e, t.start, t.stop));
+    const int k = (t.stage >= 0 && t.stage < GPTQ_NUM_STAGES) ? t.stage : GPTQ_STAGE_OTHER;
+    ms[k] += e;
+    launches[k] += 1;
+  }
+  c->timed.clear();
+  c->pool_used = 0;
+  return GPTQ_OK;
+}
 
 int gptq_sync_status(gptq_ctx* h) {
   if (!h) return GPTQ_ERR_ARG;
@@ -135,6 +175,7 @@ int gptq_hessian_accumulate(gptq_ctx* h, const void* Xc, int dtype, int64_t n_ch
       n_chunk > INT32_MAX || *n_total < 0)
     GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "hessian_accumulate: bad argument (d=%lld n_chunk=%lld)",
                  (long long)d, (long long)n_chunk);
+  gptq::StageScope stage(c, GPTQ_STAGE_HESSIAN);
   int rc = gptq::syrk_accumulate(c, Xc, dtype, n_chunk, (int)d, S, *n_total == 0);
   if (rc) return rc;
   *n_total += n_chunk;
@@ -156,6 +197,7 @@ int gptq_prepare_hinv(gptq_ctx* h, float* S, int64_t n_total, int64_t d, float p
   const int di = (int)d;
   const float scale = n_total > 0 ? (float)(2.0 / (double)n_total) : 1.f;
   const size_t dd = (size_t)d * d;
+  gptq::StageScope stage(c, GPTQ_STAGE_PREPARE);
   int rc;
   if ((rc = gptq::prep_diag(c, S, di, scale, diagv, dead))) return rc;
   if ((rc = gptq::prep_mean(c, diagv, di))) return rc;
@@ -232,11 +274,14 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   const bool pair_ws = cv.ok();
   if (!pair_ws) Ehi = Elo = Rhi = Rlo = nullptr;
   int rc;
+  gptq::StageScope stage(c, GPTQ_STAGE_GRID);  // restores the caller's stage on return
   // largest code: 2^b - 1, or 2 for the ternary grid
   const int maxq = (grid_given == 4) ? 2 : (1 << bits) - 1;
+  c->stage = GPTQ_STAGE_GRID;
   if ((grid_given == 0 || grid_given >= 3) &&
       (rc = gptq::grid_fit(c, W, w_dtype, mi, di, maxq, grid_given >= 3, group, scales, zeros)))
     return rc;
+  c->stage = GPTQ_STAGE_COLUMN;
   if ((rc = gptq::make_gcol(c, perm, di, group, dyn != 0, gcol, general ? inv : nullptr))) return rc;
   if ((rc = gptq::init_work(c, W, w_dtype, mi, di, perm, dead, !general, Wk))) return rc;
   // Two-level lazy blocks ([T] eq.(46); exact in exact arithmetic by eq.(47)-(49)): columns
@@ -251,16 +296,19 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
       const int nb = std::min(bk, s1 - i);
       const bool uniform = dyn || (group == -1) || (!general && (i / g) == ((i + nb - 1) / g));
       float* Et = E + (i - s0);
+      c->stage = GPTQ_STAGE_COLUMN;
       if ((rc = gptq::column_block(c, Wk, mi, di, i, nb, R, scales, zeros, ng, gcol, uniform,
                                    dyn, maxq, Et, Ehi ? Ehi + (i - s0) : nullptr,
                                    Elo ? Elo + (i - s0) : nullptr, gptq::kSuperCols, codes_p,
                                    loss_part)))
         return rc;
+      c->stage = GPTQ_STAGE_UPDATE;
       if ((rc = gptq::trailing_update(c, Wk, mi, di, i, nb, i + nb, s1, Et, gptq::kSuperCols, R)))
         return rc;
     }
     // tail: W[:, s1:] -= E R[s0:s1, s1:], on CTA pairs with split operands where it applies
     const int tn = di - s1, tk = s1 - s0;
+    c->stage = GPTQ_STAGE_UPDATE;
     if (tn > 0 && pair_ws && gptq::gemm_pair_applies(mi, tn, tk, Ehi, gptq::kSuperCols, Rhi, ldr,
                                                      c->num_sms)) {
       if ((rc = gptq::split_tf32(c, R + (long long)s0 * di + s1, di, tk, tn, Rhi, Rlo, ldr)))
@@ -272,6 +320,7 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
       return rc;
     }
   }
+  c->stage = GPTQ_STAGE_OUTPUT;
   if ((rc = gptq::loss_reduce(c, loss_part, parts, di, general ? loss_p : col_loss))) return rc;
   if (general &&
       (rc = gptq::unpermute(c, mi, di, inv, codes_p, Wk, loss_p, codes, W_hat, col_loss)))
@@ -285,6 +334,7 @@ int gptq_pack(gptq_ctx* h, const uint8_t* codes, int64_t m, int64_t d, int bits,
   Ctx* c = &h->c;
   if (!codes || !packed || m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || bits < 1 || bits > 8)
     GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "pack: bad argument");
+  gptq::StageScope stage(c, GPTQ_STAGE_PACK);
   return gptq::pack_codes(c, codes, (int)m, (int)d, bits, packed);
 }
 
@@ -294,6 +344,7 @@ int gptq_unpack(gptq_ctx* h, const uint32_t* packed, int64_t m, int64_t d, int b
   Ctx* c = &h->c;
   if (!codes || !packed || m < 1 || d < 1 || m > INT32_MAX || d > INT32_MAX || bits < 1 || bits > 8)
     GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "unpack: bad argument");
+  gptq::StageScope stage(c, GPTQ_STAGE_PACK);
   return gptq::unpack_codes(c, packed, (int)m, (int)d, bits, codes);
 }
 
@@ -314,6 +365,7 @@ int gptq_dequant_matmul(gptq_ctx* h, const void* X, int x_dtype, int64_t T, int6
                             ? (c->ws_bytes - gptq::kStatusBytes - 256) / 4
                             : 0;
   float* part = cv.take<float>(0);
+  gptq::StageScope stage(c, GPTQ_STAGE_DEQUANT);
   return gptq::dequant_matmul(c, X, x_dtype, (int)T, (int)d, packed, (int)m, bits, group,
                               group_id, (int)n_g, scales, zeros, Y, part, avail);
 }
@@ -332,6 +384,7 @@ int gptq_retile_codes(gptq_ctx* h, const uint32_t* packed, int64_t m, int64_t d,
       !al(packed) || !al(tiled))
     GPTQ_SET_ERR(c, GPTQ_ERR_ARG, "retile_codes: bad argument (m=%lld d=%lld)", (long long)m,
                  (long long)d);
+  gptq::StageScope stage(c, GPTQ_STAGE_DEQUANT);
   return gptq::retile_codes(c, packed, (int)m, (int)d, tiled);
 }
 
@@ -352,6 +405,7 @@ int gptq_dequant_matmul_tiled(gptq_ctx* h, const void* X, int x_dtype, int64_t T
                             ? (c->ws_bytes - gptq::kStatusBytes - 256) / 4
                             : 0;
   float* part = cv.take<float>(0);
+  gptq::StageScope stage(c, GPTQ_STAGE_DEQUANT);
   return gptq::dequant_matmul_tiled(c, X, x_dtype, (int)T, (int)d, tiled, (int)m, group,
                                     (int)n_g, scales, zeros, Y, part, avail);
 }
@@ -366,7 +420,10 @@ int gptq_twosided_factor(gptq_ctx* h, float* G, int64_t k) {
   if (!cv.ok())
     GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "twosided_factor: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
   int rc;
-  if ((rc = gptq::factor_inverse(c, G, (int)k, tmp))) return rc;
+  {
+    gptq::StageScope stage(c, GPTQ_STAGE_TWOSIDED);
+    if ((rc = gptq::factor_inverse(c, G, (int)k, tmp))) return rc;
+  }
   gptq::DeviceStatus st{};
   if ((rc = read_status(c, &st))) return rc;
   if (st.code == 0) return GPTQ_OK;
@@ -391,6 +448,7 @@ int gptq_twosided_round(gptq_ctx* h, const float* X, int64_t m, int64_t n, const
   float* RAT = cv.take<float>((size_t)m * m);
   if (!cv.ok())
     GPTQ_SET_ERR(c, GPTQ_ERR_NOMEM, "twosided_round: workspace %zu < %zu bytes", c->ws_bytes, cv.off);
+  gptq::StageScope stage(c, GPTQ_STAGE_TWOSIDED);
   return gptq::twosided_round(c, X, (int)m, (int)n, RA, RB, Z, eta, Y, C, etas, RAT);
 }
 

@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(DQ_THREADS)
   uint64_t* a_free = a_full + DQ_NA;
   uint64_t* d_full = a_free + DQ_NA;
   uint64_t* d_empty = d_full + Cfg::ND;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_empty + Cfg::ND);
+  uint64_t* drain = d_empty + Cfg::ND;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
       tc::mbar_init(&d_full[b], 1);
       tc::mbar_init(&d_empty[b], Cfg::EPW);
     }
+    tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
   }
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
         issued = j + 1;
       }
       for (int j = max(0, issued - Cfg::CST); j < issued; ++j)
-        if (!mbar_wait_sleep(&full_c[j % Cfg::CST], (uint32_t)(j / Cfg::CST) & 1u, budget))
+        if (!mbar_wait_sleep(&full_c[j % Cfg::CST], (uint32_t)(j / Cfg::CST) & 1u, kDrainCycles))
           raise_error(st, GPTQ_ERR_TIMEOUT, 42);
     }
   } else if (warp == 2) {
@@ -293,12 +295,13 @@ __global__ void __launch_bounds__(DQ_THREADS)
         issued = i + 1;
       }
       for (int i = max(0, issued - Cfg::XST); i < issued; ++i)
-        if (!mbar_wait_sleep(&full_x[i % Cfg::XST], (uint32_t)(i / Cfg::XST) & 1u, budget))
+        if (!mbar_wait_sleep(&full_x[i % Cfg::XST], (uint32_t)(i / Cfg::XST) & 1u, kDrainCycles))
           raise_error(st, GPTQ_ERR_TIMEOUT, 48);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
+      bool any = false;
       for (int i = 0; i < n && !*abort_flag; ++i) {
         const int s = i % Cfg::XST, a = i % DQ_NA, b = i % Cfg::ND;
         const uint32_t ph = (uint32_t)(i / Cfg::XST) & 1u;
@@ -318,9 +321,16 @@ __global__ void __launch_bounds__(DQ_THREADS)
           mma_f16_tmem_a(tmem + d_col + b * BN, tmem + a_col + a * DQ_A_COLS + kk * 8, bd,
                          p.idesc, kk > 0 ? 1u : 0u);
         }
+        any = true;
         tc::mma_commit(&empty_x[s]);
         tc::mma_commit(&a_free[a]);
         tc::mma_commit(&d_full[b]);
+      }
+      // every MMA has completed before TMEM is freed (after an abort the epilogue may not have
+      // waited for them)
+      if (any) {
+        tc::mma_commit(drain);
+        if (!mbar_wait_sleep(drain, 0, kDrainCycles)) raise_error(st, GPTQ_ERR_TIMEOUT, 49);
       }
     }
   } else if (warp < 3 + Cfg::DQW) {
@@ -353,7 +363,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
         const uint16_t u = *reinterpret_cast<const uint16_t*>(&hz);
         zz = (uint32_t)u | ((uint32_t)u << 16);
       }
-      if (within == 0 && !mbar_wait_sleep(&full_c[cs], cph, budget)) {
+      if (within == 0 && !__all_sync(0xffffffffu, mbar_wait_sleep(&full_c[cs], cph, budget))) {
         raise_error(st, GPTQ_ERR_TIMEOUT, 44);
         *abort_flag = 1;
         break;
@@ -371,7 +381,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
         if (lane == 0) tc::mbar_arrive(&empty_c[cs]);
       }
       // A buffer a was last read by the MMAs of step i - 4
-      if (i >= DQ_NA && !mbar_wait_sleep(&a_free[a], aph ^ 1u, budget)) {
+      if (i >= DQ_NA && !__all_sync(0xffffffffu, mbar_wait_sleep(&a_free[a], aph ^ 1u, budget))) {
         raise_error(st, GPTQ_ERR_TIMEOUT, 45);
         *abort_flag = 1;
         break;
@@ -412,7 +422,7 @@ __global__ void __launch_bounds__(DQ_THREADS)
       const float delta = delta_next;
       if (active && i + 1 < n)
         delta_next = srow[p.group_steps ? (k_begin + i + 1) / p.group_steps : 0];
-      if (!mbar_wait_sleep(&d_full[b], dph, budget)) {
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(&d_full[b], dph, budget))) {
         raise_error(st, GPTQ_ERR_TIMEOUT, 46);
         *abort_flag = 1;
         ok = false;

@@ -230,6 +230,7 @@ struct FactorRun {
   float* tmp;              // level buffers, consecutive
   cudaStream_t side;       // T2 = U12 R22 runs here, beside the left subtree
   cudaEvent_t ev[2 * 64];  // per level: U12 ready, T2 ready
+  int stage_base, stage_gemm, stage_copy;  // stages the launches are timed under
 };
 
 static int rec(FactorRun& f, int s, int e, int level, float* buf) {
@@ -238,9 +239,11 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   float* M = f.M;
   const int n = e - s;
   if (n <= FB) {
+    StageScope stage(c, f.stage_base);
     GPTQ_LAUNCH(c, k_factor_base, 1, FB_THREADS, FB_SMEM, M, ld, s, n, c->status);
     return GPTQ_OK;
   }
+  StageScope stage(c, f.stage_gemm);
   const int n1 = larger_child(n);  // < n for n > FB
   const int mid = s + n1, n2 = e - mid;
   float* U12 = buf;                                   // [n1 x n2]
@@ -277,6 +280,7 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   GemmArgs g4{n1, n2, n1, Ablk, ld, 1, T2, n2, 1, Rblk, ld, -1.f, 0.f, kAUpper};
   if ((rc = gemm_f32(c, g4))) return rc;
   // strict lower block of this level
+  c->stage = f.stage_copy;
   return copy2d(c, nullptr, 0, M + (long long)mid * ld + s, ld, n2, n1);
 }
 
@@ -295,6 +299,12 @@ int factor_inverse(Ctx* c, float* M, int d, float* tmp) {
   f.tmp = tmp;
   f.side = c->side;
   for (int k = 0; k < 2 * 64; ++k) f.ev[k] = c->ev[k];
+  // inside the hot path the factorization has stages of its own; for two-sided rounding's
+  // factors it stays under the caller's stage
+  const bool own = (c->stage == GPTQ_STAGE_PREPARE);
+  f.stage_base = own ? GPTQ_STAGE_FACTOR_BASE : c->stage;
+  f.stage_gemm = own ? GPTQ_STAGE_FACTOR_GEMM : c->stage;
+  f.stage_copy = own ? GPTQ_STAGE_FACTOR_COPY : c->stage;
   return rec(f, 0, d, 0, tmp);
 }
 

@@ -129,7 +129,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
       // drain: the leader's stage barriers count both CTAs' copies
       if (rank == 0)
         for (int s = 0; s < GP_STAGES; ++s)
-          if (issued[s] && !tc::mbar_wait_cluster(&full[s], issued_phase[s], budget))
+          if (issued[s] && !tc::mbar_wait_cluster(&full[s], issued_phase[s], kDrainCycles))
             raise_error(st, GPTQ_ERR_TIMEOUT, 32);
     }
   } else if (warp == 1) {
@@ -186,7 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
       }
       if (any) {
         tc::mma_commit_pair(drain);
-        if (!tc::mbar_wait(drain, 0, budget)) raise_error(st, GPTQ_ERR_TIMEOUT, 35);
+        if (!tc::mbar_wait(drain, 0, kDrainCycles)) raise_error(st, GPTQ_ERR_TIMEOUT, 35);
       }
     }
   } else {
@@ -203,7 +203,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
 #pragma unroll
       for (int u = 0; u < 128; ++u) m[u] = 0.f;
       for (int pp = 0; pp < nparts; ++pp) {
-        if (!tc::mbar_wait_cluster(&tfull[acc], acc_phase, budget)) {
+        if (!tc::mbar_wait_cluster_warp(&tfull[acc], acc_phase, budget)) {
           raise_error(st, GPTQ_ERR_TIMEOUT, 36);
           *abort_flag = 1;
           ok = false;
@@ -358,8 +358,10 @@ int gemm_pair(Ctx* c, int M, int N, int K, const float* Ah, const float* Al, lon
   const int npairs = std::min(p.num_tiles, c->num_sms / 2);
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           GP_SMEM));
+  // CTA pairs keep the default wait budget (a pair whose CTAs gave up at different stages could
+  // not drain every copy completing on the leader's barriers)
   GPTQ_LAUNCH(c, k_gemm_pair, 2 * npairs, GP_THREADS, GP_SMEM, mah, mal, mbh, mbl, p, c->status,
-              c->timeout_cycles);
+              kDefaultWaitCycles);
   return GPTQ_OK;
 }
 

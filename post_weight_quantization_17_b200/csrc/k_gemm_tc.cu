@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
   uint64_t* empty = conv + GT_STAGES;
   uint64_t* tfull = empty + GT_STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -86,6 +87,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       tc::mbar_init(&tfull[a], 1);
       tc::mbar_init(&tempty[a], 32 * GT_EPI_WARPS);
     }
+    tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
   }
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
         }
       }
       for (int s = 0; s < GT_STAGES; ++s)
-        if (issued[s] && !tc::mbar_wait(&full[s], issued_phase[s], budget))
+        if (issued[s] && !tc::mbar_wait(&full[s], issued_phase[s], kDrainCycles))
           raise_error(st, GPTQ_ERR_TIMEOUT, 12);
     }
   } else if (warp == 1) {
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
     if (lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
+      bool ok = true, any = false;
       for (int t = blockIdx.x; t < p.num_tiles && ok && !*abort_flag; t += gridDim.x) {
         int i0, j0, kbeg, kend;
         if (!gt_tile(p, t, i0, j0, kbeg, kend)) continue;
@@ -190,6 +192,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
               tc::mma_tf32(d_tmem, dah, dbl, p.idesc, 1u);
               tc::mma_tf32(d_tmem, dal, dbh, p.idesc, 1u);
             }
+            any = true;
             tc::mma_commit(&empty[stage]);
             if (++stage == GT_STAGES) {
               stage = 0;
@@ -203,6 +206,12 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
             acc_phase ^= 1;
           }
         }
+      }
+      // every MMA has completed before TMEM is freed (after an abort the epilogue may not have
+      // waited for them)
+      if (any) {
+        tc::mma_commit(drain);
+        if (!tc::mbar_wait(drain, 0, kDrainCycles)) raise_error(st, GPTQ_ERR_TIMEOUT, 16);
       }
     }
   } else if (warp < 2 + GT_CONV_WARPS) {
@@ -266,8 +275,8 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
 #pragma unroll
       for (int u = 0; u < 64; ++u) m[u] = 0.f;
       for (int kp = kbeg; kp < kend; kp += GT_KP) {
-        if (!tc::mbar_wait(&tfull[acc], acc_phase, budget)) {
-          raise_error(st, GPTQ_ERR_TIMEOUT, 16);
+        if (!tc::mbar_wait_warp(&tfull[acc], acc_phase, budget)) {
+          raise_error(st, GPTQ_ERR_TIMEOUT, 17);
           *abort_flag = 1;
           ok = false;
           break;

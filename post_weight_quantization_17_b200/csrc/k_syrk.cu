@@ -61,7 +61,8 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
   uint64_t* empty = full + SY_STAGES;
   uint64_t* tfull = empty + SY_STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
       tc::mbar_init(&tfull[a], 1);
       tc::mbar_init(&tempty[a], 32 * SY_EPI_WARPS);
     }
+    tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
   }
@@ -123,14 +125,14 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
       }
       // drain: every copy this thread issued has landed before the CTA may exit
       for (int s = 0; s < SY_STAGES; ++s)
-        if (issued[s] && !tc::mbar_wait(&full[s], issued_phase[s], budget))
+        if (issued[s] && !tc::mbar_wait(&full[s], issued_phase[s], kDrainCycles))
           raise_error(st, GPTQ_ERR_TIMEOUT, 2);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
+      bool ok = true, any = false;
       for (int t = blockIdx.x; t < num_tiles && ok && !*abort_flag; t += gridDim.x) {
         for (int p = 0; p < nparts && ok; ++p) {
           if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, budget)) {
@@ -159,6 +161,7 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
               const uint64_t bd = tc::sdesc_sw128(b0 + kk * 2048, SY_BOX_BYTES, 1024);
               tc::mma_f16(d_tmem, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
             }
+            any = true;
             tc::mma_commit(&empty[stage]);
             if (++stage == SY_STAGES) {
               stage = 0;
@@ -172,6 +175,12 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
             acc_phase ^= 1;
           }
         }
+      }
+      // every MMA has completed before TMEM is freed (after an abort the epilogue may not have
+      // waited for them)
+      if (any) {
+        tc::mma_commit(drain);
+        if (!tc::mbar_wait(drain, 0, kDrainCycles)) raise_error(st, GPTQ_ERR_TIMEOUT, 6);
       }
     }
   } else {
@@ -190,7 +199,7 @@ __global__ void __launch_bounds__(SY_THREADS, 1)
 #pragma unroll
       for (int u = 0; u < 128; ++u) m[u] = 0.f;
       for (int p = 0; p < nparts; ++p) {
-        if (!tc::mbar_wait(&tfull[acc], acc_phase, budget)) {
+        if (!tc::mbar_wait_warp(&tfull[acc], acc_phase, budget)) {
           raise_error(st, GPTQ_ERR_TIMEOUT, 5);
           *abort_flag = 1;
           ok = false;
@@ -375,7 +384,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
       // drain: the leader's stage barriers count both CTAs' copies
       if (rank == 0)
         for (int s = 0; s < S2_STAGES; ++s)
-          if (issued[s] && !tc::mbar_wait_cluster(&full[s], issued_phase[s], budget))
+          if (issued[s] && !tc::mbar_wait_cluster(&full[s], issued_phase[s], kDrainCycles))
             raise_error(st, GPTQ_ERR_TIMEOUT, 22);
     }
   } else if (warp == 1) {
@@ -430,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
       // every MMA of the pair has completed before either CTA may free TMEM or exit
       if (any) {
         tc::mma_commit_pair(drain);
-        if (!tc::mbar_wait(drain, 0, budget)) raise_error(st, GPTQ_ERR_TIMEOUT, 25);
+        if (!tc::mbar_wait(drain, 0, kDrainCycles)) raise_error(st, GPTQ_ERR_TIMEOUT, 25);
       }
     }
   } else {
@@ -449,7 +458,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
 #pragma unroll
       for (int u = 0; u < 128; ++u) m[u] = 0.f;
       for (int p = 0; p < nparts; ++p) {
-        if (!tc::mbar_wait_cluster(&tfull[acc], acc_phase, budget)) {
+        if (!tc::mbar_wait_cluster_warp(&tfull[acc], acc_phase, budget)) {
           raise_error(st, GPTQ_ERR_TIMEOUT, 27);
           *abort_flag = 1;
           ok = false;
@@ -558,9 +567,10 @@ int syrk_tc(Ctx* c, const void* X, int dtype, long long n, int d, float* S, bool
     GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_syrk_tc2,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM));
     const uint32_t idesc = tc::idesc_f32acc(fmt, true, true, 2 * S2_BM, S2_BN);
+    // a pair's two CTAs could give up at different stages, after which copies of one CTA that
+    // complete on the other's barriers could not all be drained: pairs keep the default budget
     GPTQ_LAUNCH(c, k_syrk_tc2, grid, SY_THREADS, S2_SMEM, map, S, d, (int)n, overwrite ? 0 : 1,
-                                                         num_tiles, idesc, c->status,
-                                                         c->timeout_cycles);
+                num_tiles, idesc, c->status, kDefaultWaitCycles);
     return GPTQ_OK;
   }
   const int nI = (d + SY_BM - 1) / SY_BM;

@@ -195,6 +195,16 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
   return true;
 }
+// Warp-uniform forms for warps that go on to warp-collective tcgen05 instructions: every lane
+// waits, and the warp proceeds only if all of them saw the phase complete, so a budget that runs
+// out on some lanes cannot split the warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, long long budget) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, budget));
+}
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t* bar, uint32_t parity,
+                                                       long long budget) {
+  return __all_sync(0xffffffffu, mbar_wait_cluster(bar, parity, budget));
+}
 // TMA tile load into this CTA's shared memory whose completion is counted on an mbarrier of
 // either CTA of the pair (`bar_cluster`: a shared::cluster address, e.g. the leader's barrier).
 // No multicast: each CTA loads only its own tiles from this GPU's memory.

@@ -38,6 +38,9 @@ def test_null_context_is_an_argument_error():
     assert L.gptq_twosided_factor(None, None, 4) == G.GPTQ_ERR_ARG
     assert L.gptq_twosided_round(None, None, 2, 2, None, None, None, None) == G.GPTQ_ERR_ARG
     assert L.gptq_sync_status(None) == G.GPTQ_ERR_ARG
+    assert L.gptq_set_wait_budget(None, 1) == G.GPTQ_ERR_ARG
+    assert L.gptq_timing_enable(None, 1) == G.GPTQ_ERR_ARG
+    assert L.gptq_timing_read(None, None, None) == G.GPTQ_ERR_ARG
     assert L.gptq_destroy(None) == G.GPTQ_ERR_ARG
     assert L.gptq_last_error(None) == b""
 

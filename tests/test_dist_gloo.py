@@ -47,5 +47,5 @@ def test_two_ranks_max_time_and_independent_layers():
 
 def test_weak_scaling_value():
     import bench
-    assert bench.weak_scaling_value(1, 4096, 4096, 0.01) == pytest.approx(4096 * 4096 / 0.01)
-    assert bench.weak_scaling_value(8, 4096, 4096, 0.02) == pytest.approx(8 * 4096 * 4096 / 0.02)
+    assert bench.weak_scaling_value(1, 4096 * 4096, 0.01) == pytest.approx(4096 * 4096 / 0.01)
+    assert bench.weak_scaling_value(8, 4096 * 4096, 0.02) == pytest.approx(8 * 4096 * 4096 / 0.02)

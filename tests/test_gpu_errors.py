@@ -91,6 +91,36 @@ def test_workspace_too_small():
         c.close()
 
 
+def test_wait_budget_runs_out_then_context_recovers():
+    """A pipeline wait that runs out: with a one-cycle wait budget the single-SM tensor path of
+    the Hessian (128 <= d < 256) gives up at its first wait that is not already satisfied, records
+    GPTQ_ERR_TIMEOUT, drains its own copies and tensor-core work, and frees its tensor memory.
+    With the default budget restored the same context computes the statistic correctly."""
+    c = G.Context(m_max=8, d_max=192, act_order=False)
+    try:
+        g = torch.Generator(device="cuda").manual_seed(7)
+        X = torch.randn(8192, 192, device="cuda", generator=g).to(torch.bfloat16)
+        S = torch.zeros(192, 192, device="cuda")
+        G.gptq_set_wait_budget(c, 1)
+        G.gptq_hessian_accumulate(c, X, S, 0)
+        with pytest.raises(G.GPTQError) as e:
+            G.gptq_sync_status(c)
+        assert e.value.code == G.GPTQ_ERR_TIMEOUT
+        G.gptq_set_wait_budget(c, 0)             # back to the default
+        n = G.gptq_hessian_accumulate(c, X, S, 0)
+        assert G.gptq_sync_status(c) == G.GPTQ_OK and n == 8192
+        Xd = X.double()
+        ref = torch.tril(Xd.T @ Xd)
+        err = (torch.tril(S).double() - ref).norm() / ref.norm()
+        assert err <= 1e-4, err
+        with pytest.raises(G.GPTQError) as e:
+            G.gptq_set_wait_budget(c, -1)
+        assert e.value.code == G.GPTQ_ERR_ARG
+        _context_still_works(c)
+    finally:
+        c.close()
+
+
 def _context_still_works(ctx):
     d = 16
     b = _bufs(8, d)

@@ -62,10 +62,10 @@ def test_noalloc_matches_gptq_quantize_layer_on_two_calls():
             torch.cuda.synchronize()
             assert torch.equal(out["scales"], ref["scales"]), f"call {call}: scales"
             assert torch.equal(out["zeros"], ref["zeros"]), f"call {call}: zeros"
-            codes_same = (out["codes"] == ref["codes"]).float().mean().item()
-            assert codes_same >= P.TOL_CODES_IDENTICAL, f"call {call}: codes {codes_same}"
-            assert P.rel_fro(out["W_hat"].cpu().numpy(), ref["W_hat"].cpu().numpy()) <= P.TOL_WHAT
-            assert P.rel_fro(out["col_loss"].cpu().numpy(), ref["col_loss"].cpu().numpy()) <= 1e-3
+            # both entry points run the same kernels on the same bytes: bit-equal outputs
+            assert torch.equal(out["codes"], ref["codes"]), f"call {call}: codes"
+            assert torch.equal(out["W_hat"], ref["W_hat"]), f"call {call}: W_hat"
+            assert torch.equal(out["col_loss"], ref["col_loss"]), f"call {call}: col_loss"
     finally:
         ctx.close()
 
