@@ -193,7 +193,7 @@ int gptq_quantize_layer(gptq_ctx* ctx, const void* W, int w_dtype, int64_t m, in
  * gptq_quantize_layer.
  *   cuda_stream  the cudaStream_t to enqueue on (NULL = legacy default stream), current device.
  *   other arguments exactly as for gptq_quantize_layer.
- * The scratch must hold about 4 m (512 + d / 32) + 12 d bytes, plus 5 m d bytes when perm is
+ * The scratch must hold about 4 m (1024 + d / 48) + 12 d bytes, plus 5 m d bytes when perm is
  * not NULL; a layer that needs more returns GPTQ_ERR_ARG (the only work enqueued then clears
  * the scratch's status word).
  * Device memory: under CUDA's lazy module loading the array is reserved on a device when the

@@ -333,27 +333,34 @@ def gptq_lazy(Wp, R, scale, zero, gcol, bits: int, block: int, dynamic: int = 0,
     loss = np.zeros(d, np.float64)
     for i in range(0, d, block):
         i2 = min(i + block, d)
-        E = np.zeros((m, i2 - i), np.float64)
+        # the block's columns as rows (Wb[t] = W[:, i + t]), so that a column is contiguous;
+        # E likewise (Eb[t] = η of column i + t)
+        Wb = W[:, i:i2].T.copy()
+        Eb = np.zeros((i2 - i, m), np.float64)
         for j in range(i, i2):
+            t = j - i
+            if dynamic > 0 and j % dynamic == 0:
+                W[:, i:i2] = Wb.T                        # the refit reads the current columns
             _dynamic_refit(W, j, dynamic, bits, scale, zero)
-            c, q, _ = quantize(W[:, j], scale[:, gcol[j]], zero[:, gcol[j]], bits, maxq)
-            rho = W[:, j] - q
+            c, q, _ = quantize(Wb[t], scale[:, gcol[j]], zero[:, gcol[j]], bits, maxq)
+            rho = Wb[t] - q
             eta = rho / R[j, j]
             loss[j] = float(np.sum(rho ** 2)) / (2.0 * R[j, j] ** 2)
             codes[:, j] = c
             Q[:, j] = q
-            E[:, j - i] = eta
-            W[:, j:i2] -= np.outer(eta, R[j, j:i2])
-        W[:, i2:] -= E @ R[i:i2, i2:]
+            Eb[t] = eta
+            Wb[t:] -= R[j, j:i2, None] * eta[None, :]   # [T] eq.(42) inside the block
+        W[:, i:i2] = Wb.T
+        W[:, i2:] -= Eb.T @ R[i:i2, i2:]                 # [T] eq.(46)
     return codes, Q, loss
 
 
 def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: float = 1e-3,
-                    dynamic: int = 0, other_zero=None, maxq=None):
+                    dynamic: int = 0, other_zero=None, maxq=None, block: int = 0):
     """Check another implementation's codes against this recursion, decision by decision.
 
-    Runs the unblocked Cholesky-form recursion ([T] eq.(42)) in fp64 on the same inputs, but at
-    every (row, column) it follows `other_codes`.  A decision that differs from this oracle's
+    Runs the Cholesky-form recursion ([T] eq.(42)) in fp64 on the same inputs, but at every
+    (row, column) it follows `other_codes`.  A decision that differs from this oracle's
     rounding is accepted iff the two codes are adjacent and the oracle's pre-round value w/Δ
     lies within `band` (in units of Δ) of the rounding boundary between them; otherwise it is
     a violation.  Several outputs are correct near a boundary, so the decisions that are
@@ -362,28 +369,40 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
     Along the replayed decisions it also records Ŵ (replay_Q) and the per-column loss
     Σ_r ρ² / (2 R_jj²) ([T] eq.(43)), which are the oracle's values for those decisions.
 
+    block = 0: unblocked, every column's update applied to all later columns at once.  block = B:
+    the lazy-block form of [W] Algorithm 1 / [T] §10: updates inside a block of B columns, then
+    W[:, i2:] -= E R[i:i2, i2:] ([T] eq.(46)); equal in exact arithmetic ([T] eq.(47)-(49)).  In
+    that form R is read one block of rows at a time, so it may be given in fp32 (each block's rows
+    are promoted to fp64 when used).
+
     dynamic = g > 0: the grid is refitted at group starts from the replay's own working
     weights (scale / zero are overwritten), as in `gptq_explicit`.  With `other_zero` (the other
     implementation's zero points, [m, n_groups]) the integer zero point is a decision too: the
     replay follows the other's z, accepting a difference iff the two are adjacent and the
     replay's pre-round value -x_min / Δ lies within `band` of the boundary between them; Δ
-    stays the replay's own.
+    stays the replay's own.  With block > 0 a group must start on a block start or lie inside
+    one block.
 
     Returns dict(n, identical, in_band, violations, max_excess, replay_Q, replay_loss,
     rows_with_flips, grid_in_band, grid_violations).
     """
+    if block and dynamic > 0 and dynamic % block != 0 and block % dynamic != 0:
+        raise ValueError("dynamic groups must start on block starts or lie inside a block")
     W = np.array(Wp, dtype=np.float64, copy=True)
-    R = np.asarray(R, np.float64)
+    if not block:
+        R = np.asarray(R, np.float64)
     other = np.asarray(other_codes, np.int64)
     m, d = W.shape
     maxq = _code_max(bits, maxq)
-    identical = in_band = violations = 0
-    max_excess = 0.0
+    st = dict(identical=0, in_band=0, violations=0, max_excess=0.0, grid_in_band=0,
+              grid_violations=0)
     Qr = np.zeros((m, d), np.float64)
     loss = np.zeros(d, np.float64)
     flipped = np.zeros(m, bool)
-    grid_in_band = grid_violations = 0
-    for j in range(d):
+
+    def decide(j, r_jj, wj):
+        """Column j (current values wj): follow the other implementation's decision, record
+        it, return η."""
         _dynamic_refit(W, j, dynamic, bits, scale, zero)
         if dynamic > 0 and other_zero is not None and j % dynamic == 0:
             k = j // dynamic
@@ -398,37 +417,58 @@ def decision_replay(Wp, R, scale, zero, gcol, bits: int, other_codes, band: floa
                 lo = np.minimum(z_o, z_g)[zdiff]
                 dist = np.abs(t[zdiff].astype(np.float64) - (lo + 0.5))
                 ok = (np.abs(z_o - z_g)[zdiff] == 1) & (dist <= band)
-                grid_in_band += int(np.sum(ok))
-                grid_violations += int(np.sum(~ok))
+                st["grid_in_band"] += int(np.sum(ok))
+                st["grid_violations"] += int(np.sum(~ok))
             zero[:, k] = z_g
         delta = np.asarray(scale[:, gcol[j]], np.float32)
         z = np.asarray(zero[:, gcol[j]], np.int64)
-        c_o, _, u = quantize(W[:, j], delta, z, bits, maxq)
+        c_o, _, u = quantize(wj, delta, z, bits, maxq)
         c_g = other[:, j]
         same = c_o == c_g
-        identical += int(np.sum(same))
+        st["identical"] += int(np.sum(same))
         diff = ~same
-        flipped |= diff
+        flipped[diff] = True
         if np.any(diff):
             lo = np.minimum(c_o[diff], c_g[diff])
             adjacent = np.abs(c_o[diff] - c_g[diff]) == 1
             boundary = (lo - z[diff]).astype(np.float64) + 0.5
             dist = np.abs(u[diff].astype(np.float64) - boundary)
             ok = adjacent & (dist <= band) & (lo >= 0) & (lo + 1 <= maxq)
-            in_band += int(np.sum(ok))
-            violations += int(np.sum(~ok))
+            st["in_band"] += int(np.sum(ok))
+            st["violations"] += int(np.sum(~ok))
             if np.any(~ok):
-                max_excess = max(max_excess, float(np.max(dist[~ok])))
+                st["max_excess"] = max(st["max_excess"], float(np.max(dist[~ok])))
         cg = np.clip(c_g, 0, maxq)
         q = (delta * (cg - z).astype(np.float32)).astype(np.float32).astype(np.float64)
-        rho = W[:, j] - q
-        eta = rho / R[j, j]
-        loss[j] = float(np.sum(rho ** 2)) / (2.0 * R[j, j] ** 2)
-        W[:, j:] -= np.outer(eta, R[j, j:])
+        rho = wj - q
+        loss[j] = float(np.sum(rho ** 2)) / (2.0 * r_jj ** 2)
         Qr[:, j] = q
-    return dict(n=m * d, identical=identical, in_band=in_band, violations=violations,
-                max_excess=max_excess, replay_Q=Qr, replay_loss=loss, rows_with_flips=flipped,
-                grid_in_band=grid_in_band, grid_violations=grid_violations)
+        return rho / r_jj
+
+    if not block:
+        for j in range(d):
+            eta = decide(j, R[j, j], W[:, j])
+            W[:, j:] -= np.outer(eta, R[j, j:])
+    else:
+        for i in range(0, d, block):
+            i2 = min(i + block, d)
+            Rb = np.asarray(R[i:i2, i:], np.float64)     # this block's rows, columns i..d-1
+            # the block's columns as rows (Wb[t] = W[:, i + t]); η likewise
+            Wb = W[:, i:i2].T.copy()
+            Eb = np.zeros((i2 - i, m), np.float64)
+            for j in range(i, i2):
+                t = j - i
+                if dynamic > 0 and j % dynamic == 0:
+                    W[:, i:i2] = Wb.T                    # the refit reads the current columns
+                eta = decide(j, Rb[t, t], Wb[t])
+                Eb[t] = eta
+                Wb[t:] -= Rb[t, t:i2 - i, None] * eta[None, :]
+            W[:, i:i2] = Wb.T
+            W[:, i2:] -= Eb.T @ Rb[:, i2 - i:]
+    return dict(n=m * d, identical=st["identical"], in_band=st["in_band"],
+                violations=st["violations"], max_excess=st["max_excess"], replay_Q=Qr,
+                replay_loss=loss, rows_with_flips=flipped, grid_in_band=st["grid_in_band"],
+                grid_violations=st["grid_violations"])
 
 
 # --------------------------------------------------------------------------------------------

@@ -23,6 +23,7 @@ struct GemmArgs {
   float* C; long long ldc;
   float alpha, beta;
   int flags;
+  int partial_k;  // tensor path: k-elements per TMEM partial (multiple of 32; 0: 128)
 };
 
 constexpr int GBK = 8, GTHREADS = 256;

@@ -202,8 +202,9 @@ int gptq_prepare_hinv(gptq_ctx* h, float* S, int64_t n_total, int64_t d, float p
   if ((rc = gptq::prep_diag(c, S, di, scale, diagv, dead))) return rc;
   if ((rc = gptq::prep_mean(c, diagv, di))) return rc;
   if ((rc = gptq::prep_perm(c, diagv, di, act_order, perm))) return rc;
-  if ((rc = gptq::prep_build(c, S, di, scale, diagv, perm, !act_order, R))) return rc;
-  if ((rc = gptq::prep_copy(c, R, S, dd))) return rc;
+  bool wrote_S = false;
+  if ((rc = gptq::prep_build(c, S, di, scale, diagv, perm, !act_order, R, &wrote_S))) return rc;
+  if (!wrote_S && (rc = gptq::prep_copy(c, R, S, dd))) return rc;
   float pd = percdamp;
   for (int attempt = 0; attempt <= 3; ++attempt) {
     if (attempt > 0 && (rc = gptq::prep_copy(c, S, R, dd))) return rc;
@@ -286,8 +287,9 @@ int gptq_quantize_layer(gptq_ctx* h, const void* W, int w_dtype, int64_t m, int6
   if ((rc = gptq::init_work(c, W, w_dtype, mi, di, perm, dead, !general, Wk))) return rc;
   // Two-level lazy blocks ([T] eq.(46); exact in exact arithmetic by eq.(47)-(49)): columns
   // are quantized in tiles of bk <= 128; after a tile only the rest of its super-block of
-  // sb = 4 bk columns is updated, and after a super-block one GEMM with K = sb updates the
-  // remaining tail.
+  // sb = 8 bk columns is updated, and after a super-block one GEMM with K = sb updates the
+  // remaining tail (a long K, so that the tail GEMM's read-modify-write of W is small beside
+  // its products).
   const int bk = std::min(block, gptq::kColMax);
   const int sb = bk * (gptq::kSuperCols / gptq::kColMax);
   for (int s0 = 0; s0 < di; s0 += sb) {

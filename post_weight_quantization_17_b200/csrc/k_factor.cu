@@ -16,6 +16,8 @@
 // inverted inside one CTA, in registers.  T2 = U12 R22 needs only the right subtree, so it runs on a second
 // stream beside the left subtree's factorization.  A non-positive or non-finite pivot raises GPTQ_ERR_NOT_PD /
 // GPTQ_ERR_NONFINITE in the device status word (the host retries with more damping).
+#include <algorithm>
+
 #include "kernels.h"
 #include "gemm_simt.cuh"
 
@@ -185,24 +187,34 @@ __global__ void __launch_bounds__(FB_THREADS, 1) k_factor_base(float* __restrict
   }
 }
 
+// dst[rows x cols] = src (or 0 when src is null).  Grid: x over 1024-column slices of a row (256
+// threads, 4 columns each), y over rows (grid-strided); 16-byte accesses when rows are aligned.
 __global__ void k_copy2d(const float* __restrict__ src, long long lds, float* __restrict__ dst,
-                         long long ldd, int rows, int cols) {
+                         long long ldd, int rows, int cols, int vec) {
   pdl_wait();
   pdl_release();
-  long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  long long total = (long long)rows * cols;
-  for (; e < total; e += (long long)gridDim.x * blockDim.x) {
-    int r = (int)(e / cols), k = (int)(e % cols);
-    dst[(long long)r * ldd + k] = src ? src[(long long)r * lds + k] : 0.f;
+  const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (c0 >= cols) return;
+  for (int r = blockIdx.y; r < rows; r += gridDim.y) {
+    float* d = dst + (long long)r * ldd + c0;
+    const float* s = src ? src + (long long)r * lds + c0 : nullptr;
+    if (vec && c0 + 4 <= cols) {
+      *reinterpret_cast<float4*>(d) =
+          s ? *reinterpret_cast<const float4*>(s) : make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      for (int u = 0; u < 4 && c0 + u < cols; ++u) d[u] = s ? s[u] : 0.f;
+    }
   }
 }
 
 static int copy2d(Ctx* c, const float* src, long long lds, float* dst, long long ldd, int rows,
                   int cols) {
-  long long total = (long long)rows * cols;
-  if (total <= 0) return GPTQ_OK;
-  int blocks = (int)std::min<long long>((total + 255) / 256, (long long)c->num_sms * 16);
-  GPTQ_LAUNCH(c, k_copy2d, blocks, 256, 0, src, lds, dst, ldd, rows, cols);
+  if (rows <= 0 || cols <= 0) return GPTQ_OK;
+  auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  const int vec = (ldd % 4 == 0) && al(dst) && (!src || ((lds % 4 == 0) && al(src)));
+  const int gx = (cols + 1023) / 1024;
+  const int gy = std::min(rows, std::max(1, c->num_sms * 16 / gx));
+  GPTQ_LAUNCH(c, k_copy2d, dim3(gx, gy), 256, 0, src, lds, dst, ldd, rows, cols, vec);
   return GPTQ_OK;
 }
 
@@ -217,11 +229,28 @@ static size_t level_floats(int n) {
 // (the right one has n - larger_child(n) <= n/2 columns) and smaller than n for n > FB.
 static int larger_child(int n) { return (((n + 1) / 2 + FB - 1) / FB) * FB; }
 
-size_t factor_tmp_floats(int d) {
-  size_t total = 0;
-  for (int n = d; n > FB; n = larger_child(n)) total += 2 * level_floats(n);
-  return total + 64;
+// Nodes whose right child has at least this many columns run their four products on CTA pairs
+// (k_gemm_pair) with operands split into tf32 halves beforehand; the rest on k_gemm_tc /
+// k_gemm_small.  The pair path needs 16-byte aligned rows (ld and n2 multiples of 4).
+constexpr int kFactorPairMin = 512;
+static bool pair_node(int n2, long long ld) {
+  return n2 >= kFactorPairMin && n2 % 4 == 0 && ld % 4 == 0;
 }
+// A pair node's buffers: the halves of B (later of R11: n1 x n1), of R22, of U12 and of T2.
+static size_t pair_level_floats(int n1, int n2) {
+  return 2 * (size_t)n1 * n1 + 2 * (size_t)n2 * n2 + 4 * (size_t)n1 * n2;
+}
+
+// Scratch of the recursion below a node of n columns: its own level's buffers, then (one child
+// at a time) the children's.
+static size_t node_floats(int n, long long ld) {
+  if (n <= FB) return 0;
+  const int n1 = larger_child(n), n2 = n - n1;
+  const size_t own = pair_node(n2, ld) ? pair_level_floats(n1, n2) : 2 * level_floats(n);
+  return own + std::max(node_floats(n1, ld), node_floats(n2, ld));
+}
+
+size_t factor_tmp_floats(int d) { return node_floats(d, d) + 64; }
 
 struct FactorRun {
   Ctx* c;
@@ -231,7 +260,89 @@ struct FactorRun {
   cudaStream_t side;       // T2 = U12 R22 runs here, beside the left subtree
   cudaEvent_t ev[2 * 64];  // per level: U12 ready, T2 ready
   int stage_base, stage_gemm, stage_copy;  // stages the launches are timed under
+  bool pair;                               // large nodes on CTA pairs (k_gemm_pair)
 };
+
+static int rec(FactorRun& f, int s, int e, int level, float* buf);
+
+// A node on CTA pairs: the same four products as below, with the operands split into tf32
+// halves first (B and R22 before the right child's results are used, R11 after the left child),
+// and U12 and T2 written by their products directly as halves, since they are only operands.
+static int rec_pair(FactorRun& f, int s, int e, int level, float* buf) {
+  Ctx* c = f.c;
+  const long long ld = f.ld;
+  float* M = f.M;
+  const int n = e - s, n1 = larger_child(n), mid = s + n1, n2 = e - mid;
+  float* Bh = buf;                                  // B's halves, later R11's (n1 x n1)
+  float* Bl = Bh + (size_t)n1 * n1;
+  float* R22h = Bl + (size_t)n1 * n1;
+  float* R22l = R22h + (size_t)n2 * n2;
+  float* U12h = R22l + (size_t)n2 * n2;
+  float* U12l = U12h + (size_t)n1 * n2;
+  float* T2h = U12l + (size_t)n1 * n2;
+  float* T2l = T2h + (size_t)n1 * n2;
+  float* next = T2l + (size_t)n1 * n2;
+  int rc = rec(f, mid, e, level + 1, next);
+  if (rc) return rc;
+  const float* Bblk = M + (long long)s * ld + mid;   // rows s..mid, cols mid..e (H_λ)
+  float* Rblk = M + (long long)s * ld + mid;         // becomes R12
+  const float* R22 = M + (long long)mid * ld + mid;
+  float* Ablk = M + (long long)s * ld + s;
+  StageScope stage(c, f.stage_copy);
+  if ((rc = split_tf32(c, Bblk, ld, n1, n2, Bh, Bl, n2))) return rc;
+  if ((rc = split_tf32(c, R22, ld, n2, n2, R22h, R22l, n2))) return rc;
+  c->stage = f.stage_gemm;
+  // U12 = B R22^T: opB(k, j) = R22[j][k] (K-major), zero for k < j
+  GemmPairArgs g{};
+  g.M = n1; g.N = n2; g.K = n2;
+  g.Ah = Bh; g.Al = Bl; g.lda = n2;
+  g.Bh = R22h; g.Bl = R22l; g.ldb = n2; g.b_kmajor = true;
+  g.Ch = U12h; g.Cl = U12l; g.ldc = n2; g.alpha = 1.f; g.beta = 0.f; g.flags = kBLower;
+  g.partial_k = kFactorPartialK;
+  if ((rc = gemm_pair(c, g))) return rc;
+  // A' = A - U12 U12^T, tiles touching the upper triangle
+  GemmPairArgs g2{};
+  g2.M = n1; g2.N = n1; g2.K = n2;
+  g2.Ah = U12h; g2.Al = U12l; g2.lda = n2;
+  g2.Bh = U12h; g2.Bl = U12l; g2.ldb = n2; g2.b_kmajor = true;
+  g2.C = Ablk; g2.ldc = ld; g2.alpha = -1.f; g2.beta = 1.f; g2.flags = kCUpper;
+  g2.partial_k = kFactorPartialK;
+  if ((rc = gemm_pair(c, g2))) return rc;
+  // T2 = U12 R22 (R22(k, j) = 0 for k > j) on the side stream, beside the left subtree
+  cudaEvent_t ev_u = f.ev[2 * level], ev_t = f.ev[2 * level + 1];
+  GPTQ_CUDA_CHECK(c, cudaEventRecord(ev_u, c->stream));
+  GPTQ_CUDA_CHECK(c, cudaStreamWaitEvent(f.side, ev_u, 0));
+  {
+    cudaStream_t main = c->stream;
+    c->stream = f.side;
+    GemmPairArgs g3{};
+    g3.M = n1; g3.N = n2; g3.K = n2;
+    g3.Ah = U12h; g3.Al = U12l; g3.lda = n2;
+    g3.Bh = R22h; g3.Bl = R22l; g3.ldb = n2; g3.b_kmajor = false;
+    g3.Ch = T2h; g3.Cl = T2l; g3.ldc = n2; g3.alpha = 1.f; g3.beta = 0.f; g3.flags = kBUpper;
+    g3.partial_k = kFactorPartialK;
+    rc = gemm_pair(c, g3);
+    c->stream = main;
+    if (rc) return rc;
+  }
+  GPTQ_CUDA_CHECK(c, cudaEventRecord(ev_t, f.side));
+  if ((rc = rec(f, s, mid, level + 1, next))) return rc;
+  GPTQ_CUDA_CHECK(c, cudaStreamWaitEvent(c->stream, ev_t, 0));
+  // R12 = -R11 T2 (R11(i, k) = 0 for k < i)
+  c->stage = f.stage_copy;
+  if ((rc = split_tf32(c, Ablk, ld, n1, n1, Bh, Bl, n1))) return rc;
+  c->stage = f.stage_gemm;
+  GemmPairArgs g4{};
+  g4.M = n1; g4.N = n2; g4.K = n1;
+  g4.Ah = Bh; g4.Al = Bl; g4.lda = n1;
+  g4.Bh = T2h; g4.Bl = T2l; g4.ldb = n2; g4.b_kmajor = false;
+  g4.C = Rblk; g4.ldc = ld; g4.alpha = -1.f; g4.beta = 0.f; g4.flags = kAUpper;
+  g4.partial_k = kFactorPartialK;
+  if ((rc = gemm_pair(c, g4))) return rc;
+  // strict lower block of this level
+  c->stage = f.stage_copy;
+  return copy2d(c, nullptr, 0, M + (long long)mid * ld + s, ld, n2, n1);
+}
 
 static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   Ctx* c = f.c;
@@ -243,6 +354,7 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
     GPTQ_LAUNCH(c, k_factor_base, 1, FB_THREADS, FB_SMEM, M, ld, s, n, c->status);
     return GPTQ_OK;
   }
+  if (f.pair && pair_node(n - larger_child(n), ld)) return rec_pair(f, s, e, level, buf);
   StageScope stage(c, f.stage_gemm);
   const int n1 = larger_child(n);  // < n for n > FB
   const int mid = s + n1, n2 = e - mid;
@@ -256,10 +368,10 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   const float* R22 = M + (long long)mid * ld + mid;
   float* Ablk = M + (long long)s * ld + s;
   // U12 = B R22^T  (opB(k,j) = R22[j][k], zero for k < j)
-  GemmArgs g{n1, n2, n2, Bblk, ld, 1, R22, 1, ld, U12, n2, 1.f, 0.f, kBLower};
+  GemmArgs g{n1, n2, n2, Bblk, ld, 1, R22, 1, ld, U12, n2, 1.f, 0.f, kBLower, kFactorPartialK};
   if ((rc = gemm_f32(c, g))) return rc;
   // A' = A - U12 U12^T  (upper tiles only)
-  GemmArgs g2{n1, n1, n2, U12, n2, 1, U12, 1, n2, Ablk, ld, -1.f, 1.f, kCUpper};
+  GemmArgs g2{n1, n1, n2, U12, n2, 1, U12, 1, n2, Ablk, ld, -1.f, 1.f, kCUpper, kFactorPartialK};
   if ((rc = gemm_f32(c, g2))) return rc;
   // T2 = U12 R22 (R22(k,j) = 0 for k > j) on the side stream, beside the left subtree
   cudaEvent_t ev_u = f.ev[2 * level], ev_t = f.ev[2 * level + 1];
@@ -268,7 +380,7 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   {
     cudaStream_t main = c->stream;
     c->stream = f.side;
-    GemmArgs g3{n1, n2, n2, U12, n2, 1, R22, ld, 1, T2, n2, 1.f, 0.f, kBUpper};
+    GemmArgs g3{n1, n2, n2, U12, n2, 1, R22, ld, 1, T2, n2, 1.f, 0.f, kBUpper, kFactorPartialK};
     rc = gemm_f32(c, g3);
     c->stream = main;
     if (rc) return rc;
@@ -277,7 +389,7 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   if ((rc = rec(f, s, mid, level + 1, next))) return rc;
   GPTQ_CUDA_CHECK(c, cudaStreamWaitEvent(c->stream, ev_t, 0));
   // R12 = -R11 T2  (R11(i,k) = 0 for k < i)
-  GemmArgs g4{n1, n2, n1, Ablk, ld, 1, T2, n2, 1, Rblk, ld, -1.f, 0.f, kAUpper};
+  GemmArgs g4{n1, n2, n1, Ablk, ld, 1, T2, n2, 1, Rblk, ld, -1.f, 0.f, kAUpper, kFactorPartialK};
   if ((rc = gemm_f32(c, g4))) return rc;
   // strict lower block of this level
   c->stage = f.stage_copy;
@@ -305,6 +417,8 @@ int factor_inverse(Ctx* c, float* M, int d, float* tmp) {
   f.stage_base = own ? GPTQ_STAGE_FACTOR_BASE : c->stage;
   f.stage_gemm = own ? GPTQ_STAGE_FACTOR_GEMM : c->stage;
   f.stage_copy = own ? GPTQ_STAGE_FACTOR_COPY : c->stage;
+  f.pair = c->num_sms >= 2 && (reinterpret_cast<uintptr_t>(M) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(tmp) & 15) == 0;
   return rec(f, 0, d, 0, tmp);
 }
 

@@ -9,8 +9,9 @@
 // accumulator (relative error ~2^-21 per product, against 2^-11 for plain TF32; clearing the
 // low bits instead of rounding would double the error that the factorization's conditioning
 // then amplifies).  The tensor
-// core's accumulation over many MMAs loses low bits, so partial sums of KP = 128 k-elements are
-// taken from TMEM and added in fp32 into a register accumulator by the epilogue warps.
+// core rounds its fp32 accumulator toward zero at every MMA, so partial sums of kp k-elements
+// (128 by default, 32 in the factorization) are taken from TMEM and added in fp32 into a
+// register accumulator by the epilogue warps.
 //   warp 0       TMA producer: A box 128 x 32, B box 128 x 32 (K-major) or 4 x (32 x 32)
 //                (N-major), 128-byte swizzle (32-byte atoms for the N-major tf32 operand, the
 //                only smem layout the tensor core takes for it), 3-stage ring
@@ -27,7 +28,7 @@
 
 namespace gptq {
 
-constexpr int GT_BM = 128, GT_BN = 128, GT_BK = 32, GT_STAGES = 3, GT_KP = 128;
+constexpr int GT_BM = 128, GT_BN = 128, GT_BK = 32, GT_STAGES = 3;
 constexpr int GT_TILE_BYTES = GT_BM * GT_BK * 4;  // 16 KB: one fp32 operand tile
 constexpr int GT_STAGE_BYTES = 4 * GT_TILE_BYTES;  // A hi, A lo, B hi, B lo
 constexpr int GT_SMEM = GT_STAGES * GT_STAGE_BYTES + 1024 + 256;
@@ -41,14 +42,25 @@ struct GemmTcParams {
   float alpha, beta;
   int flags;
   int b_nmajor;
-  int tiles_n, num_tiles;
+  int tiles_m, tiles_n, num_tiles;
+  int kp;  // k-elements per TMEM partial
   uint32_t idesc;
 };
 
+// Tiles are visited in groups of GT_GROUP tile rows, column by column inside a group, so that
+// the ~148 tiles of one wave form a near-square block (16 rows x ~9 columns) and share their A
+// row slabs and B column slabs through L2; in plain row-major order a wave of a wide product
+// spans one tile row and ~148 columns, and every B slab then streams from HBM.
+constexpr int GT_GROUP = 16;
+
 __device__ __forceinline__ bool gt_tile(const GemmTcParams& p, int t, int& i0, int& j0, int& kbeg,
                                         int& kend) {
-  i0 = (t / p.tiles_n) * GT_BM;
-  j0 = (t % p.tiles_n) * GT_BN;
+  const int group = t / (GT_GROUP * p.tiles_n);
+  const int first = group * GT_GROUP;
+  const int rows = min(GT_GROUP, p.tiles_m - first);
+  const int local = t - group * GT_GROUP * p.tiles_n;
+  i0 = (first + local % rows) * GT_BM;
+  j0 = (local / rows) * GT_BN;
   if ((p.flags & kCUpper) && i0 > j0 + GT_BN - 1) return false;
   if ((p.flags & kCLower) && j0 > i0 + GT_BM - 1) return false;
   kbeg = 0;
@@ -152,7 +164,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       for (int t = blockIdx.x; t < p.num_tiles && ok && !*abort_flag; t += gridDim.x) {
         int i0, j0, kbeg, kend;
         if (!gt_tile(p, t, i0, j0, kbeg, kend)) continue;
-        for (int kp = kbeg; kp < kend && ok; kp += GT_KP) {
+        for (int kp = kbeg; kp < kend && ok; kp += p.kp) {
           if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, budget)) {
             raise_error(st, GPTQ_ERR_TIMEOUT, 13);
             *abort_flag = 1;
@@ -161,7 +173,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
           }
           tc::fence_after_sync();
           const uint32_t d_tmem = tmem + acc * GT_BN;
-          const int kp1 = min(kend, kp + GT_KP);
+          const int kp1 = min(kend, kp + p.kp);
           for (int k0 = kp; k0 < kp1; k0 += GT_BK) {
             if (!tc::mbar_wait(&conv[stage], phase, budget)) {
               raise_error(st, GPTQ_ERR_TIMEOUT, 14);
@@ -274,7 +286,7 @@ __global__ void __launch_bounds__(GT_THREADS, 1)
       float m[64];
 #pragma unroll
       for (int u = 0; u < 64; ++u) m[u] = 0.f;
-      for (int kp = kbeg; kp < kend; kp += GT_KP) {
+      for (int kp = kbeg; kp < kend; kp += p.kp) {
         if (!tc::mbar_wait_warp(&tfull[acc], acc_phase, budget)) {
           raise_error(st, GPTQ_ERR_TIMEOUT, 17);
           *abort_flag = 1;
@@ -403,7 +415,9 @@ int gemm_tc(Ctx* c, const GemmArgs& g) {
   p.C = g.C; p.ldc = g.ldc; p.alpha = g.alpha; p.beta = g.beta; p.flags = g.flags;
   p.b_nmajor = b_nmajor ? 1 : 0;
   p.tiles_n = (g.N + GT_BN - 1) / GT_BN;
-  p.num_tiles = p.tiles_n * ((g.M + GT_BM - 1) / GT_BM);
+  p.tiles_m = (g.M + GT_BM - 1) / GT_BM;
+  p.num_tiles = p.tiles_n * p.tiles_m;
+  p.kp = g.partial_k > 0 ? std::max(GT_BK, g.partial_k / GT_BK * GT_BK) : 128;
   p.idesc = tc::idesc_f32acc(2u, false, b_nmajor, GT_BM, GT_BN);
   const int grid = std::min(p.num_tiles, c->num_sms);
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,

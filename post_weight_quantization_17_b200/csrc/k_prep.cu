@@ -85,31 +85,41 @@ int prep_perm(Ctx* c, const float* diagv, int d, int act_order, int32_t* perm) {
 }
 
 // H'[a][b] = scale * S_sym[π_a][π_b], diagonal from diagv (dead fix-up).  S holds its lower
-// triangle.  Identity permutation: 32x32 tiles, the mirrored tile is read coalesced and
-// transposed through shared memory.
-__global__ void k_build_identity(const float* __restrict__ S, int d, float scale,
-                                 const float* __restrict__ diagv, float* __restrict__ Hp) {
+// triangle.  Identity permutation: block (J, I) with J <= I reads the 32 x 32 tile S[I][J] of the
+// lower triangle once (coalesced, through shared memory) and writes that tile and its mirror
+// (J, I) of H', to Hp and, when S2 is given, to S2 as well.  S2 may be S itself: a block reads
+// only its own lower tile, before writing it or its mirror, and no other block reads either.
+__global__ void k_build_identity(const float* S, int d, float scale,
+                                 const float* __restrict__ diagv, float* __restrict__ Hp,
+                                 float* S2) {
   pdl_wait();
   pdl_release();
-  __shared__ float lo[32][33];
-  __shared__ float up[32][33];
-  const int tr = blockIdx.y * 32, tc = blockIdx.x * 32;
+  const int I = blockIdx.y, J = blockIdx.x;
+  if (J > I) return;
+  __shared__ float t[32][33];
   const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  const int r0 = I * 32, c0 = J * 32;
   for (int r = ty; r < 32; r += 8) {
-    int a = tr + r, b = tc + tx;
-    lo[r][tx] = (a < d && b < d) ? S[(long long)a * d + b] : 0.f;      // S[a][b]
-    int a2 = tc + r, b2 = tr + tx;
-    up[r][tx] = (a2 < d && b2 < d) ? S[(long long)a2 * d + b2] : 0.f;  // S[tc+r][tr+tx]
+    const int a = r0 + r, b = c0 + tx;
+    t[r][tx] = (a < d && b < d && b <= a) ? S[(long long)a * d + b] : 0.f;
   }
   __syncthreads();
+  // tile (I, J): rows r0 + r, columns c0 + tx
   for (int r = ty; r < 32; r += 8) {
-    int a = tr + r, b = tc + tx;
+    const int a = r0 + r, b = c0 + tx;
     if (a >= d || b >= d) continue;
-    float v;
-    if (a == b) v = diagv[a];
-    else if (a > b) v = lo[r][tx] * scale;
-    else v = up[tx][r] * scale;  // S[b][a]
+    const float v = (a == b) ? diagv[a] : (a > b ? t[r][tx] : t[tx][r]) * scale;
     Hp[(long long)a * d + b] = v;
+    if (S2) S2[(long long)a * d + b] = v;
+  }
+  if (I == J) return;
+  // mirror (J, I): rows c0 + r, columns r0 + tx, H'[c0 + r][r0 + tx] = scale S[r0 + tx][c0 + r]
+  for (int r = ty; r < 32; r += 8) {
+    const int a = c0 + r, b = r0 + tx;
+    if (a >= d || b >= d) continue;
+    const float v = t[tx][r] * scale;
+    Hp[(long long)a * d + b] = v;
+    if (S2) S2[(long long)a * d + b] = v;
   }
 }
 
@@ -132,11 +142,13 @@ __global__ void k_build_perm(const float* __restrict__ S, int d, float scale,
   }
 }
 
-int prep_build(Ctx* c, const float* S, int d, float scale, const float* diagv,
-               const int32_t* perm, bool identity, float* Hp) {
+int prep_build(Ctx* c, float* S, int d, float scale, const float* diagv,
+               const int32_t* perm, bool identity, float* Hp, bool* wrote_S) {
+  *wrote_S = false;
   if (identity) {
     dim3 grid((d + 31) / 32, (d + 31) / 32), block(32, 8);
-    GPTQ_LAUNCH(c, k_build_identity, grid, block, 0, S, d, scale, diagv, Hp);
+    GPTQ_LAUNCH(c, k_build_identity, grid, block, 0, (const float*)S, d, scale, diagv, Hp, S);
+    *wrote_S = true;
   } else {
     dim3 grid((d + 255) / 256 < 8 ? (d + 255) / 256 : 8, d);
     GPTQ_LAUNCH(c, k_build_perm, grid, 256, 0, S, d, scale, diagv, perm, Hp);

@@ -208,8 +208,8 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 }
 
 // ------------------------------------------------------------------------------------------
-// a5: one block of up to 128 columns for 32 rows per CTA (8 warps, 4 rows per warp, 8 lanes
-// per row).  The block is walked in four 32-column sub-blocks; in a sub-block lane q of a row
+// a5: one block of up to 128 columns for 48 rows per CTA (12 warps, 4 rows per warp, 8 lanes
+// per row; two CTAs share an SM, so 12288 rows take one round on 148 SMs).  The block is walked in four 32-column sub-blocks; in a sub-block lane q of a row
 // owns the 4 consecutive columns 4q .. 4q+3 in registers.  A column step fetches the column's
 // value from its owner lane (width-8 shuffle), the 8 lanes run the sequential chain (divide,
 // round, clip, residual, η) side by side, and each lane updates only its own later columns
@@ -223,10 +223,10 @@ int init_work(Ctx* c, const void* W, int w_dtype, int m, int d, const int32_t* p
 // Markstein's theorem (IBM J. Res. Dev. 34(1), 1990: y within half an ulp of 1/Δ and q0 within
 // an ulp of w/Δ make RN(q0 + r y) = RN(w/Δ)) this is the same fp32 value as a division, at a
 // third of its latency on the column chain.
-constexpr int kColWarps = 8;
+constexpr int kColWarps = 12;                // 48 rows per CTA: two CTAs fit an SM
 constexpr int kColLanes = 8;                 // lanes per row
 constexpr int kColSub = 4 * kColLanes;       // sub-block width: 4 columns per lane
-constexpr int kColCtaRows = 32;
+constexpr int kColCtaRows = 48;
 constexpr int kColLd = 132;  // padded row of the staging buffers (16-byte rows)
 constexpr int kColSmem = 128 * 128 * 4 + kColCtaRows * kColLd * 4 + kColWarps * 128 * 4;
 static_assert(kColCtaRows == kColWarps * 32 / kColLanes && kColCtaRows == kColRows, "rows per CTA");
@@ -432,7 +432,7 @@ __device__ __forceinline__ void col_walk(float (*St)[kColLd], float (*lossw)[128
 }
 
 template <bool UNIFORM>
-__global__ void __launch_bounds__(32 * kColWarps) k_colblock(
+__global__ void __launch_bounds__(32 * kColWarps, 2) k_colblock(
     float* __restrict__ Wk, int m, int d, int i, int nb, const float* __restrict__ R,
     float* __restrict__ scales, int32_t* __restrict__ zeros, int ng,
     const int32_t* __restrict__ gcol, int dyn, int maxq, float* __restrict__ E,
@@ -551,7 +551,7 @@ __global__ void __launch_bounds__(32 * kColWarps) k_colblock(
     col_walk<UNIFORM, false>(St, lossw, args, r, row, nb, d, i, ldE, vec, Wk, E, Ehi, Elo, codes,
                           dyn, ng, scales, zeros);
   __syncthreads();
-  // loss partial Σ_rows η² per column, the 8 warps' sums in a fixed order
+  // loss partial Σ_rows η² per column, the warps' sums in a fixed order
   for (int t = tid; t < nb; t += blockDim.x) {
     float sacc = 0.f;
 #pragma unroll

@@ -290,16 +290,39 @@ constexpr int S2_B_BYTES = (S2_BN / 128) * SY_BOX_BYTES;  // 16 KB: this CTA's 1
 constexpr int S2_STAGE_BYTES = S2_A_BYTES + S2_B_BYTES;
 constexpr int S2_SMEM = S2_STAGES * S2_STAGE_BYTES + 1024 + 256;
 
-__device__ __forceinline__ void syrk2_tile_coords(int t, int& I, int& J) {
-  int i = 0;
+// Tile t -> (I, J), J <= I, of the lower triangle of 256 x 256 tiles (nI row blocks).  Tiles go
+// in groups of SY2_GROUP row blocks walked column by column (rows I of the group with I >= J), so
+// that the 74 tiles of one wave cover ~8 row blocks and ~9 column blocks of X: every pair walks
+// the token axis in lockstep, and a wave's X slabs are then fetched from HBM once for ~17
+// feature blocks instead of once per tile (in row-major order a wave of a wide triangle spans one
+// row block and ~74 column blocks).
+constexpr int SY2_GROUP = 8;
+__device__ __forceinline__ void syrk2_tile_coords(int t, int nI, int& I, int& J) {
+  int first = 0;
   for (;;) {
-    if (t <= i) {  // row-block i of 256 has tiles J = 0 .. i
-      I = i;
-      J = t;
-      return;
+    const int last = min(first + SY2_GROUP, nI) - 1;
+    const int rows = last - first + 1;
+    const int below = rows * first;                      // columns J < first: all rows
+    const int cnt = below + rows * (rows + 1) / 2;       // + the group's own triangle
+    if (t < cnt) {
+      if (t < below) {
+        J = t / rows;
+        I = first + t % rows;
+        return;
+      }
+      t -= below;
+      for (int j = first;; ++j) {                        // column j holds rows j .. last
+        const int c = last - j + 1;
+        if (t < c) {
+          J = j;
+          I = j + t;
+          return;
+        }
+        t -= c;
+      }
     }
-    t -= i + 1;
-    ++i;
+    t -= cnt;
+    first += SY2_GROUP;
   }
 }
 
@@ -356,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
       const uint32_t leader_full = tc::map_to_rank(full, 0);
       for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
         int I, J;
-        syrk2_tile_coords(t, I, J);
+        syrk2_tile_coords(t, (d + 255) / 256, I, J);
         const int ra = 256 * I + S2_BM * rank, rb = 256 * J + 128 * rank;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!tc::mbar_wait_cluster(&empty[stage], phase ^ 1, budget)) {
@@ -453,7 +476,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
     bool ok = true;
     for (int t = pair; t < num_tiles && ok && !*abort_flag; t += npairs) {
       int I, J;
-      syrk2_tile_coords(t, I, J);
+      syrk2_tile_coords(t, (d + 255) / 256, I, J);
       float m[128];
 #pragma unroll
       for (int u = 0; u < 128; ++u) m[u] = 0.f;

@@ -11,8 +11,9 @@ int syrk_accumulate(Ctx* c, const void* X, int dtype, long long n, int d, float*
 int prep_diag(Ctx* c, const float* S, int d, float scale, float* diagv, uint8_t* dead);
 int prep_mean(Ctx* c, const float* diagv, int d);
 int prep_perm(Ctx* c, const float* diagv, int d, int act_order, int32_t* perm);
-int prep_build(Ctx* c, const float* S, int d, float scale, const float* diagv, const int32_t* perm,
-               bool identity, float* Hp);
+// H' into Hp; with the identity order also into S itself (*wrote_S), else S is left as it was.
+int prep_build(Ctx* c, float* S, int d, float scale, const float* diagv, const int32_t* perm,
+               bool identity, float* Hp, bool* wrote_S);
 int prep_copy(Ctx* c, const float* src, float* dst, size_t count);
 int prep_damp(Ctx* c, float* Hl, int d, float percdamp);
 
@@ -43,6 +44,30 @@ bool gemm_pair_applies(int M, int N, int K, const float* Ah, long long lda, cons
 int gemm_pair(Ctx* c, int M, int N, int K, const float* Ah, const float* Al, long long lda,
               const float* Bh, const float* Bl, long long ldb, float* C, long long ldc, float alpha,
               float beta);
+// The general form: B either N-major ([K, N] row-major, ldb) or K-major (B(k, j) = Bh[j ldb + k]);
+// structure flags of gemm_simt.cuh (kAUpper, kALower, kBUpper, kBLower restrict each tile's k
+// range, kCUpper computes only tiles touching the upper triangle); with Ch / Cl set (and
+// beta = 0) the result alpha A B is written as its tf32 halves there (row stride ldc), not to C.
+struct GemmPairArgs {
+  int M, N, K;
+  const float *Ah, *Al;
+  long long lda;
+  const float *Bh, *Bl;
+  long long ldb;
+  bool b_kmajor;
+  float* C;
+  float *Ch, *Cl;
+  long long ldc;
+  float alpha, beta;
+  int flags;
+  // k-elements per TMEM partial (a multiple of 32; 0: 128).  The tensor core rounds its fp32
+  // accumulator toward zero at every MMA, so a partial's error grows with the MMAs it sums;
+  // products whose errors the factorization amplifies take short partials.
+  int partial_k;
+};
+int gemm_pair(Ctx* c, const GemmPairArgs& g);
+// k-elements per TMEM partial in the factorization's products (k_gemm_pair and k_gemm_tc)
+constexpr int kFactorPartialK = 32;
 int split_tf32(Ctx* c, const float* src, long long lds, int rows, int cols, float* hi, float* lo,
                long long ldd);
 int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int k, int c0, int c1,
@@ -76,8 +101,8 @@ int dequant_matmul_tiled(Ctx* c, const void* X, int x_dtype, int T, int d,
 int twosided_round(Ctx* c, const float* X, int m, int n, const float* RA, const float* RB,
                    float* Z, float* eta, float* Y, float* C, float* etas, float* RAT);
 
-constexpr int kColRows = 32;      // rows per column-block CTA (8 warps, 8 lanes per row)
+constexpr int kColRows = 48;      // rows per column-block CTA (12 warps, 8 lanes per row)
 constexpr int kColMax = 128;      // columns per kernel block
-constexpr int kSuperCols = 512;   // columns per super-block of the two-level lazy update
+constexpr int kSuperCols = 1024;  // columns per super-block of the two-level lazy update
 
 }  // namespace gptq

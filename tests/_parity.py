@@ -96,9 +96,10 @@ TOL_DYN_SCALE = 1e-4
 
 
 def check_layer(gpu, Wn, H, spec, block=None, method="explicit", dynamic=False, grid=None,
-                grid_kind="minmax"):
+                grid_kind="minmax", replay_block=0):
     """Oracle on the same H and W; returns a dict of the measured discrepancies after
-    asserting the contract's tolerances.
+    asserting the contract's tolerances.  replay_block > 0 replays the decisions in the
+    lazy-block form (for large layers; same decisions as the unblocked replay).
 
     dynamic: the GPU ran with dynamic groups (grid_given = 2).  Each group's grid is then fitted
     on weights that already carry fp32 compensation, so Δ is compared with the replay's own fit
@@ -140,7 +141,7 @@ def check_layer(gpu, Wn, H, spec, block=None, method="explicit", dynamic=False, 
         assert res["grid_scale_rel"] <= TOL_DYN_SCALE, res
     else:
         rep = O.decision_replay(o["Wp"], o["R"], o["scale"], o["zero"], o["gcol"], spec.bits,
-                                codes_p, band=BAND, maxq=o["maxq"])
+                                codes_p, band=BAND, maxq=o["maxq"], block=replay_block)
     res["identical"] = rep["identical"] / rep["n"]
     res["in_band"] = rep["in_band"]
     res["violations"] = rep["violations"]

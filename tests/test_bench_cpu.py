@@ -31,3 +31,41 @@ def test_w4a16_cpu_sample_extrapolates_by_rows():
     s, full, desc = bench.oracle_w4a16_sample(1024, 512, 4, 64)
     assert 0 < s and full == pytest.approx(s * 1024 / 64)
     assert "64 of 1024 rows" in desc
+
+
+def test_gpus_n_without_launcher_starts_its_own_ranks(monkeypatch):
+    """--gpus N > 1 outside torchrun re-launches bench.py under torch.distributed.run with N
+    processes on this node (rendezvous on 127.0.0.1) and the same arguments."""
+    sys.path.insert(0, ROOT)
+    import bench
+    seen = {}
+
+    def fake_call(cmd, cwd=None):
+        seen["cmd"], seen["cwd"] = cmd, cwd
+        return 0
+
+    monkeypatch.setattr(bench.subprocess, "call", fake_call)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4", "--steps", "2", "--warmup", "3"])
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert e.value.code == 0
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert cmd[-6:] == ["--gpus", "4", "--steps", "2", "--warmup", "3"]
+    assert cmd[-7].endswith("bench.py")
+
+
+def test_workload_configs():
+    sys.path.insert(0, ROOT)
+    import bench
+    g5 = bench.workload(5)
+    assert len(g5) == 1 and g5[0].mats[0].m == 12288 and g5[0].x_spec.chunk == 8192
+    assert bench.weights_per_step(g5) == 12288 * 49152
+    assert bench.workload(5, bits=2)[0].mats[0].bits == 2
+    g4 = bench.workload(4)
+    assert [len(g.mats) for g in g4] == [3, 1, 2, 1]
+    assert bench.weights_per_step(g4) == 4 * 4096 * 4096 + 2 * 11008 * 4096 + 4096 * 11008
+    assert all(g.x_spec.chunk == g.x_spec.n_tokens for g in g4)   # one call over all tokens
+    assert bench.baseline_cols(49152, 65536) == 2048 and bench.baseline_cols(100, 512) == 100

@@ -432,6 +432,38 @@ def test_decision_replay_accepts_self_and_flags_planted_mistake():
     assert rep["rows_with_flips"][3] and rep["rows_with_flips"].sum() == 1
 
 
+@pytest.mark.parametrize("block,dynamic,act_order", [(8, 0, False), (5, 0, True),
+                                                     (16, 8, False), (4, 8, True)])
+def test_decision_replay_lazy_blocks_equal_unblocked(block, dynamic, act_order):
+    """The lazy-block form of the replay ([T] eq.(46), equal to the unblocked recursion by
+    eq.(47)-(49)) takes the same decisions and gives the same Ŵ and loss, also when it follows
+    codes with planted mistakes (a flip in band and one far outside) and with R given in fp32."""
+    W, X = _layer(12, 40, 200, 21 + block)
+    H = O.hessian(X)
+    out = O.gptq_layer(W, H, 3, 8, method="lazy", block=8, act_order=act_order,
+                       dynamic=bool(dynamic))
+    codes_p = out["codes"][:, out["perm"]].copy()
+    codes_p[2, 7] = min(codes_p[2, 7] + 1, 7)           # may or may not be in band
+    codes_p[5, 21] = (codes_p[5, 21] + 3) % 8            # far outside the band
+    for R in (out["R"], out["R"].astype(np.float32)):
+        runs = []
+        for blk in (0, block):
+            if dynamic:
+                sc, ze = O.dynamic_grid_arrays(12, 40, dynamic)
+            else:
+                sc, ze = out["scale"].copy(), out["zero"].copy()
+            runs.append(O.decision_replay(out["Wp"], R, sc, ze, out["gcol"], 3, codes_p,
+                                          dynamic=dynamic, block=blk,
+                                          other_zero=out["zero"] if dynamic else None))
+        a, b = runs
+        for k in ("n", "identical", "in_band", "violations", "grid_in_band", "grid_violations"):
+            assert a[k] == b[k], k
+        assert a["violations"] >= 1
+        assert np.array_equal(a["rows_with_flips"], b["rows_with_flips"])
+        assert np.allclose(a["replay_Q"], b["replay_Q"], rtol=0, atol=1e-12)
+        assert np.allclose(a["replay_loss"], b["replay_loss"], rtol=1e-9, atol=0)
+
+
 # ---------------------------------------------------------------- packing
 def test_pack_layout_definition():
     codes = np.array([[1, 2, 3, 4, 5, 6, 7, 8, 9]])
