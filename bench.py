@@ -68,7 +68,48 @@ def parse(argv=None):
                          "(gptq_retile_codes, outside the timed region)")
     ap.add_argument("--n-tokens", type=int, default=0,
                     help="calibration tokens (profiling captures only; the bench line uses all)")
+    ap.add_argument("--probe", choices=["factor", "tail", "hessian"], default=None,
+                    help="profiling captures only: run one library call at a chosen size and exit "
+                         "(factor: gptq_prepare_hinv on an SPD H of d = --probe-d; tail: that plus "
+                         "gptq_quantize_layer of a 12288 x d layer; hessian: one "
+                         "gptq_hessian_accumulate of 8192 tokens x d)")
+    ap.add_argument("--probe-d", type=int, default=16384)
     return ap.parse_args(argv)
+
+
+def run_probe(args):
+    """One library call at a chosen size, for an ncu capture of its kernels (no timing, no JSON
+    line).  Inputs are seeded random data generated on the device."""
+    import torch
+    import post_weight_quantization_17_b200 as G
+    torch.cuda.set_device(0)
+    d, dev = args.probe_d, torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(0)
+    if args.probe in ("factor", "tail"):
+        A = torch.randn(d, 2 * d, device=dev, generator=g) / (2 * d) ** 0.5
+        S = A @ A.T
+        del A
+        S += 0.1 * torch.eye(d, device=dev)
+        ctx = G.Context(m_max=12288, d_max=d, act_order=False)
+        R = torch.empty(d, d, device=dev)
+        perm = torch.empty(d, dtype=torch.int32, device=dev)
+        dead = torch.empty(d, dtype=torch.uint8, device=dev)
+        G.gptq_prepare_hinv(ctx, S, 0, 0.01, False, R, perm, dead)
+        if args.probe == "tail":
+            m = 12288
+            W = (torch.randn(m, d, device=dev, generator=g) * 0.01).half()
+            b = G.LayerBuffers(m, d, 4, 128, dev, with_factor=False)
+            G.gptq_quantize_layer(ctx, W, R, None, dead, 4, 128, 128, 0, b.scales, b.zeros,
+                                  b.codes, b.W_hat, b.col_loss)
+    else:
+        X = torch.randn(8192, d, device=dev, generator=g).to(torch.bfloat16)
+        S = torch.empty(d, d, device=dev)
+        ctx = G.Context(m_max=8, d_max=d, act_order=False)
+        G.gptq_hessian_accumulate(ctx, X, S, 0)
+    G.gptq_sync_status(ctx)
+    ctx.close()
+    torch.cuda.synchronize()
+    print(f"probe {args.probe} d={d} done", flush=True)
 
 
 @dataclasses.dataclass
@@ -245,18 +286,19 @@ def kernel_source_digest(files):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, digest: str, per_launch_scale: float = 1.0):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this exact
+def ncu_traffic(key: str, digest: str):
+    """DRAM bytes (read + write) per step of a stage's kernels from the committed ncu launch
+    list (profiles/ncu_traffic.json, keyed "<stage>@config<k>"), if it was taken on this exact
     kernel source; else None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
-    e = j.get(kernel)
+    e = j.get(key)
     if not e or e.get("source_digest") != digest:
         return None
-    return e["dram_bytes_per_launch"] * per_launch_scale
+    return e["dram_bytes_per_step"]
 
 
 def dist_setup(args):
@@ -423,14 +465,12 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- our path
+_CS = "post_weight_quantization_17_b200/csrc/"
 STAGE_KERNEL_FILES = {
-    "a1_hessian": ["post_weight_quantization_17_b200/csrc/k_syrk.cu",
-                   "post_weight_quantization_17_b200/csrc/tc_util.cuh"],
-    "a3_factor_gemm": ["post_weight_quantization_17_b200/csrc/k_gemm_tc.cu",
-                       "post_weight_quantization_17_b200/csrc/tc_util.cuh"],
-    "a6_update": ["post_weight_quantization_17_b200/csrc/k_gemm_pair.cu",
-                  "post_weight_quantization_17_b200/csrc/k_gemm_tc.cu",
-                  "post_weight_quantization_17_b200/csrc/tc_util.cuh"],
+    "a1_hessian": [_CS + "k_syrk.cu", _CS + "tc_util.cuh"],
+    "a3_factor_gemm": [_CS + "k_factor.cu", _CS + "k_gemm_pair.cu", _CS + "k_gemm_tc.cu",
+                       _CS + "gemm_simt.cuh", _CS + "tc_util.cuh"],
+    "a6_update": [_CS + "k_gemm_pair.cu", _CS + "k_gemm_tc.cu", _CS + "tc_util.cuh"],
 }
 
 
@@ -609,7 +649,7 @@ def run_ours(args):
         launches_main = (kern or {}).get({"a1_hessian": "hessian", "a3_factor_gemm": "factor_gemm",
                                           "a6_update": "update"}[main_name], (0, 0))[1]
         roofline["launches_per_step"] = launches_main
-        tr = ncu_traffic(main_name, digest)
+        tr = ncu_traffic(f"{main_name}@config{args.config}", digest)
         roofline["traffic"] = tr
         roofline["traffic_per"] = "step" if tr is not None else None
 
@@ -837,6 +877,9 @@ def run_w4a16(args):
 def main():
     argv = sys.argv[1:]
     args = parse(argv)
+    if args.probe:
+        run_probe(args)
+        return
     if args.w4a16:
         run_w4a16(args)
         return

@@ -168,6 +168,9 @@ def test_fc2_175b_full_size():
       4. R H_λ R^T = I on 64 sampled rows within 1e-4 (an identity that holds at any size);
       5. per bit width, 64 sampled rows by decision replay against the GPU's R promoted to fp64
          (validated by 3 and 4): grid and packed words bit-exact, codes, Ŵ."""
+    import time
+    t0 = time.perf_counter()
+    phase = {}
     dev = torch.device("cuda")
     spec4, spec2 = CONFIGS[5]
     d, m = spec4.d, spec4.m
@@ -207,6 +210,7 @@ def test_fc2_175b_full_size():
     H_g = np.where(lo, Sl, Sl.T) * (2.0 / n)            # S holds the lower triangle
     res["H_block"] = P.rel_fro(H_g, blk_o.numpy())
     assert res["H_diag"] <= P.TOL_H and res["H_block"] <= P.TOL_H, res
+    phase["H"] = time.perf_counter() - t0
     # ---- 1. truncated instance: the first 8192 input features, whole library, full parity
     dt = 8192
     spec_t = dataclasses.replace(spec4, d=dt, name="fc2_first_8192_features")
@@ -227,6 +231,7 @@ def test_fc2_175b_full_size():
                                         for k, v in r.items()}
         del gpu
     ctx_t.close()
+    phase["truncated"] = time.perf_counter() - t0
     del xt_chunks, Ht, Wt, Wtn
     torch.cuda.empty_cache()
     # symmetric copy of H for the identity check (prepare overwrites S)
@@ -264,6 +269,7 @@ def test_fc2_175b_full_size():
     M = (Y @ Ra.T).cpu().numpy()
     res["RHRt_minus_I"] = float(np.linalg.norm(M - np.eye(len(pick))) / np.sqrt(len(pick)))
     assert res["RHRt_minus_I"] <= P.TOL_HINV, res
+    phase["factor_checks"] = time.perf_counter() - t0
     del Hs, Y, Ra
     torch.cuda.empty_cache()
     # ---- 5. sampled rows of the full layer, per bit width, by decision replay on the GPU's R
@@ -305,4 +311,6 @@ def test_fc2_175b_full_size():
         del W, scales, zeros, codes, W_hat, packed
         torch.cuda.empty_cache()
     ctx.close()
+    phase["rows"] = time.perf_counter() - t0
+    res["seconds_cumulative"] = {k: round(v, 1) for k, v in phase.items()}
     print("fc2 full size:", {k: (f"{v:.3e}" if isinstance(v, float) else v) for k, v in res.items()})
