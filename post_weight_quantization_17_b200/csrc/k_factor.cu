@@ -231,8 +231,10 @@ static int larger_child(int n) { return (((n + 1) / 2 + FB - 1) / FB) * FB; }
 
 // Nodes whose right child has at least this many columns run their four products on CTA pairs
 // (k_gemm_pair) with operands split into tf32 halves beforehand; the rest on k_gemm_tc /
-// k_gemm_small.  The pair path needs 16-byte aligned rows (ld and n2 multiples of 4).
-constexpr int kFactorPairMin = 512;
+// k_gemm_small (below this size a grid of 256 x 256 tiles leaves most of the 74 pairs idle, and
+// the single-CTA GEMM measured faster).  The pair path needs 16-byte aligned rows (ld and n2
+// multiples of 4).
+constexpr int kFactorPairMin = 2048;
 static bool pair_node(int n2, long long ld) {
   return n2 >= kFactorPairMin && n2 % 4 == 0 && ld % 4 == 0;
 }

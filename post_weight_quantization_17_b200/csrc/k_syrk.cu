@@ -500,9 +500,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SY_THREADS, 1)
         __syncwarp();
         if (lane == 0) {
           if (rank == 0)
-            tc::mbar_arrive(&tempty[acc]);
+            tc::mbar_arrive_relaxed(&tempty[acc]);
           else
-            tc::mbar_arrive_remote(leader_tempty + 8u * acc);
+            tc::mbar_arrive_remote_relaxed(leader_tempty + 8u * acc);
         }
         if (++acc == 2) {
           acc = 0;
