@@ -484,6 +484,7 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     2. prepare: dead features, act-order permutation, damping, G and R (with retry);
     3. working copy W_work = W with dead columns zeroed, permuted into processing order;
     4. the column recursion: `method` = "explicit" (eq.(22)/(26)) or "lazy" (eq.(42)/(46));
+       "prepare" stops before it (codes, W_hat and col_loss are None);
     5. un-permute codes, Ŵ and the per-column loss back to original column order.
 
     dynamic=True (group > 0): dynamic groups ([T] §8.3): the grid of processing group j // g is
@@ -521,6 +522,15 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     Wp = Wwork[:, perm]
     dyn = int(group) if dynamic else 0
     gcol = np.arange(d) // dyn if dynamic else _group_of_column(perm, d, group)
+    group_id = np.empty(d, np.int64)
+    group_id[perm] = gcol
+    if method == "prepare":
+        # steps 1-3 only: the grid, the factor and the working copy, for callers that replay
+        # another implementation's decisions instead of running the recursion
+        return dict(codes=None, W_hat=None, scale=scale, zero=zero, col_loss=None, perm=perm,
+                    dead=dead, lam=prep["lam"], G=prep["G"], R=prep["R"],
+                    H_lambda=prep["H_lambda"], retries=prep["retries"], Wp=Wp, gcol=gcol,
+                    group_id=group_id, maxq=maxq)
     if method == "explicit":
         codes_p, Q_p, loss_p, _ = gptq_explicit(Wp, prep["G"], scale, zero, gcol, bits, dyn,
                                                 maxq)
@@ -535,8 +545,6 @@ def gptq_layer(W, H, bits: int, group: int, block: int = 128, percdamp: float = 
     codes[:, perm] = codes_p
     W_hat[:, perm] = Q_p
     col_loss[perm] = loss_p
-    group_id = np.empty(d, np.int64)
-    group_id[perm] = gcol
     return dict(codes=codes, W_hat=W_hat, scale=scale, zero=zero, col_loss=col_loss,
                 perm=perm, dead=dead, lam=prep["lam"], G=prep["G"], R=prep["R"],
                 H_lambda=prep["H_lambda"], retries=prep["retries"], Wp=Wp, gcol=gcol,

@@ -226,7 +226,11 @@ def test_fc2_175b_full_size():
     Wtn = Wt.float().cpu().double().numpy()
     for spec in (spec_t, dataclasses.replace(spec_t, bits=2)):
         gpu = P.gpu_run(ctx_t, spec, Wt, xt_chunks)
-        r = P.check_layer(gpu, Wtn, Ht, spec, method="lazy", replay_block=128)
+        # 4-bit: the whole check; 2-bit: the same, except that the decisions, Ŵ and the loss are
+        # compared with the replay only (the free-running recursion and layer error take minutes
+        # of CPU time at this size)
+        r = P.check_layer(gpu, Wtn, Ht, spec, method="lazy", replay_block=128,
+                          free_running=spec.bits == 4)
         res[f"trunc_{spec.bits}bit"] = {k: round(v, 8) if isinstance(v, float) else v
                                         for k, v in r.items()}
         del gpu

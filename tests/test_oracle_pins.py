@@ -727,3 +727,14 @@ def test_tile_codes4_layout():
     # row block 1 holds rows 128, 129 and 126 zero rows; column block 1 holds 4 words per row
     assert np.count_nonzero(t) == np.count_nonzero(packed)
     assert np.array_equal(O.untile_codes4(t, m, d), packed)
+
+
+def test_gptq_layer_prepare_only_matches_the_full_run():
+    W, X = _layer(8, 40, 160, 23)
+    H = O.hessian(X)
+    full = O.gptq_layer(W, H, 4, 8, method="lazy", block=8, act_order=True)
+    prep = O.gptq_layer(W, H, 4, 8, method="prepare", block=8, act_order=True)
+    assert prep["codes"] is None and prep["W_hat"] is None and prep["col_loss"] is None
+    for k in ("scale", "zero", "perm", "dead", "G", "R", "H_lambda", "Wp", "gcol", "group_id"):
+        assert np.array_equal(prep[k], full[k]), k
+    assert prep["lam"] == full["lam"] and prep["maxq"] == full["maxq"]
