@@ -187,34 +187,28 @@ __global__ void __launch_bounds__(FB_THREADS, 1) k_factor_base(float* __restrict
   }
 }
 
-// dst[rows x cols] = src (or 0 when src is null).  Grid: x over 1024-column slices of a row (256
-// threads, 4 columns each), y over rows (grid-strided); 16-byte accesses when rows are aligned.
-__global__ void k_copy2d(const float* __restrict__ src, long long lds, float* __restrict__ dst,
-                         long long ldd, int rows, int cols, int vec) {
+// Zeros the strict lower triangle of the d x d matrix M (row stride ld).  Grid: x over
+// 1024-column slices of a row (256 threads, 4 columns each), y over rows (grid-strided).
+__global__ void k_zero_lower(float* __restrict__ M, long long ld, int d, int vec) {
   pdl_wait();
   pdl_release();
   const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
-  if (c0 >= cols) return;
-  for (int r = blockIdx.y; r < rows; r += gridDim.y) {
-    float* d = dst + (long long)r * ldd + c0;
-    const float* s = src ? src + (long long)r * lds + c0 : nullptr;
-    if (vec && c0 + 4 <= cols) {
-      *reinterpret_cast<float4*>(d) =
-          s ? *reinterpret_cast<const float4*>(s) : make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      for (int u = 0; u < 4 && c0 + u < cols; ++u) d[u] = s ? s[u] : 0.f;
-    }
+  for (int r = blockIdx.y; r < d; r += gridDim.y) {
+    if (c0 >= r) continue;
+    float* row = M + (long long)r * ld + c0;
+    if (vec && c0 + 4 <= r)
+      *reinterpret_cast<float4*>(row) = make_float4(0.f, 0.f, 0.f, 0.f);
+    else
+      for (int u = 0; u < 4 && c0 + u < r; ++u) row[u] = 0.f;
   }
 }
 
-static int copy2d(Ctx* c, const float* src, long long lds, float* dst, long long ldd, int rows,
-                  int cols) {
-  if (rows <= 0 || cols <= 0) return GPTQ_OK;
-  auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
-  const int vec = (ldd % 4 == 0) && al(dst) && (!src || ((lds % 4 == 0) && al(src)));
-  const int gx = (cols + 1023) / 1024;
-  const int gy = std::min(rows, std::max(1, c->num_sms * 16 / gx));
-  GPTQ_LAUNCH(c, k_copy2d, dim3(gx, gy), 256, 0, src, lds, dst, ldd, rows, cols, vec);
+static int zero_lower(Ctx* c, float* M, long long ld, int d) {
+  if (d <= 1) return GPTQ_OK;
+  const int vec = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(M) & 15) == 0);
+  const int gx = (d + 1023) / 1024;
+  const int gy = std::min(d, std::max(1, c->num_sms * 16 / gx));
+  GPTQ_LAUNCH(c, k_zero_lower, dim3(gx, gy), 256, 0, M, ld, d, vec);
   return GPTQ_OK;
 }
 
@@ -292,7 +286,7 @@ static int rec_pair(FactorRun& f, int s, int e, int level, float* buf) {
   float* Ablk = M + (long long)s * ld + s;
   StageScope stage(c, f.stage_copy);
   if ((rc = split_tf32(c, Bblk, ld, n1, n2, Bh, Bl, n2))) return rc;
-  if ((rc = split_tf32(c, R22, ld, n2, n2, R22h, R22l, n2))) return rc;
+  if ((rc = split_tf32(c, R22, ld, n2, n2, R22h, R22l, n2, true))) return rc;
   c->stage = f.stage_gemm;
   // U12 = B R22^T: opB(k, j) = R22[j][k] (K-major), zero for k < j
   GemmPairArgs g{};
@@ -332,7 +326,7 @@ static int rec_pair(FactorRun& f, int s, int e, int level, float* buf) {
   GPTQ_CUDA_CHECK(c, cudaStreamWaitEvent(c->stream, ev_t, 0));
   // R12 = -R11 T2 (R11(i, k) = 0 for k < i)
   c->stage = f.stage_copy;
-  if ((rc = split_tf32(c, Ablk, ld, n1, n1, Bh, Bl, n1))) return rc;
+  if ((rc = split_tf32(c, Ablk, ld, n1, n1, Bh, Bl, n1, true))) return rc;
   c->stage = f.stage_gemm;
   GemmPairArgs g4{};
   g4.M = n1; g4.N = n2; g4.K = n1;
@@ -340,10 +334,7 @@ static int rec_pair(FactorRun& f, int s, int e, int level, float* buf) {
   g4.Bh = T2h; g4.Bl = T2l; g4.ldb = n2; g4.b_kmajor = false;
   g4.C = Rblk; g4.ldc = ld; g4.alpha = -1.f; g4.beta = 0.f; g4.flags = kAUpper;
   g4.partial_k = kFactorPartialK;
-  if ((rc = gemm_pair(c, g4))) return rc;
-  // strict lower block of this level
-  c->stage = f.stage_copy;
-  return copy2d(c, nullptr, 0, M + (long long)mid * ld + s, ld, n2, n1);
+  return gemm_pair(c, g4);
 }
 
 static int rec(FactorRun& f, int s, int e, int level, float* buf) {
@@ -392,10 +383,7 @@ static int rec(FactorRun& f, int s, int e, int level, float* buf) {
   GPTQ_CUDA_CHECK(c, cudaStreamWaitEvent(c->stream, ev_t, 0));
   // R12 = -R11 T2  (R11(i,k) = 0 for k < i)
   GemmArgs g4{n1, n2, n1, Ablk, ld, 1, T2, n2, 1, Rblk, ld, -1.f, 0.f, kAUpper, kFactorPartialK};
-  if ((rc = gemm_f32(c, g4))) return rc;
-  // strict lower block of this level
-  c->stage = f.stage_copy;
-  return copy2d(c, nullptr, 0, M + (long long)mid * ld + s, ld, n2, n1);
+  return gemm_f32(c, g4);
 }
 
 int factor_inverse(Ctx* c, float* M, int d, float* tmp) {
@@ -421,7 +409,15 @@ int factor_inverse(Ctx* c, float* M, int d, float* tmp) {
   f.stage_copy = own ? GPTQ_STAGE_FACTOR_COPY : c->stage;
   f.pair = c->num_sms >= 2 && (reinterpret_cast<uintptr_t>(M) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(tmp) & 15) == 0;
-  return rec(f, 0, d, 0, tmp);
+  int rc = rec(f, 0, d, 0, tmp);
+  if (rc) return rc;
+  // Below the diagonal M still holds H_λ and the products' by-products: no product reads there
+  // (each tile's k-range starts at its own first row or column, so the only entries below the
+  // diagonal that a product reads lie inside a diagonal block of <= 128, which the base kernel
+  // zeroed, and the CTA-pair products read triangular operands through splits that zero them),
+  // so the strict lower triangle is cleared once, here.
+  StageScope stage(c, f.stage_copy);
+  return zero_lower(c, M, d, d);
 }
 
 }  // namespace gptq

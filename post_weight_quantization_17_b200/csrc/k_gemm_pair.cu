@@ -380,12 +380,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GP_THREADS, 1)
   }
 }
 
-// x -> (hi, lo) for a rows x cols block (row strides lds, ldd).  Grid: x over 1024-column slices
-// of a row (256 threads, 4 columns each), y over rows (grid-strided); 16-byte accesses when the
-// block's rows are 16-byte aligned.
+// x -> (hi, lo) for a rows x cols block (row strides lds, ldd); with upper set, the halves of
+// the elements below the block's diagonal (column < row) are written as zeros whatever src holds.
+// Grid: x over 1024-column slices of a row (256 threads, 4 columns each), y over rows
+// (grid-strided); 16-byte accesses when the block's rows are 16-byte aligned.
 __global__ void k_split_tf32(const float* __restrict__ src, long long lds, int rows, int cols,
                              float* __restrict__ hi, float* __restrict__ lo, long long ldd,
-                             int vec) {
+                             int vec, int upper) {
   pdl_wait();
   pdl_release();
   const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
@@ -395,7 +396,13 @@ __global__ void k_split_tf32(const float* __restrict__ src, long long lds, int r
     float* h = hi + (long long)r * ldd + c0;
     float* l = lo + (long long)r * ldd + c0;
     if (vec && c0 + 4 <= cols) {
-      const float4 x = *reinterpret_cast<const float4*>(s);
+      float4 x = *reinterpret_cast<const float4*>(s);
+      if (upper && c0 < r) {
+        x.x = 0.f;
+        if (c0 + 1 < r) x.y = 0.f;
+        if (c0 + 2 < r) x.z = 0.f;
+        if (c0 + 3 < r) x.w = 0.f;
+      }
       const float4 xh = make_float4(tc::tf32_rna(x.x), tc::tf32_rna(x.y), tc::tf32_rna(x.z),
                                     tc::tf32_rna(x.w));
       *reinterpret_cast<float4*>(h) = xh;
@@ -404,7 +411,7 @@ __global__ void k_split_tf32(const float* __restrict__ src, long long lds, int r
                       tc::tf32_rna(x.z - xh.z), tc::tf32_rna(x.w - xh.w));
     } else {
       for (int u = 0; u < 4 && c0 + u < cols; ++u) {
-        const float x = s[u];
+        const float x = (upper && c0 + u < r) ? 0.f : s[u];
         const float xh = tc::tf32_rna(x);
         h[u] = xh;
         l[u] = tc::tf32_rna(x - xh);
@@ -414,13 +421,14 @@ __global__ void k_split_tf32(const float* __restrict__ src, long long lds, int r
 }
 
 int split_tf32(Ctx* c, const float* src, long long lds, int rows, int cols, float* hi, float* lo,
-               long long ldd) {
+               long long ldd, bool upper) {
   if (rows <= 0 || cols <= 0) return GPTQ_OK;
   auto al = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
   const int vec = (lds % 4 == 0) && (ldd % 4 == 0) && al(src) && al(hi) && al(lo);
   const int gx = (cols + 1023) / 1024;
   const int gy = std::min(rows, std::max(1, c->num_sms * 16 / gx));
-  GPTQ_LAUNCH(c, k_split_tf32, dim3(gx, gy), 256, 0, src, lds, rows, cols, hi, lo, ldd, vec);
+  GPTQ_LAUNCH(c, k_split_tf32, dim3(gx, gy), 256, 0, src, lds, rows, cols, hi, lo, ldd, vec,
+              upper ? 1 : 0);
   return GPTQ_OK;
 }
 

@@ -68,8 +68,9 @@ struct GemmPairArgs {
 int gemm_pair(Ctx* c, const GemmPairArgs& g);
 // k-elements per TMEM partial in the factorization's products (k_gemm_pair and k_gemm_tc)
 constexpr int kFactorPartialK = 32;
+// (hi, lo) halves of a rows x cols block; upper: the block's strict lower triangle as zeros
 int split_tf32(Ctx* c, const float* src, long long lds, int rows, int cols, float* hi, float* lo,
-               long long ldd);
+               long long ldd, bool upper = false);
 int trailing_update(Ctx* c, float* Wk, int m, int d, int i, int k, int c0, int c1,
                     const float* E, int ldE, const float* R);
 int loss_reduce(Ctx* c, const float* loss_part, int parts, int d, float* loss_p);
