@@ -469,8 +469,9 @@ _CS = "post_weight_quantization_17_b200/csrc/"
 STAGE_KERNEL_FILES = {
     "a1_hessian": [_CS + "k_syrk.cu", _CS + "tc_util.cuh"],
     "a3_factor_gemm": [_CS + "k_factor.cu", _CS + "k_gemm_pair.cu", _CS + "k_gemm_tc.cu",
-                       _CS + "gemm_simt.cuh", _CS + "tc_util.cuh"],
-    "a6_update": [_CS + "k_gemm_pair.cu", _CS + "k_gemm_tc.cu", _CS + "tc_util.cuh"],
+                       _CS + "gemm_simt.cuh", _CS + "tc_util.cuh", _CS + "tile_upper.h"],
+    "a6_update": [_CS + "k_gemm_pair.cu", _CS + "k_gemm_tc.cu", _CS + "tc_util.cuh",
+                  _CS + "tile_upper.h"],
 }
 
 

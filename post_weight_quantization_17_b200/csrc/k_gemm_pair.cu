@@ -28,6 +28,7 @@
 #include "kernels.h"
 #include "gemm_simt.cuh"
 #include "tc_util.cuh"
+#include "tile_upper.h"
 
 #include <algorithm>
 
@@ -58,8 +59,14 @@ struct GemmPairParams {
 // Tile t -> (tile row, tile column), in groups of GP_GROUP tile rows walked column by column, so
 // that the 74 tiles of one wave form a near-square block (8 x ~9) and share operand slabs through
 // L2 (row-major order would give each tile of a wave its own B slab).
+// A product computed only where C touches the upper triangle (kCUpper) enumerates just those
+// tiles, in the same grouped order (tile_upper.h).
 constexpr int GP_GROUP = 8;
 __device__ __forceinline__ void gp_tile(const GemmPairParams& p, int t, int& tm, int& tn) {
+  if (p.flags & kCUpper) {
+    upper_tile(p.tiles_m, p.tiles_n, GP_GROUP, t, tm, tn);
+    return;
+  }
   const int group = t / (GP_GROUP * p.tiles_n);
   const int first = group * GP_GROUP;
   const int rows = min(GP_GROUP, p.tiles_m - first);
@@ -491,7 +498,8 @@ int gemm_pair(Ctx* c, const GemmPairArgs& g) {
   p.kbp = g.partial_k > 0 ? std::max(1, g.partial_k / GP_BK) : 4;
   p.tiles_n = (g.N + 255) / 256;
   p.tiles_m = (g.M + 255) / 256;
-  p.num_tiles = p.tiles_n * p.tiles_m;
+  p.num_tiles = (g.flags & kCUpper) ? upper_tiles(p.tiles_m, p.tiles_n, GP_GROUP)
+                                     : p.tiles_n * p.tiles_m;
   p.idesc = tc::idesc_f32acc(2u, false, !g.b_kmajor, 256, 256);
   const int npairs = std::min(p.num_tiles, c->num_sms / 2);
   GPTQ_CUDA_CHECK(c, cudaFuncSetAttribute(k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
