@@ -375,10 +375,11 @@ def cores_used():
 
 
 # ----------------------------------------------------------------------------- oracle leg
-def oracle_instance(W, x_chunks, spec, cols: int, grid: str = "static"):
+def oracle_instance(W, x_chunks, spec, cols: int, grid: str = "static", layer_d: int = 0):
     """The CPU oracle, timed, on a leading block of one layer: the first `cols` input features
     (columns of W and the matching rows of X) with every row of W and every token given.  W is
-    a torch tensor [m, d], x_chunks an iterable of token-major torch chunks [C, d] (any device).
+    a torch tensor [m, d], x_chunks an iterable of token-major torch chunks [C, d] (any device);
+    layer_d: the whole layer's input features, for the description (default spec.d).
     Returns (seconds, weights quantized, description)."""
     import numpy as np
     from oracle import gptq_oracle as O
@@ -407,7 +408,7 @@ def oracle_instance(W, x_chunks, spec, cols: int, grid: str = "static"):
         O.pack(codes, spec.bits)
     dt = time.perf_counter() - t0
     desc = (f"the whole hot path (H over {n} tokens, prepare, lazy-block quantization, pack) on "
-            f"the layer's first {cols} of {spec.d} input features: {m}x{cols} weights, timed "
+            f"the layer's first {cols} of {layer_d or spec.d} input features: {m}x{cols} weights, timed "
             "in full, not extrapolated")
     return dt, m * cols, desc
 
@@ -439,12 +440,12 @@ def run_reference(args):
     W = make_weight(sub, 1, "cpu")
     X = XSource(sub, 1, "cpu").chunk(0)
     for _ in range(args.warmup):
-        oracle_instance(W, [X], sub, cols, args.grid)
+        oracle_instance(W, [X], sub, cols, args.grid, spec.d)
     times = []
     desc, n_w = "", 0
     t_start = time.perf_counter()
     for _ in range(args.steps):
-        dt, n_w, desc = oracle_instance(W, [X], sub, cols, args.grid)
+        dt, n_w, desc = oracle_instance(W, [X], sub, cols, args.grid, spec.d)
         times.append(dt)
     wall = time.perf_counter() - t_start
     per = sum(times) / len(times)
@@ -517,7 +518,7 @@ def stage_rooflines(groups, stage_ms, kern, peaks, tf32):
     if kern:
         k = lambda n: kern.get(n, (0.0, 0))[0]
         tensor("a3_factor_gemm", f_fact, k("factor_gemm"), fp32_peak, tf_src,
-               "kernel events (profiled step); the second stream's GEMMs overlap the first's")
+               "kernel events (profiled step, run on one stream so that no two launches overlap)")
         tensor("a6_update", f_upd, k("update"), fp32_peak, tf_src, "kernel events (profiled step)")
         hbm("a4_grid", b_grid, k("grid"))
         hbm("a5_column", b_col, k("column"))
@@ -642,7 +643,8 @@ def run_ours(args):
     if roofline:
         roofline["stage"] = main_name
         roofline["kernel"] = {"a1_hessian": "k_syrk_tc2 (S += X^T X)",
-                              "a3_factor_gemm": "k_gemm_tc (factorization recursion GEMMs)",
+                              "a3_factor_gemm": "k_gemm_pair + k_gemm_tc + k_gemm_small "
+                                                "(factorization products)",
                               "a6_update": "k_gemm_pair + k_gemm_tc (lazy trailing updates)"}[
             main_name]
         digest = kernel_source_digest(STAGE_KERNEL_FILES[main_name])

@@ -96,15 +96,15 @@ enum {
 
 /* Per-stage kernel timing, for measurement.  on != 0: from now on every kernel this context
  * launches is bracketed by two CUDA events on its stream (which serializes it with its
- * neighbours: programmatic dependent launch no longer overlaps their set-up), and the records
- * kept so far are dropped; on == 0: launches are no longer timed.  Errors: ARG. */
+ * neighbours: programmatic dependent launch no longer overlaps their set-up), the factorization
+ * runs all its launches on the context stream (no second stream, so no two timed launches
+ * overlap), and the records kept so far are dropped; on == 0: launches are no longer timed.
+ * Errors: ARG. */
 int gptq_timing_enable(gptq_ctx* ctx, int on);
 
 /* Synchronizes on the last timed launch and adds up, per stage, the time between each timed
  * launch's two events (ms, host double[GPTQ_NUM_STAGES]) and the number of timed launches (host
- * int64_t[GPTQ_NUM_STAGES]); then drops the records.  Launches on the factorization's second
- * stream overlap those on the first, so the sum of a stage can exceed its elapsed time.
- * Errors: ARG, CUDA. */
+ * int64_t[GPTQ_NUM_STAGES]); then drops the records.  Errors: ARG, CUDA. */
 int gptq_timing_read(gptq_ctx* ctx, double* ms, int64_t* launches);
 
 /* Synchronizes the context stream, returns and clears the device status word

@@ -399,7 +399,9 @@ int factor_inverse(Ctx* c, float* M, int d, float* tmp) {
   f.M = M;
   f.ld = d;
   f.tmp = tmp;
-  f.side = c->side;
+  // with per-stage timing on, T2 runs on the main stream too, so that no two timed launches
+  // overlap and each launch's events measure that kernel alone
+  f.side = c->timing ? c->stream : c->side;
   for (int k = 0; k < 2 * 64; ++k) f.ev[k] = c->ev[k];
   // inside the hot path the factorization has stages of its own; for two-sided rounding's
   // factors it stays under the caller's stage
