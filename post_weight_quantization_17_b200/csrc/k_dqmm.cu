@@ -64,6 +64,11 @@ struct DqCfg {
   static_assert(DQ_NA * DQ_A_COLS + ND * BN <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(3 + DQW + EPW == DQ_THREADS / 32, "warp roles");
+  // the ring starts on a 1024-byte boundary (rounded up at run time) and every codes box, codes
+  // stage and X stage is a whole number of 1024-byte swizzle repeats, so the tiled layout's
+  // pre-applied 128-byte swizzle (chunk ^ (row & 7)) lines up with the hardware's
+  static_assert(DQ_BOX % 1024 == 0 && C_BYTES % 1024 == 0 && X_BYTES % 1024 == 0,
+                "swizzle alignment of the rings");
 };
 
 struct DqParams {
