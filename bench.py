@@ -706,8 +706,8 @@ def run_ours(args):
 
     # end to end through the public API with host buffers (pinned), copies inside the region:
     # X goes up in slabs on a copy stream, double-buffered, each slab's Hessian update running
-    # while the next slab is in flight; W goes up beside it; then prepare, quantize, pack, and the
-    # packed codes with their grid come back to the host
+    # while the next slab is in flight; W goes up behind the slabs; then prepare, quantize, pack,
+    # and the packed codes with their grid come back to the host
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, G, ctx, stream, data, world, W_total)
@@ -777,11 +777,6 @@ def run_e2e(args, G, ctx, stream, data, world, W_total):
             k = 0
             for (g, chunks, Ws, S, R, perm, dead, outs), (X_host, W_host, o_host) in zip(data, host):
                 d = g.x_spec.d
-                for W, Wh in zip(Ws, W_host):
-                    with torch.cuda.stream(copy_stream):
-                        W.copy_(Wh, non_blocking=True)
-                w_landed = torch.cuda.Event()
-                w_landed.record(copy_stream)
                 n_total = 0
                 for xh in X_host:
                     u = k % 2
@@ -796,6 +791,13 @@ def run_e2e(args, G, ctx, stream, data, world, W_total):
                     n_total = G.gptq_hessian_accumulate(ctx, buf, S, n_total)
                     free[u].record(stream)
                     k += 1
+                # W goes up behind the slabs (it is needed only after the factorization), so the
+                # first slab lands as early as it can
+                for W, Wh in zip(Ws, W_host):
+                    with torch.cuda.stream(copy_stream):
+                        W.copy_(Wh, non_blocking=True)
+                w_landed = torch.cuda.Event()
+                w_landed.record(copy_stream)
                 G.gptq_prepare_hinv(ctx, S, n_total, g.x_spec.percdamp, g.x_spec.act_order, R,
                                     perm, dead)
                 stream.wait_event(w_landed)
