@@ -508,6 +508,16 @@ STAGE_KERNEL_FILES = {
 }
 
 
+def peak_regime(clk) -> str:
+    """The regime the timed steps ran in, from the clocks sampled over them: "sustained" when the
+    power cap held the median SM clock below 90 % of its maximum (the kernels then take the
+    sustained peaks: bf16 from the peaks file, TF32 measured the same way), else "burst"."""
+    if clk and clk.get("sm_mhz") and clk.get("sm_max_mhz") and \
+            clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"]:
+        return "sustained"
+    return "burst"
+
+
 def stage_rooflines(groups, stage_ms, kern, peaks, tf32, regime="burst"):
     """Per-stage roofline entries: algorithmic work of the stage (flop or bytes, per step) over
     its time per step, against the peak of the unit that bounds it.  stage_ms: event times of the
@@ -674,15 +684,8 @@ def run_ours(args):
     per_step_s = total_s / args.steps
     value = weak_scaling_value(world, W_total, per_step_s)
 
-    # the peaks' regime follows the clocks sampled over the timed steps: when the power cap held
-    # the SM clock below 90 % of its maximum, the kernels ran in the sustained regime and take
-    # the sustained figures (bf16 from the peaks file, TF32 measured here the same way)
-    regime = "burst"
-    tf32_sus = None
-    if clk and clk.get("sm_mhz") and clk.get("sm_max_mhz") and \
-            clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"]:
-        regime = "sustained"
-        tf32_sus = measure_tf32_sustained(dev)
+    regime = peak_regime(clk)
+    tf32_sus = measure_tf32_sustained(dev) if regime == "sustained" else None
     stages = stage_rooflines(groups, stage_ms, kern, peaks, tf32_sus or tf32, regime)
     # the headline roofline: the stage that takes the longest
     main_name = max((n for n in ("a1_hessian", "a3_factor_gemm", "a6_update") if n in stages),

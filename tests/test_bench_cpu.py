@@ -69,3 +69,25 @@ def test_workload_configs():
     assert bench.weights_per_step(g4) == 4 * 4096 * 4096 + 2 * 11008 * 4096 + 4096 * 11008
     assert all(g.x_spec.chunk == g.x_spec.n_tokens for g in g4)   # one call over all tokens
     assert bench.baseline_cols(49152, 65536) == 2048 and bench.baseline_cols(100, 512) == 100
+
+
+def test_peak_regime_and_stage_peaks():
+    """The roofline peaks follow the regime of the timed steps: sustained when the power cap held
+    the median SM clock below 90 % of its maximum, burst otherwise (or without clock samples)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.peak_regime({"sm_mhz": 1425.0, "sm_max_mhz": 1965.0}) == "sustained"
+    assert bench.peak_regime({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}) == "burst"
+    assert bench.peak_regime({"sm_mhz": 1800.0, "sm_max_mhz": 1965.0}) == "burst"
+    assert bench.peak_regime(None) == "burst"
+    peaks = {"bf16": 1672.7, "bf16_sustained": 1410.6, "hbm": 6544.3, "source": "measured"}
+    g5 = bench.workload(5)
+    st = {"hessian": 140.0, "prepare": 470.0}
+    sus = bench.stage_rooflines(g5, st, None, peaks, 600.0, "sustained")
+    bur = bench.stage_rooflines(g5, st, None, peaks, 750.0, "burst")
+    assert sus["a1_hessian"]["peak"] == 1410.6 and bur["a1_hessian"]["peak"] == 1672.7
+    assert sus["a3_factor"]["peak"] == pytest.approx(200.0)      # TF32 / 3
+    assert bur["a3_factor"]["peak"] == pytest.approx(250.0)
+    f = 158332895625216.0    # N d (d + 1) for the fc2 layer: 65536 x 49152 x 49153
+    assert sus["a1_hessian"]["work"] == f
+    assert sus["a1_hessian"]["achieved"] == pytest.approx(f / 0.140 / 1e12)
